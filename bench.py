@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the SSD chunked-scan forward on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                [--workload NAME] [--path auto|simt|tcgen05]
+
+One step = one pass of the whole forward path (chunk_cumsum, chunk_state,
+state_passing, chunk_scan) over one batch of the workload, inputs resident in
+HBM. The default workload is the Mamba-2-2.7B-shaped layer (batch 4, T 4096,
+80 heads, P 64, N 128, Q 256, bf16 in / fp32 state). Its inputs (~360 MB) are
+larger than L2, so no flush runs between steps. Prints one JSON line on rank 0.
+
+Under torchrun every rank runs the same per-GPU workload (weak scaling: the
+(batch, head) units are independent; no data-path collective), the timed
+region is bracketed by barriers and the time is the max over ranks.
+
+--impl reference times the CPU fp64 oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "SSD fwd tokens·heads/s and TFLOP/s at 2.7B-layer shape; % BF16 tensor peak"
+UNIT = "tokens·heads/s"
+DEFAULT_WORKLOAD = "mamba2_2p7b_layer"
+
+
+# --------------------------------------------------------------------------- #
+# Algorithmic work (the per-unit figures of the design notes)
+# --------------------------------------------------------------------------- #
+
+def algorithmic_flops(w) -> float:
+    """F = b * C_n * [H (Q(Q+1) P + 4 Q N P) + G Q(Q+1) N]: the masked quadratic
+    term and C B^T on the lower triangle, the chunk state and the state read-out."""
+    cn = w.seqlen // w.chunk
+    Q, N, P = w.chunk, w.dstate, w.headdim
+    return w.batch * cn * (w.nheads * (Q * (Q + 1) * P + 4 * Q * N * P) + w.ngroups * Q * (Q + 1) * N)
+
+
+def _esize(w):
+    return 2 if w.dtype == "bf16" else 4
+
+
+def algorithmic_bytes(w) -> float:
+    """Minimum I/O of the forward: X, Y, B, C, log a, D, seq_idx, init and final states."""
+    e = _esize(w)
+    b, T, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    by = 2 * b * T * H * P * e + 2 * b * T * G * N * e + b * T * H * 4
+    if w.has_D != "none":
+        by += H * 4
+    if w.varlen != "none":
+        by += b * T * 4
+    nseq = w.nseq if w.varlen != "none" else 1
+    if w.has_init:
+        by += b * nseq * H * N * P * 4
+    by += b * nseq * H * N * P * 4  # final states are returned
+    return by
+
+
+def kernel_model(w):
+    """Algorithmic bytes and flops per launch of each kernel of the unfused path.
+
+    chunk_cumsum  reads log a, writes cs.
+    chunk_state   reads X, B, cs; writes one fp32 state per (b, chunk, h);
+                  flops 2 Q N P per (b, chunk, h).
+    state_passing reads the states and cs, writes the incoming states
+                  (in place) and the final states; 2 N P flops per (b, chunk, h).
+    chunk_scan    reads X, B, C, cs, D and the incoming states; writes Y;
+                  flops Q(Q+1)P + 2QNP per (b, chunk, h) + Q(Q+1)N per (b, chunk, g).
+    """
+    e = _esize(w)
+    b, T, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
+    cn = T // Q
+    st = b * cn * H * N * P * 4
+    xb = b * T * H * P * e
+    bcb = b * T * G * N * e
+    csb = b * T * H * 4
+    nseq = w.nseq if w.varlen != "none" else 1
+    fin = b * nseq * H * N * P * 4
+    return {
+        "chunk_cumsum": dict(bytes=2 * csb, flops=b * T * H),
+        "chunk_state": dict(bytes=xb + bcb + csb + st, flops=b * cn * H * 2 * Q * N * P),
+        "state_passing": dict(bytes=2 * st + csb / Q + fin, flops=b * cn * H * 2 * N * P),
+        "chunk_scan": dict(bytes=2 * xb + 2 * bcb + csb + st,
+                           flops=b * cn * (H * (Q * (Q + 1) * P + 2 * Q * N * P) + G * Q * (Q + 1) * N)),
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm_gbs=float(pk["hbm_gbs"]), bf16_tflops=float(pk["bf16_tflops"]),
+                    bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# --------------------------------------------------------------------------- #
+# Clock sampling during the timed region
+# --------------------------------------------------------------------------- #
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# Distributed helpers (also exercised by the CPU gloo tests)
+# --------------------------------------------------------------------------- #
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max over ranks of a scalar (a control-plane reduction, not a data path)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized():
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(units_per_rank: float, seconds_per_rank: float, device=None):
+    """Whole-job throughput: units of all ranks / the slowest rank's time."""
+    import torch.distributed as dist
+    ws = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
+    t = reduce_max(seconds_per_rank, device)
+    return units_per_rank * ws / t, t
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle leg
+# --------------------------------------------------------------------------- #
+
+def oracle_sample(w, inputs, budget_s: float = 12.0):
+    """Time the oracle on whole (batch row, head) pairs of the workload, one
+    batch row and `cores` heads per call, until about budget_s seconds of CPU
+    work or the whole workload; return (token·heads/s, cores, sample, seconds)."""
+    import oracle
+    cores = max(1, oracle.max_threads())
+    done, t_total = 0, 0.0
+    for b in range(w.batch):
+        for h0 in range(0, w.nheads, cores):
+            if t_total >= budget_s:
+                break
+            hs = slice(h0, min(w.nheads, h0 + cores))
+            X = inputs["X"][b:b + 1, :, hs]
+            la = inputs["log_a"][b:b + 1, :, hs]
+            D = None if inputs["D"] is None else inputs["D"][hs]
+            init = None if inputs["init_states"] is None else inputs["init_states"][b:b + 1, :, hs]
+            seq = None if inputs["seq_idx"] is None else inputs["seq_idx"][b:b + 1]
+            if w.ngroups != 1:
+                raise NotImplementedError("oracle sampling assumes one group")
+            t0 = time.perf_counter()
+            oracle.ssd_reference(X, la, inputs["B"][b:b + 1], inputs["C"][b:b + 1], D, init, seq,
+                                 nseq=inputs["nseq"], nthreads=cores)
+            t_total += time.perf_counter() - t0
+            done += X.shape[2]
+    return done * w.seqlen / t_total, cores, f"{done} (batch row, head) pairs x {w.seqlen} tokens of {w.name}", t_total
+
+
+# --------------------------------------------------------------------------- #
+# Reference arm: the oracle as the timed CPU program
+# --------------------------------------------------------------------------- #
+
+def run_reference(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    inputs = make_inputs(w)
+    import oracle
+    cores = oracle.max_threads()
+    hs = list(range(min(w.nheads, max(1, cores))))
+    X = inputs["X"][:1, :, hs]
+    la = inputs["log_a"][:1, :, hs]
+    D = None if inputs["D"] is None else inputs["D"][hs]
+    init = None if inputs["init_states"] is None else inputs["init_states"][:1, :, hs]
+    seq = None if inputs["seq_idx"] is None else inputs["seq_idx"][:1]
+    step = lambda: oracle.ssd_reference(X, la, inputs["B"][:1], inputs["C"][:1], D, init, seq,
+                                        nseq=inputs["nseq"], nthreads=cores)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    units = len(hs) * w.seqlen
+    value = units * args.steps / dt
+    sample = f"1 batch row x {len(hs)} heads x {w.seqlen} tokens of {w.name} per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, args):
+    nseq = w.nseq if w.varlen != "none" else 1
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "nheads": w.nheads, "headdim": w.headdim,
+            "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk, "nseq": nseq,
+            "parallelism": f"dp{args.gpus}" if args.gpus > 1 else "single",
+            "l2": "inputs larger than L2, no flush" if algorithmic_bytes(w) > 126e6 else "L2 flushed between steps"}
+
+
+# --------------------------------------------------------------------------- #
+# Our arm
+# --------------------------------------------------------------------------- #
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    ws, rank, local = dist_env()
+    if args.gpus > 1 and ws != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={ws}: launch with torchrun")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import mamba_ssd_layer_chunked_b200 as ssd
+
+    inputs = make_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def dev_t(a, dt=torch.float32):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dt).to(dev)
+
+    X, la, B, C = dev_t(inputs["X"], tdt), dev_t(inputs["log_a"]), dev_t(inputs["B"], tdt), dev_t(inputs["C"], tdt)
+    D, init = dev_t(inputs["D"]), dev_t(inputs["init_states"])
+    seq = None if inputs["seq_idx"] is None else torch.from_numpy(inputs["seq_idx"]).to(dev)
+    nseq = inputs["nseq"] if seq is not None else None
+    p = ssd.problem_from(X, B, w.chunk, inputs["nseq"], args.path)
+    Y = torch.empty_like(X)
+    b, T, H, P = X.shape
+    N = B.shape[3]
+    F = torch.empty((b, inputs["nseq"], H, N, P), dtype=torch.float32, device=dev)
+    wsp = torch.empty(ssd.workspace_bytes(p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssd.ssd_fwd(X, la, B, C, w.chunk, D=D, init_states=init, seq_idx=seq, nseq=nseq, path=args.path,
+                    out=Y, final_out=F, workspace=wsp)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clocks = ClockSampler(local) if rank == 0 and not args.no_clocks else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    barrier()
+    t_dev = ev0.elapsed_time(ev1) / 1e3
+    units = w.tokens_heads * args.steps
+    value, t_max = aggregate(units, t_dev, dev if ws > 1 else None)
+    ms_per_step = t_max / args.steps * 1e3
+
+    # per-kernel durations: the same four steps through the step entry points,
+    # with events between them on the launching stream
+    names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
+    lib = ssd.lib()
+    import ctypes
+    nc = T // w.chunk
+    cs = wsp[: b * T * H * 4].view(torch.float32)
+    off = (b * T * H * 4 + 255) // 256 * 256
+    states = wsp[off: off + b * nc * H * N * P * 4].view(torch.float32)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    vp = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    pr = ctypes.byref(p)
+    launches = [
+        lambda: lib.ssd_chunk_cumsum(pr, vp(la), vp(cs), sp),
+        lambda: lib.ssd_chunk_state(pr, vp(X), vp(B), vp(cs), vp(seq), vp(states), vp(F), sp),
+        lambda: lib.ssd_state_passing(pr, vp(cs), vp(states), vp(states), vp(init), vp(seq), vp(F), sp),
+        lambda: lib.ssd_chunk_scan(pr, vp(X), vp(B), vp(C), vp(cs), vp(D), vp(states), vp(init), vp(seq), vp(Y), sp),
+    ]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        for j, fn in enumerate(launches):
+            rc = fn()
+            if rc != 0:
+                raise RuntimeError(f"{names[j]} failed: {ssd.status_string(rc)}")
+            evs[i][j + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    per_kernel = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)) / 1e3
+                  for j, n in enumerate(names)}
+    clk = clocks.stop() if clocks else None
+
+    # end to end through the public call on pinned HOST buffers
+    host = dict(X=X.cpu().pin_memory(), la=la.cpu().pin_memory(), B=B.cpu().pin_memory(), C=C.cpu().pin_memory(),
+                D=None if D is None else D.cpu().pin_memory(),
+                init=None if init is None else init.cpu().pin_memory(),
+                seq=None if seq is None else seq.cpu().pin_memory())
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = Y.numel() * Y.element_size() + F.numel() * F.element_size()
+    Yh = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
+    Fh = torch.empty(F.shape, dtype=F.dtype, pin_memory=True)
+
+    def e2e_step():
+        Xd, lad, Bd, Cd = (host[k].to(dev, non_blocking=True) for k in ("X", "la", "B", "C"))
+        Dd = None if host["D"] is None else host["D"].to(dev, non_blocking=True)
+        initd = None if host["init"] is None else host["init"].to(dev, non_blocking=True)
+        seqd = None if host["seq"] is None else host["seq"].to(dev, non_blocking=True)
+        ssd.ssd_fwd(Xd, lad, Bd, Cd, w.chunk, D=Dd, init_states=initd, seq_idx=seqd, nseq=nseq, path=args.path,
+                    out=Y, final_out=F, workspace=wsp)
+        Yh.copy_(Y, non_blocking=True)
+        Fh.copy_(F, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_value, _ = aggregate(units, e0.elapsed_time(e1) / 1e3, dev if ws > 1 else None)
+
+    # roofline of the dominant kernel
+    model = kernel_model(w)
+    dom = max(per_kernel, key=per_kernel.get)
+    peaks = load_peaks()
+    km = model[dom]
+    ai = km["flops"] / km["bytes"]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if ai < ridge:
+        achieved = km["bytes"] / per_kernel[dom] / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = km["flops"] / per_kernel[dom] / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = peaks["source"]
+
+    step_s = t_max / args.steps
+    flops = algorithmic_flops(w)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, args),
+        "tflops": flops * ws / step_s / 1e12,
+        "pct_bf16_peak": flops / step_s / 1e12 / peaks["bf16_tflops"],
+        "pct_hbm": algorithmic_bytes(w) / step_s / 1e9 / peaks["hbm_gbs"],
+        "path": "tcgen05" if ssd.path_supported(p, "tcgen05") and args.path != "simt" else "simt",
+        "per_kernel_us": {k: v * 1e6 for k, v in per_kernel.items()},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        v, cores, sample, secs = oracle_sample(w, inputs, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                                  "seconds": secs}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if ws > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

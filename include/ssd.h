@@ -1,0 +1,192 @@
+/*
+ * ssd.h -- C ABI of the B200 (sm_100a) SSD chunked-scan forward library
+ * (libssd_b200.so).
+ *
+ * The operation is the Mamba-2 SSD layer (A, X, B, C) -> Y for a scalar decay
+ * per head. For every batch row b and head h, with group g = h / (nheads/ngroups):
+ *
+ *   H_t = a_t H_{t-1} + B_t x_t^T,   y_t = C_t^T H_t + D_h x_t,   a_t = exp(log_a_t)
+ *
+ * with H_t in R^{dstate x headdim}. Source: "Mamba-2: writing the recurrent state
+ * as a structured matrix" (wq-win.github.io/llm/088-mamba2.html), section 2.1
+ * (recurrence and unrolled sum) and section 2.2 (dual form Y = [L o (C B^T)] X,
+ * L_ts = prod_{j=s+1..t} a_j); the D x skip term is the discrete state space form
+ * of "Mamba and state space models" (wang-x-xia.github.io), section 2.
+ *
+ * The library computes it with the block decomposition of the same page,
+ * section 3 ("Mamba-2 - Transformer and SSM share one algebra",
+ * awesome.papernotes.org, design 2, gives the same four steps): within-chunk
+ * cumulative sum of log a (chunk_cumsum), per-chunk end states with a zero
+ * incoming state (chunk_state), a short scan of the states over chunks
+ * (state_passing), and the per-chunk output = masked quadratic term plus the
+ * incoming state decayed to each position and read out by C (chunk_scan).
+ *
+ * Conventions (all entry points):
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates, frees or synchronises, never exits or aborts, and keeps no
+ *    mutable global state besides a per-device cache of kernel attributes that
+ *    is set once. Every call is asynchronous on `stream` (a cudaStream_t passed
+ *    as void*; NULL means the legacy default stream) and is thread-safe.
+ *  - Layouts are dense row-major (C order) with the last dimension contiguous.
+ *    Every pointer must be 16-byte aligned.
+ *  - Arguments are validated on the host before anything is launched; on an
+ *    error status nothing has been enqueued. SSD_ERR_CUDA reports a launch
+ *    error (the message of cudaGetLastError is available from
+ *    ssd_last_cuda_error_string on the calling thread).
+ *  - seq_idx is device memory and is never read on the host. In-contract values
+ *    are: seq_idx[b, 0] = 0, non-decreasing along t, steps of 0 or 1, and every
+ *    value < nseq. A change between t-1 and t starts an independent sequence:
+ *    its state starts from init_states[b, seq_idx[b, t]] (or zero) and the
+ *    finished sequence's state becomes its final state (the pages require that
+ *    only independent-sample boundaries stop state propagation: section 2.3 and
+ *    the section 5 testing advice of the wq-win page). Out-of-contract values
+ *    give unspecified results but never out-of-bounds accesses (kernels clamp
+ *    ids to [0, nseq)).
+ *  - init_states is the state before the first token of each sequence (H_{-1}):
+ *    the first a_t decays it (the chunk-split example of the wq-win page,
+ *    section 2.3, decays the carried state 5 by 0.5).
+ *  - final_states[b, s] is the state after the last token of sequence s; ids
+ *    in (seq_idx[b, seqlen-1], nseq) that never occur keep their initial state
+ *    (or zero).
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,  /* null required pointer, bad dims, misaligned pointer */
+    SSD_ERR_UNSUPPORTED = 2,  /* valid problem this build or device cannot run */
+    SSD_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+    SSD_ERR_CUDA = 4          /* a CUDA call or kernel launch failed */
+} ssd_status;
+
+typedef enum {
+    SSD_DTYPE_F32 = 0,   /* X, B, C, Y in fp32 */
+    SSD_DTYPE_BF16 = 1   /* X, B, C, Y in bfloat16 */
+} ssd_dtype;
+
+/* Kernel family. AUTO picks the tensor-core (tcgen05) kernels when the problem
+ * is in their domain (see ssd_path_supported) and the SIMT fp32 kernels
+ * otherwise. SIMT and TCGEN05 force one family (TCGEN05 returns
+ * SSD_ERR_UNSUPPORTED outside its domain). */
+typedef enum {
+    SSD_PATH_AUTO = 0,
+    SSD_PATH_SIMT = 1,
+    SSD_PATH_TCGEN05 = 2
+} ssd_path;
+
+typedef struct {
+    int64_t batch;     /* b  >= 1 */
+    int64_t seqlen;    /* T  >= 1, a multiple of chunk */
+    int64_t nheads;    /* H  >= 1, a multiple of ngroups */
+    int64_t headdim;   /* P: multiple of 16, <= 256 */
+    int64_t dstate;    /* N: multiple of 16, <= 256 */
+    int64_t ngroups;   /* G: heads h*G/H .. share B, C group g */
+    int64_t chunk;     /* Q: 64, 128 or 256 */
+    int64_t nseq;      /* sequences per batch row: 1 when seq_idx is NULL */
+    ssd_dtype dtype;   /* dtype of X, B, C and Y; log_a, D and states are fp32 */
+    ssd_path path;
+} ssd_problem;
+
+/* Status text, static storage. */
+const char* ssd_status_string(ssd_status s);
+
+/* Text of the last CUDA error seen by an entry point on the calling thread
+ * ("" if none). */
+const char* ssd_last_cuda_error_string(void);
+
+/* Host-side validation of a problem (no device access besides querying the
+ * current device's compute capability). */
+ssd_status ssd_check_problem(const ssd_problem* p);
+
+/* 1 if `path` (SIMT or TCGEN05) can run problem p on the current device. */
+int ssd_path_supported(const ssd_problem* p, ssd_path path);
+
+/* Bytes of workspace ssd_fwd needs, or (size_t)-1 if p is invalid. The
+ * workspace holds the chunk cumulative sums (batch*seqlen*nheads fp32) and one
+ * state per chunk (batch*nchunks*nheads*dstate*headdim fp32), each 256-byte
+ * aligned. */
+size_t ssd_fwd_workspace_bytes(const ssd_problem* p);
+
+/*
+ * ssd_fwd: the whole forward pass, Y and final states from X, log a, B, C.
+ *   X            [batch, seqlen, nheads, headdim]            dtype, required
+ *   log_a        [batch, seqlen, nheads]                     fp32, required; finite,
+ *                                                            <= 0 is the tested domain
+ *   B, C         [batch, seqlen, ngroups, dstate]            dtype, required
+ *   D            [nheads]                                    fp32 or NULL (= 0)
+ *   init_states  [batch, nseq, nheads, dstate, headdim]      fp32 or NULL (= 0)
+ *   seq_idx      [batch, seqlen]                             int32 or NULL (one sequence)
+ *   Y            [batch, seqlen, nheads, headdim]            dtype, out, required
+ *   final_states [batch, nseq, nheads, dstate, headdim]      fp32, out, or NULL
+ *   workspace    >= ssd_fwd_workspace_bytes(p) bytes of device memory (its
+ *                contents on entry are ignored; on exit they are unspecified)
+ * Y is rounded to nearest even from the fp32 result when dtype is bf16.
+ */
+ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, const void* B,
+                   const void* C, const float* D, const float* init_states,
+                   const int32_t* seq_idx, void* Y, float* final_states, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* ---- the four steps, callable one by one (ssd_fwd runs them in this order) ----
+ * nchunks = seqlen / chunk. cs is [batch, nheads, nchunks, chunk] fp32; a "state
+ * buffer" is [batch, nchunks, nheads, dstate, headdim] fp32. */
+
+/* Bytes of one state buffer. */
+size_t ssd_states_bytes(const ssd_problem* p);
+
+/* Step 1, chunk_cumsum: cs[b, h, c, k] = sum_{j <= k} log_a[b, c*chunk + j, h],
+ * the within-chunk inclusive cumulative sum; exp(cs[k] - cs[l]) is the decay
+ * prod_{j=l+1..k} a_j of the segment mask L (papernotes design 2, "A_cumsum"
+ * and "L = exp(segment_sum(A))"). */
+ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs, void* stream);
+
+/* Step 2, chunk_state: per chunk c, the end state of the chunk's LAST sequence
+ * piece with a zero incoming state,
+ *   states[b, c, h] = sum_{l in last piece} exp(cs[Q-1] - cs[l]) B_l x_l^T
+ * (wq-win section 3 "local_end_state"; papernotes design 2 right factors).
+ * When seq_idx and final_states are both non-NULL, it also writes, for every
+ * sequence s that ends strictly inside chunk c at token e, the zero-start partial
+ * sum_{l in s's piece of c, l <= e} exp(cs[e] - cs[l]) B_l x_l^T into
+ * final_states[b, s]; ssd_state_passing completes those entries. */
+ssd_status ssd_chunk_state(const ssd_problem* p, const void* X, const void* B, const float* cs,
+                           const int32_t* seq_idx, float* states, float* final_states,
+                           void* stream);
+
+/* Step 3, state_passing: the short recurrence over chunks
+ *   H_c = exp(cs_c[Q-1] - cs_c[st-1]) H_start + S_c
+ * (wq-win section 3 "real_end_state = block_decay * previous_state +
+ * local_end_state"; st is the start of the chunk's last piece, cs[-1] = 0,
+ * H_start is the carried state or, after a boundary, the new sequence's initial
+ * state). Reads the chunk states from `chunk_states` and writes the INCOMING
+ * state of every chunk (the state before its first token, for that token's
+ * sequence) to `incoming`; the two may be the same buffer (in place). Writes
+ * final_states when non-NULL (completing the partials of ssd_chunk_state). */
+ssd_status ssd_state_passing(const ssd_problem* p, const float* cs, const float* chunk_states,
+                             float* incoming, const float* init_states, const int32_t* seq_idx,
+                             float* final_states, void* stream);
+
+/* Step 4, chunk_scan: per chunk,
+ *   y_k = sum_{l <= k, same sequence} exp(cs[k] - cs[l]) (C_k . B_l) x_l
+ *       + exp(cs[k] - cs[st_k - 1]) C_k^T H_start(k) + D_h x_k
+ * (wq-win section 3: local_output = (L o C B^T) X plus the incoming state decayed
+ * to each position and read out by C; H_start(k) is `incoming[b, c, h]` for the
+ * chunk's first sequence and init_states (or zero) for a sequence starting at
+ * st_k inside the chunk). */
+ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, const void* C,
+                          const float* cs, const float* D, const float* incoming,
+                          const float* init_states, const int32_t* seq_idx, void* Y,
+                          void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_H */

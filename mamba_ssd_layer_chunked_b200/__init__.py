@@ -1,0 +1,32 @@
+"""B200 (sm_100a) SSD chunked-scan forward: a C-ABI CUDA library
+(libssd_b200.so, include/ssd.h) and its thin Python binding.
+
+    from mamba_ssd_layer_chunked_b200 import ssd_fwd
+    Y, final_states = ssd_fwd(X, log_a, B, C, chunk=256, D=D, init_states=h0,
+                              seq_idx=seq_idx, nseq=nseq)
+
+Importing the package loads the library and raises ImportError when it has
+not been built (``python -m mamba_ssd_layer_chunked_b200.build``): there is no
+fallback implementation.
+"""
+from .ssd import (  # noqa: F401
+    LIB_PATH,
+    Problem,
+    SSDError,
+    chunk_cumsum,
+    chunk_scan,
+    chunk_state,
+    declared_functions,
+    lib,
+    make_problem,
+    path_supported,
+    problem_from,
+    ssd_fwd,
+    ssd_fwd_host,
+    state_passing,
+    states_bytes,
+    status_string,
+    workspace_bytes,
+)
+
+lib()  # fail loudly at import when the CUDA library is missing

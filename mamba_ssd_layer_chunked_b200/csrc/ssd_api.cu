@@ -1,0 +1,234 @@
+// ssd_api.cu -- host side of the C ABI declared in include/ssd.h: argument
+// validation, workspace sizing, kernel-family selection and the launch
+// sequence chunk_cumsum -> chunk_state -> state_passing -> chunk_scan on the
+// caller's stream. Nothing here allocates, synchronises or reads device memory.
+
+#include <cstdio>
+#include <cstring>
+
+#include "ssd_common.cuh"
+#include "ssd_tc.cuh"
+
+namespace {
+
+thread_local char g_cuda_err[256] = "";
+
+ssd_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return SSD_OK;
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return SSD_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host-only checks of the problem description (no device access).
+ssd_status check_dims(const ssd_problem* p) {
+    if (!p) return SSD_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->seqlen < 1 || p->nheads < 1 || p->headdim < 1 || p->dstate < 1 ||
+        p->ngroups < 1 || p->chunk < 1 || p->nseq < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (p->nheads % p->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (p->dtype != SSD_DTYPE_F32 && p->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (p->path != SSD_PATH_AUTO && p->path != SSD_PATH_SIMT && p->path != SSD_PATH_TCGEN05)
+        return SSD_ERR_INVALID_ARG;
+    if (p->chunk != 64 && p->chunk != 128 && p->chunk != 256) return SSD_ERR_UNSUPPORTED;
+    if (p->seqlen % p->chunk != 0) return SSD_ERR_UNSUPPORTED;
+    if (p->headdim % 16 != 0 || p->headdim > 256 || p->dstate % 16 != 0 || p->dstate > 256)
+        return SSD_ERR_UNSUPPORTED;
+    // grid and index limits: every flattened grid dimension stays below 2^31
+    const int64_t nchunks = p->seqlen / p->chunk;
+    if (p->batch > (1 << 20) || p->seqlen > (1 << 26) || p->nheads > (1 << 16) || p->nseq > (1 << 24))
+        return SSD_ERR_UNSUPPORTED;
+    if (p->batch * p->nheads * nchunks * 4 > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+    if (p->batch * p->seqlen > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+// The build targets sm_100a only: the device must be compute capability 10.0.
+ssd_status check_device() {
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SSD_ERR_UNSUPPORTED;
+    }
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SSD_ERR_UNSUPPORTED;
+    }
+    return (major == 10 && minor == 0) ? SSD_OK : SSD_ERR_UNSUPPORTED;
+}
+
+ssd::Dims make_dims(const ssd_problem* p) {
+    ssd::Dims d;
+    d.batch = (int)p->batch;
+    d.seqlen = (int)p->seqlen;
+    d.nheads = (int)p->nheads;
+    d.headdim = (int)p->headdim;
+    d.dstate = (int)p->dstate;
+    d.ngroups = (int)p->ngroups;
+    d.chunk = (int)p->chunk;
+    d.nseq = (int)p->nseq;
+    d.nchunks = (int)(p->seqlen / p->chunk);
+    d.heads_per_group = (int)(p->nheads / p->ngroups);
+    return d;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t cs_bytes(const ssd_problem* p) { return (size_t)p->batch * p->seqlen * p->nheads * sizeof(float); }
+
+size_t states_bytes(const ssd_problem* p) {
+    return (size_t)p->batch * (p->seqlen / p->chunk) * p->nheads * p->dstate * p->headdim * sizeof(float);
+}
+
+bool use_tc(const ssd_problem* p) {
+    if (p->path == SSD_PATH_SIMT) return false;
+    return ssd::tc_supported(p);
+}
+
+ssd_status check_common(const ssd_problem* p, const int32_t* seq_idx) {
+    ssd_status s = check_dims(p);
+    if (s != SSD_OK) return s;
+    if (!seq_idx && p->nseq != 1) return SSD_ERR_INVALID_ARG;
+    return SSD_OK;
+}
+
+// Device-dependent checks, run after every host-side argument check.
+ssd_status check_runnable(const ssd_problem* p) {
+    ssd_status s = check_device();
+    if (s != SSD_OK) return s;
+    if (p->path == SSD_PATH_TCGEN05 && !ssd::tc_supported(p)) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+template <typename... Ptrs>
+bool all_aligned(Ptrs... ps) {
+    const void* arr[] = {static_cast<const void*>(ps)...};
+    for (const void* q : arr)
+        if (q && !aligned16(q)) return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(ssd_status s) {
+    switch (s) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_INVALID_ARG: return "invalid argument";
+        case SSD_ERR_UNSUPPORTED: return "unsupported problem or device";
+        case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSD_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char* ssd_last_cuda_error_string(void) { return g_cuda_err; }
+
+ssd_status ssd_check_problem(const ssd_problem* p) {
+    ssd_status s = check_dims(p);
+    if (s != SSD_OK) return s;
+    if ((s = check_device()) != SSD_OK) return s;
+    if (p->path == SSD_PATH_TCGEN05 && !ssd::tc_supported(p)) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+int ssd_path_supported(const ssd_problem* p, ssd_path path) {
+    if (check_dims(p) != SSD_OK || check_device() != SSD_OK) return 0;
+    if (path == SSD_PATH_SIMT) return 1;
+    if (path == SSD_PATH_TCGEN05) return ssd::tc_supported(p) ? 1 : 0;
+    return 0;
+}
+
+size_t ssd_states_bytes(const ssd_problem* p) {
+    if (check_dims(p) != SSD_OK) return (size_t)-1;
+    return states_bytes(p);
+}
+
+size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
+    if (check_dims(p) != SSD_OK) return (size_t)-1;
+    return align256(cs_bytes(p)) + align256(states_bytes(p));
+}
+
+ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs, void* stream) {
+    ssd_status s = check_dims(p);  // log a only: nseq and seq_idx play no part here
+    if (s != SSD_OK) return s;
+    if (!log_a || !cs) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(log_a, cs)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_device()) != SSD_OK) return s;
+    return cuda_status(ssd::launch_chunk_cumsum(make_dims(p), log_a, cs, (cudaStream_t)stream));
+}
+
+ssd_status ssd_chunk_state(const ssd_problem* p, const void* X, const void* B, const float* cs,
+                           const int32_t* seq_idx, float* states, float* final_states, void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!X || !B || !cs || !states) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, B, cs, seq_idx, states, final_states)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_runnable(p)) != SSD_OK) return s;
+    const ssd::Dims d = make_dims(p);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (use_tc(p)) return cuda_status(ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, final_states, st));
+    return cuda_status(ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st));
+}
+
+ssd_status ssd_state_passing(const ssd_problem* p, const float* cs, const float* chunk_states, float* incoming,
+                             const float* init_states, const int32_t* seq_idx, float* final_states,
+                             void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!cs || !chunk_states || !incoming) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(cs, chunk_states, incoming, init_states, seq_idx, final_states)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_runnable(p)) != SSD_OK) return s;
+    return cuda_status(ssd::launch_state_passing(make_dims(p), cs, chunk_states, incoming, init_states, seq_idx,
+                                                 final_states, (cudaStream_t)stream));
+}
+
+ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, const void* C, const float* cs,
+                          const float* D, const float* incoming, const float* init_states,
+                          const int32_t* seq_idx, void* Y, void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!X || !B || !C || !cs || !incoming || !Y) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, B, C, cs, D, incoming, init_states, seq_idx, Y)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_runnable(p)) != SSD_OK) return s;
+    const ssd::Dims d = make_dims(p);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (use_tc(p))
+        return cuda_status(ssd::launch_chunk_scan_tc(d, X, B, C, cs, D, incoming, init_states, seq_idx, Y, st));
+    return cuda_status(
+        ssd::launch_chunk_scan_simt(d, p->dtype, X, B, C, cs, D, incoming, init_states, seq_idx, Y, st));
+}
+
+ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, const void* B, const void* C,
+                   const float* D, const float* init_states, const int32_t* seq_idx, void* Y,
+                   float* final_states, void* workspace, size_t workspace_bytes, void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, log_a, B, C, D, init_states, seq_idx, Y, final_states, workspace))
+        return SSD_ERR_INVALID_ARG;
+    const size_t need = ssd_fwd_workspace_bytes(p);
+    if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
+    if ((s = check_runnable(p)) != SSD_OK) return s;
+    const ssd::Dims d = make_dims(p);
+    cudaStream_t st = (cudaStream_t)stream;
+    float* cs = static_cast<float*>(workspace);
+    float* states = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(cs_bytes(p)));
+    cudaError_t e = ssd::launch_chunk_cumsum(d, log_a, cs, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    const bool tc = use_tc(p);
+    e = tc ? ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, final_states, st)
+           : ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    // in place: the chunk states become the incoming states
+    e = ssd::launch_state_passing(d, cs, states, states, init_states, seq_idx, final_states, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = tc ? ssd::launch_chunk_scan_tc(d, X, B, C, cs, D, states, init_states, seq_idx, Y, st)
+           : ssd::launch_chunk_scan_simt(d, p->dtype, X, B, C, cs, D, states, init_states, seq_idx, Y, st);
+    return cuda_status(e);
+}
+
+}  // extern "C"

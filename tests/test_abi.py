@@ -1,0 +1,125 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/ssd.h declares, and rejects bad arguments on the host before any
+launch. Calls here use fake device addresses only where a host check is sure to
+reject the call first, so the tests are also safe on a GPU machine."""
+import ctypes
+
+import pytest
+
+import mamba_ssd_layer_chunked_b200 as ssd
+from mamba_ssd_layer_chunked_b200 import ssd as _ssd
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA = range(5)
+FAKE = 0x10000  # 16-byte aligned fake device address (never dereferenced here)
+
+
+def prob(**kw):
+    base = dict(batch=2, seqlen=512, nheads=4, headdim=64, dstate=128, ngroups=1, chunk=256, nseq=1,
+                dtype=ssd.ssd.SSD_DTYPE_BF16, path=0)
+    base.update(kw)
+    return ssd.Problem(**base)
+
+
+def test_library_exports_every_declared_function():
+    names = ssd.declared_functions()
+    assert "ssd_fwd" in names and "ssd_fwd_workspace_bytes" in names
+    lib = ssd.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) >= {"ssd_status_string", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
+                          "ssd_chunk_scan", "ssd_check_problem", "ssd_path_supported", "ssd_states_bytes",
+                          "ssd_last_cuda_error_string"}
+
+
+def test_problem_struct_layout():
+    assert ctypes.sizeof(ssd.Problem) == 8 * 8 + 2 * 4
+
+
+def test_status_strings():
+    for s, text in [(OK, "ok"), (INVALID, "invalid argument"), (WORKSPACE, "workspace missing or too small")]:
+        assert ssd.status_string(s) == text
+    assert ssd.status_string(99) == "unknown status"
+
+
+def test_workspace_bytes_formula():
+    p = prob()
+    cs = 2 * 512 * 4 * 4
+    st = 2 * (512 // 256) * 4 * 128 * 64 * 4
+    align = lambda x: (x + 255) // 256 * 256
+    assert ssd.workspace_bytes(p) == align(cs) + align(st)
+    assert ssd.states_bytes(p) == st
+
+
+@pytest.mark.parametrize("field,value,expect", [
+    ("batch", 0, INVALID), ("seqlen", 0, INVALID), ("nheads", 0, INVALID), ("headdim", -1, INVALID),
+    ("dstate", 0, INVALID), ("ngroups", 3, INVALID), ("nseq", 0, INVALID), ("dtype", 7, INVALID),
+    ("path", 9, INVALID), ("chunk", 100, UNSUPPORTED), ("seqlen", 500, UNSUPPORTED),
+    ("headdim", 24, UNSUPPORTED), ("dstate", 512, UNSUPPORTED)])
+def test_bad_problem_rejected(field, value, expect):
+    p = prob(**{field: value})
+    lib = ssd.lib()
+    assert lib.ssd_fwd_workspace_bytes(ctypes.byref(p)) == ctypes.c_size_t(-1).value
+    assert lib.ssd_check_problem(ctypes.byref(p)) == expect
+    assert lib.ssd_fwd(ctypes.byref(p), *([FAKE] * 9), FAKE, 1 << 30, None) == expect
+
+
+def test_null_problem_rejected():
+    lib = ssd.lib()
+    assert lib.ssd_check_problem(None) == INVALID
+    assert lib.ssd_fwd(None, *([FAKE] * 9), FAKE, 1 << 30, None) == INVALID
+
+
+def _fwd(p, X=FAKE, la=FAKE, B=FAKE, C=FAKE, D=None, init=None, seq=None, Y=FAKE, fin=None, ws=FAKE,
+         wsb=1 << 30):
+    return ssd.lib().ssd_fwd(ctypes.byref(p), X, la, B, C, D, init, seq, Y, fin, ws, wsb, None)
+
+
+@pytest.mark.parametrize("arg", ["X", "la", "B", "C", "Y"])
+def test_null_required_pointer(arg):
+    assert _fwd(prob(), **{arg: None}) == INVALID
+
+
+@pytest.mark.parametrize("arg", ["X", "la", "B", "C", "D", "init", "seq", "Y", "fin", "ws"])
+def test_misaligned_pointer(arg):
+    p = prob(nseq=2) if arg == "seq" else prob()
+    kw = {arg: FAKE + 4}
+    if arg == "seq":
+        kw = {"seq": FAKE + 4}
+    assert _fwd(p, **kw) == INVALID
+
+
+def test_nseq_needs_seq_idx():
+    assert _fwd(prob(nseq=3)) == INVALID
+
+
+def test_workspace_checks():
+    p = prob()
+    need = ssd.workspace_bytes(p)
+    assert _fwd(p, ws=None) == WORKSPACE
+    assert _fwd(p, wsb=need - 1) == WORKSPACE
+
+
+def test_step_entry_points_validate_on_host():
+    lib = ssd.lib()
+    p = prob()
+    assert lib.ssd_chunk_cumsum(ctypes.byref(p), None, FAKE, None) == INVALID
+    assert lib.ssd_chunk_cumsum(ctypes.byref(p), FAKE + 8, FAKE, None) == INVALID
+    assert lib.ssd_chunk_state(ctypes.byref(p), None, FAKE, FAKE, None, FAKE, None, None) == INVALID
+    assert lib.ssd_state_passing(ctypes.byref(p), FAKE, None, FAKE, None, None, None, None) == INVALID
+    assert lib.ssd_chunk_scan(ctypes.byref(p), FAKE, FAKE, None, FAKE, None, FAKE, None, None, FAKE,
+                              None) == INVALID
+    q = prob(nseq=2)
+    assert lib.ssd_state_passing(ctypes.byref(q), FAKE, FAKE, FAKE, None, None, None, None) == INVALID
+
+
+def test_binding_rejects_host_tensors_and_bad_shapes():
+    import torch
+    X = torch.zeros(1, 256, 2, 16)
+    la = torch.zeros(1, 256, 2)
+    B = torch.zeros(1, 256, 1, 16)
+    with pytest.raises(ValueError):
+        _ssd._check_shapes(X, la[:, :, :1], B, B, None, None, None, 1)
+    with pytest.raises(TypeError):
+        _ssd._check_shapes(X.double(), la, B.double(), B.double(), None, None, None, 1)
+    with pytest.raises(ValueError):
+        _ssd._ptr(X)  # CPU tensor
