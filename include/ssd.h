@@ -135,6 +135,33 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
                    const int32_t* seq_idx, void* Y, float* final_states, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/* Size of the fixed scratch array used by ssd_fwd_noalloc (64 MiB). */
+#define SSD_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * ssd_fwd_noalloc: ssd_fwd without a workspace argument, for callers that may
+ * not allocate device memory (hosts that plan all device memory ahead of time,
+ * or loops that cannot afford an allocation's implicit synchronisation). The
+ * pages have no counterpart of this entry point; it only changes where the
+ * scratch lives.
+ *   Arguments, layouts and results are those of ssd_fwd. The scratch is a fixed
+ *   SSD_NOALLOC_SCRATCH_BYTES array in the library's device memory, reserved on
+ *   every GPU that loads the library until the process exits; nothing is
+ *   allocated per call.
+ *   Problems with ssd_fwd_workspace_bytes(p) > SSD_NOALLOC_SCRATCH_BYTES return
+ *   SSD_ERR_WORKSPACE before anything is launched.
+ *   The first call on a device looks the array's address up (once per device,
+ *   with that device current); make that first call before any stream capture.
+ *   If the lookup fails the call returns SSD_ERR_CUDA.
+ *   All calls share the one array: calls that may overlap on the GPU (other
+ *   streams or threads) race on it, so the caller must order them. Leftover
+ *   contents from earlier calls are harmless: every scratch byte is written
+ *   before it is read.
+ */
+ssd_status ssd_fwd_noalloc(const ssd_problem* p, const void* X, const float* log_a, const void* B,
+                           const void* C, const float* D, const float* init_states,
+                           const int32_t* seq_idx, void* Y, float* final_states, void* stream);
+
 /* ---- the four steps, callable one by one (ssd_fwd runs them in this order) ----
  * nchunks = seqlen / chunk. cs is [batch, nheads, nchunks, chunk] fp32; a "state
  * buffer" is [batch, nchunks, nheads, dstate, headdim] fp32. */
