@@ -72,16 +72,25 @@ def algorithmic_bytes(w) -> float:
     return by
 
 
-def kernel_model(w):
-    """Algorithmic bytes and flops per launch of each kernel of the unfused path.
+def kernel_model(w, seglen=None):
+    """Algorithmic bytes and flops per launch of each kernel.
 
-    chunk_cumsum  reads log a, writes cs.
-    chunk_state   reads X, B, cs; writes one fp32 state per (b, chunk, h);
-                  flops 2 Q N P per (b, chunk, h).
-    state_passing reads the states and cs, writes the incoming states
-                  (in place) and the final states; 2 N P flops per (b, chunk, h).
-    chunk_scan    reads X, B, C, cs, D and the incoming states; writes Y;
-                  flops Q(Q+1)P + 2QNP per (b, chunk, h) + Q(Q+1)N per (b, chunk, g).
+    Chunked path (chunk Q):
+      chunk_cumsum  reads log a, writes cs.
+      chunk_state   reads X, B, cs; writes one fp32 state per (b, chunk, h);
+                    2 Q N P flops per (b, chunk, h).
+      state_passing reads the states and cs, writes the incoming states and the
+                    final states; 2 N P flops per (b, chunk, h).
+      chunk_scan    reads X, B, C, cs, D and the incoming states; writes Y;
+                    Q(Q+1)P + 2QNP flops per (b, chunk, h) + Q(Q+1)N per (b, chunk, g).
+    Fused path (segments of `seglen`, tiles of 128):
+      segment_state   reads X, B, log a; writes one fp32 state and one decay per
+                      (b, segment, h); 2 N P flops per token and head.
+      segment_passing reads and writes the segment states; 2 N P flops per
+                      (b, segment, h).
+      fused_scan      reads X, B, C, log a, D, the segment incoming states and
+                      initial states; writes Y and the final states; per (b, tile, h)
+                      128*129 P + 4*128 N P flops, per (b, tile, g) 128*129 N.
     """
     e = _esize(w)
     b, T, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
@@ -92,13 +101,25 @@ def kernel_model(w):
     csb = b * T * H * 4
     nseq = w.nseq if w.varlen != "none" else 1
     fin = b * nseq * H * N * P * 4
-    return {
+    init = fin if w.has_init else 0
+    out = {
         "chunk_cumsum": dict(bytes=2 * csb, flops=b * T * H),
         "chunk_state": dict(bytes=xb + bcb + csb + st, flops=b * cn * H * 2 * Q * N * P),
-        "state_passing": dict(bytes=2 * st + csb / Q + fin, flops=b * cn * H * 2 * N * P),
-        "chunk_scan": dict(bytes=2 * xb + 2 * bcb + csb + st,
+        "state_passing": dict(bytes=2 * st + csb / Q + fin + init, flops=b * cn * H * 2 * N * P),
+        "chunk_scan": dict(bytes=2 * xb + 2 * bcb + csb + st + init,
                            flops=b * cn * (H * (Q * (Q + 1) * P + 2 * Q * N * P) + G * Q * (Q + 1) * N)),
     }
+    if seglen:
+        nseg = -(-T // seglen)
+        sst = b * nseg * H * N * P * 4
+        ntile = -(-T // 128)
+        out.update({
+            "segment_state": dict(bytes=xb + bcb + csb + sst + b * nseg * H * 4, flops=b * T * H * 2 * N * P),
+            "segment_passing": dict(bytes=2 * sst + b * nseg * H * 4 + init, flops=b * nseg * H * 2 * N * P),
+            "fused_scan": dict(bytes=2 * xb + 2 * bcb + csb + (sst if nseg > 1 else 0) + init + fin,
+                               flops=b * ntile * (H * (128 * 129 * P + 4 * 128 * N * P) + G * 128 * 129 * N)),
+        })
+    return out
 
 
 def load_peaks():
@@ -271,6 +292,16 @@ def run_reference(args, w):
     return 0
 
 
+def family(ssd, p, path):
+    """Kernel family ssd_fwd runs for problem p under the requested path."""
+    if path in ("simt", "tcgen05", "fused"):
+        return path
+    for f in ("fused", "tcgen05"):
+        if ssd.path_supported(p, f):
+            return f
+    return "simt"
+
+
 def workload_config(w, args):
     nseq = w.nseq if w.varlen != "none" else 1
     return {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "nheads": w.nheads, "headdim": w.headdim,
@@ -342,25 +373,47 @@ def run_ours(args, w):
     value, t_max = aggregate(units, t_dev, dev if ws > 1 else None)
     ms_per_step = t_max / args.steps * 1e3
 
-    # per-kernel durations: the same four steps through the step entry points,
-    # with events between them on the launching stream
-    names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
-    lib = ssd.lib()
+    # per-kernel durations: the kernels of the path ssd_fwd runs, launched one by
+    # one through their C-ABI entry points, events between them on the stream
     import ctypes
-    nc = T // w.chunk
-    cs = wsp[: b * T * H * 4].view(torch.float32)
-    off = (b * T * H * 4 + 255) // 256 * 256
-    states = wsp[off: off + b * nc * H * N * P * 4].view(torch.float32)
+    lib = ssd.lib()
+    fam = family(ssd, p, args.path)
     sp = ctypes.c_void_p(stream.cuda_stream)
     vp = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
     pr = ctypes.byref(p)
-    launches = [
-        lambda: lib.ssd_chunk_cumsum(pr, vp(la), vp(cs), sp),
-        lambda: lib.ssd_chunk_state(pr, vp(X), vp(B), vp(cs), vp(seq), vp(states), vp(F), sp),
-        lambda: lib.ssd_state_passing(pr, vp(cs), vp(states), vp(states), vp(init), vp(seq), vp(F), sp),
-        lambda: lib.ssd_chunk_scan(pr, vp(X), vp(B), vp(C), vp(cs), vp(D), vp(states), vp(init), vp(seq), vp(Y), sp),
-    ]
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    seglen = None
+    if fam == "fused":
+        seglen = ssd.fused_segment_length(p)
+        nseg = -(-T // seglen)
+        sst = wsp[: b * nseg * H * N * P * 4].view(torch.float32)
+        soff = (b * nseg * H * N * P * 4 + 255) // 256 * 256
+        sdec = wsp[soff: soff + b * nseg * H * 4].view(torch.float32)
+        names, launches = [], []
+        if nseg > 1:
+            names += ["segment_state", "segment_passing"]
+            launches += [
+                lambda: lib.ssd_segment_state(pr, seglen, vp(X), vp(la), vp(B), vp(seq), vp(sst), vp(sdec), sp),
+                lambda: lib.ssd_segment_passing(pr, seglen, vp(sst), vp(sdec), vp(init), vp(seq), sp)]
+        names.append("fused_scan")
+        launches.append(lambda: lib.ssd_fused_scan(pr, seglen, vp(X), vp(la), vp(B), vp(C), vp(D),
+                                                   vp(sst) if nseg > 1 else None, vp(init), vp(seq), vp(Y), vp(F),
+                                                   sp))
+    else:
+        pk = ssd.problem_from(X, B, w.chunk, inputs["nseq"], "tcgen05" if fam == "tcgen05" else "simt")
+        pr = ctypes.byref(pk)
+        nc = T // w.chunk
+        cs = wsp[: b * T * H * 4].view(torch.float32)
+        off = (b * T * H * 4 + 255) // 256 * 256
+        states = wsp[off: off + b * nc * H * N * P * 4].view(torch.float32)
+        names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
+        launches = [
+            lambda: lib.ssd_chunk_cumsum(pr, vp(la), vp(cs), sp),
+            lambda: lib.ssd_chunk_state(pr, vp(X), vp(B), vp(cs), vp(seq), vp(states), vp(F), sp),
+            lambda: lib.ssd_state_passing(pr, vp(cs), vp(states), vp(states), vp(init), vp(seq), vp(F), sp),
+            lambda: lib.ssd_chunk_scan(pr, vp(X), vp(B), vp(C), vp(cs), vp(D), vp(states), vp(init), vp(seq), vp(Y),
+                                       sp),
+        ]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)] for _ in range(args.steps)]
     for i in range(args.steps):
         evs[i][0].record(stream)
         for j, fn in enumerate(launches):
@@ -405,7 +458,7 @@ def run_ours(args, w):
     e2e_value, _ = aggregate(units, e0.elapsed_time(e1) / 1e3, dev if ws > 1 else None)
 
     # roofline of the dominant kernel
-    model = kernel_model(w)
+    model = kernel_model(w, seglen)
     dom = max(per_kernel, key=per_kernel.get)
     peaks = load_peaks()
     km = model[dom]
@@ -431,11 +484,12 @@ def run_ours(args, w):
         "tflops": flops * ws / step_s / 1e12,
         "pct_bf16_peak": flops / step_s / 1e12 / peaks["bf16_tflops"],
         "pct_hbm": algorithmic_bytes(w) / step_s / 1e9 / peaks["hbm_gbs"],
-        "path": "tcgen05" if ssd.path_supported(p, "tcgen05") and args.path != "simt" else "simt",
+        "path": fam,
+        "segment_length": seglen,
         "per_kernel_us": {k: v * 1e6 for k, v in per_kernel.items()},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": len(launches) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -457,7 +511,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05", "fused"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")

@@ -72,14 +72,22 @@ typedef enum {
     SSD_DTYPE_BF16 = 1   /* X, B, C, Y in bfloat16 */
 } ssd_dtype;
 
-/* Kernel family. AUTO picks the tensor-core (tcgen05) kernels when the problem
- * is in their domain (see ssd_path_supported) and the SIMT fp32 kernels
- * otherwise. SIMT and TCGEN05 force one family (TCGEN05 returns
- * SSD_ERR_UNSUPPORTED outside its domain). */
+/* Kernel family.
+ *   SIMT     the four steps as fp32 SIMT kernels (any supported shape, fp32 or bf16);
+ *   TCGEN05  the four steps with chunk_state and chunk_scan on the tensor cores
+ *            (bf16, headdim 64, dstate 64 or 128, chunk 128 or 256, an even
+ *            number of heads per group);
+ *   FUSED    the two-level path of ssd_segment_state / ssd_segment_passing /
+ *            ssd_fused_scan (bf16, headdim 64, dstate 64 or 128, an even number
+ *            of heads per group; any chunk): the state crosses HBM once per
+ *            segment instead of once per chunk.
+ * AUTO picks FUSED, else TCGEN05, else SIMT, by what the problem allows. An
+ * explicit family outside its domain returns SSD_ERR_UNSUPPORTED. */
 typedef enum {
     SSD_PATH_AUTO = 0,
     SSD_PATH_SIMT = 1,
-    SSD_PATH_TCGEN05 = 2
+    SSD_PATH_TCGEN05 = 2,
+    SSD_PATH_FUSED = 3
 } ssd_path;
 
 typedef struct {
@@ -106,13 +114,14 @@ const char* ssd_last_cuda_error_string(void);
  * current device's compute capability). */
 ssd_status ssd_check_problem(const ssd_problem* p);
 
-/* 1 if `path` (SIMT or TCGEN05) can run problem p on the current device. */
+/* 1 if `path` (SIMT, TCGEN05 or FUSED) can run problem p on the current device. */
 int ssd_path_supported(const ssd_problem* p, ssd_path path);
 
-/* Bytes of workspace ssd_fwd needs, or (size_t)-1 if p is invalid. The
- * workspace holds the chunk cumulative sums (batch*seqlen*nheads fp32) and one
- * state per chunk (batch*nchunks*nheads*dstate*headdim fp32), each 256-byte
- * aligned. */
+/* Bytes of workspace ssd_fwd needs, or (size_t)-1 if p is invalid: the larger
+ * of the chunked paths' need (the chunk cumulative sums, batch*seqlen*nheads
+ * fp32, and one state per chunk, batch*nchunks*nheads*dstate*headdim fp32) and
+ * the fused path's need (one state and one decay per segment), each part
+ * 256-byte aligned. */
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p);
 
 /*
@@ -211,6 +220,53 @@ ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, co
                           const float* cs, const float* D, const float* incoming,
                           const float* init_states, const int32_t* seq_idx, void* Y,
                           void* stream);
+
+/* ---- the fused path: the same block decomposition at two levels ----
+ * The sequence axis is cut into segments of `seglen` tokens (a multiple of 128,
+ * at most 2048; the last segment may be shorter). Inside a segment the state is
+ * carried on chip across 128-token tiles aligned to the sequence starts, so a
+ * state goes through HBM once per segment. nseg = ceil(seqlen / seglen); a
+ * "segment state buffer" is [batch, nseg, nheads, dstate, headdim] fp32 and a
+ * "segment decay buffer" [batch, nseg, nheads] fp32. These entry points cover
+ * the FUSED family's domain only (SSD_ERR_UNSUPPORTED elsewhere). */
+
+/* Segment length ssd_fwd uses for p on the current device (-1 if p is invalid
+ * or outside the fused domain). */
+int64_t ssd_fused_segment_length(const ssd_problem* p);
+
+/* Right factors per segment: for the segment's last sequence piece [st, s1),
+ *   seg_states[b, j, h] = sum_{l in [st, s1)} (prod_{k=l+1..s1-1} a_k) B_l x_l^T
+ *   seg_decay[b, j, h]  = prod_{k in [st, s1)} a_k
+ * (wq-win section 3, "local_end_state" and "block_decay", for a block that is a
+ * segment). */
+ssd_status ssd_segment_state(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a,
+                             const void* B, const int32_t* seq_idx, float* seg_states, float* seg_decay,
+                             void* stream);
+
+/* Centre factors: H_end(j) = seg_decay(j) * H_start(j) + seg_states(j), with
+ * H_start(j) = H_end(j-1) when the last piece of segment j continues the
+ * sequence of segment j-1, else that sequence's initial state (or zero).
+ * Overwrites seg_states[b, j, h] with the state entering segment j for the
+ * sequence of its first token: H_end(j-1) when that token continues the
+ * sequence of the previous token, else that sequence's initial state (or
+ * zero). */
+ssd_status ssd_segment_passing(const ssd_problem* p, int64_t seglen, float* seg_states,
+                               const float* seg_decay, const float* init_states,
+                               const int32_t* seq_idx, void* stream);
+
+/* Per segment: walks 128-token tiles aligned to sequence starts; per tile
+ *   y_k = sum_{l <= k in tile} exp(cs_k - cs_l) (C_k . B_l) x_l + exp(cs_k) C_k^T H + D_h x_k
+ *   H  <- exp(cs_end) H + sum_{l in tile} exp(cs_end - cs_l) B_l x_l^T
+ * starting from seg_incoming[b, j, h] (the output of ssd_segment_passing) for
+ * the segment's first sequence and from the initial state (or zero) for every
+ * sequence that starts later in the segment;
+ * writes Y and, when non-NULL, final_states for every sequence that ends in
+ * the segment (and the initial state for ids after the row's last sequence).
+ * seg_incoming may be NULL when seqlen <= seglen. */
+ssd_status ssd_fused_scan(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a,
+                          const void* B, const void* C, const float* D, const float* seg_incoming,
+                          const float* init_states, const int32_t* seq_idx, void* Y,
+                          float* final_states, void* stream);
 
 #ifdef __cplusplus
 }

@@ -17,6 +17,10 @@ from .ssd import (  # noqa: F401
     chunk_scan,
     chunk_state,
     declared_functions,
+    fused_scan,
+    fused_segment_length,
+    segment_passing,
+    segment_state,
     lib,
     make_problem,
     path_supported,

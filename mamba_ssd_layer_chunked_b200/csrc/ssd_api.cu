@@ -29,7 +29,8 @@ ssd_status check_dims(const ssd_problem* p) {
         return SSD_ERR_INVALID_ARG;
     if (p->nheads % p->ngroups != 0) return SSD_ERR_INVALID_ARG;
     if (p->dtype != SSD_DTYPE_F32 && p->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
-    if (p->path != SSD_PATH_AUTO && p->path != SSD_PATH_SIMT && p->path != SSD_PATH_TCGEN05)
+    if (p->path != SSD_PATH_AUTO && p->path != SSD_PATH_SIMT && p->path != SSD_PATH_TCGEN05 &&
+        p->path != SSD_PATH_FUSED)
         return SSD_ERR_INVALID_ARG;
     if (p->chunk != 64 && p->chunk != 128 && p->chunk != 256) return SSD_ERR_UNSUPPORTED;
     if (p->seqlen % p->chunk != 0) return SSD_ERR_UNSUPPORTED;
@@ -82,10 +83,26 @@ size_t states_bytes(const ssd_problem* p) {
     return (size_t)p->batch * (p->seqlen / p->chunk) * p->nheads * p->dstate * p->headdim * sizeof(float);
 }
 
+// kernels of the chunked steps (chunk_state, chunk_scan)
 bool use_tc(const ssd_problem* p) {
     if (p->path == SSD_PATH_SIMT) return false;
     return ssd::tc_supported(p);
 }
+
+// family ssd_fwd runs
+ssd_path fwd_family(const ssd_problem* p) {
+    switch (p->path) {
+        case SSD_PATH_SIMT: return SSD_PATH_SIMT;
+        case SSD_PATH_TCGEN05: return SSD_PATH_TCGEN05;
+        case SSD_PATH_FUSED: return SSD_PATH_FUSED;
+        default: break;
+    }
+    if (ssd::fused_supported(p)) return SSD_PATH_FUSED;
+    if (ssd::tc_supported(p)) return SSD_PATH_TCGEN05;
+    return SSD_PATH_SIMT;
+}
+
+size_t chunked_workspace_bytes(const ssd_problem* p) { return align256(cs_bytes(p)) + align256(states_bytes(p)); }
 
 ssd_status check_common(const ssd_problem* p, const int32_t* seq_idx) {
     ssd_status s = check_dims(p);
@@ -99,6 +116,7 @@ ssd_status check_runnable(const ssd_problem* p) {
     ssd_status s = check_device();
     if (s != SSD_OK) return s;
     if (p->path == SSD_PATH_TCGEN05 && !ssd::tc_supported(p)) return SSD_ERR_UNSUPPORTED;
+    if (p->path == SSD_PATH_FUSED && !ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
     return SSD_OK;
 }
 
@@ -130,15 +148,14 @@ const char* ssd_last_cuda_error_string(void) { return g_cuda_err; }
 ssd_status ssd_check_problem(const ssd_problem* p) {
     ssd_status s = check_dims(p);
     if (s != SSD_OK) return s;
-    if ((s = check_device()) != SSD_OK) return s;
-    if (p->path == SSD_PATH_TCGEN05 && !ssd::tc_supported(p)) return SSD_ERR_UNSUPPORTED;
-    return SSD_OK;
+    return check_runnable(p);
 }
 
 int ssd_path_supported(const ssd_problem* p, ssd_path path) {
     if (check_dims(p) != SSD_OK || check_device() != SSD_OK) return 0;
     if (path == SSD_PATH_SIMT) return 1;
     if (path == SSD_PATH_TCGEN05) return ssd::tc_supported(p) ? 1 : 0;
+    if (path == SSD_PATH_FUSED) return ssd::fused_supported(p) ? 1 : 0;
     return 0;
 }
 
@@ -149,7 +166,64 @@ size_t ssd_states_bytes(const ssd_problem* p) {
 
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
     if (check_dims(p) != SSD_OK) return (size_t)-1;
-    return align256(cs_bytes(p)) + align256(states_bytes(p));
+    size_t need = chunked_workspace_bytes(p);
+    if (ssd::fused_supported(p)) {
+        const ssd::Dims d = make_dims(p);
+        const size_t f = ssd::fused_workspace_bytes(d, ssd::fused_default_seglen(d));
+        if (f > need) need = f;
+    }
+    return need;
+}
+
+int64_t ssd_fused_segment_length(const ssd_problem* p) {
+    if (check_dims(p) != SSD_OK || !ssd::fused_supported(p)) return -1;
+    return ssd::fused_default_seglen(make_dims(p));
+}
+
+ssd_status ssd_segment_state(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a,
+                             const void* B, const int32_t* seq_idx, float* seg_states, float* seg_decay,
+                             void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!X || !log_a || !B || !seg_states || !seg_decay) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, log_a, B, seq_idx, seg_states, seg_decay)) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = make_dims(p);
+    if (!ssd::fused_seglen_ok(d, seglen)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_device()) != SSD_OK) return s;
+    if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+    return cuda_status(ssd::launch_segment_state(d, (int)seglen, X, log_a, B, seq_idx, seg_states, seg_decay,
+                                                 (cudaStream_t)stream));
+}
+
+ssd_status ssd_segment_passing(const ssd_problem* p, int64_t seglen, float* seg_states, const float* seg_decay,
+                               const float* init_states, const int32_t* seq_idx, void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!seg_states || !seg_decay) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(seg_states, seg_decay, init_states, seq_idx)) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = make_dims(p);
+    if (!ssd::fused_seglen_ok(d, seglen)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_device()) != SSD_OK) return s;
+    if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+    return cuda_status(ssd::launch_segment_passing(d, (int)seglen, seg_states, seg_decay, init_states, seq_idx,
+                                                   (cudaStream_t)stream));
+}
+
+ssd_status ssd_fused_scan(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a, const void* B,
+                          const void* C, const float* D, const float* seg_incoming, const float* init_states,
+                          const int32_t* seq_idx, void* Y, float* final_states, void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
+    if (p->seqlen > seglen && !seg_incoming) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, log_a, B, C, D, seg_incoming, init_states, seq_idx, Y, final_states))
+        return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = make_dims(p);
+    if (!ssd::fused_seglen_ok(d, seglen)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_device()) != SSD_OK) return s;
+    if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+    return cuda_status(ssd::launch_fused_scan(d, (int)seglen, X, log_a, B, C, D, seg_incoming, init_states, seq_idx,
+                                              Y, final_states, (cudaStream_t)stream));
 }
 
 ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs, void* stream) {
@@ -215,11 +289,29 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
     if ((s = check_runnable(p)) != SSD_OK) return s;
     const ssd::Dims d = make_dims(p);
     cudaStream_t st = (cudaStream_t)stream;
+    const ssd_path fam = fwd_family(p);
+    if (fam == SSD_PATH_FUSED) {
+        const int seglen = ssd::fused_default_seglen(d);
+        const int nseg = (d.seqlen + seglen - 1) / seglen;
+        float* seg_states = static_cast<float*>(workspace);
+        const size_t stb = (size_t)d.batch * nseg * d.nheads * d.dstate * d.headdim * sizeof(float);
+        float* seg_decay = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(stb));
+        cudaError_t e = cudaSuccess;
+        if (nseg > 1) {
+            e = ssd::launch_segment_state(d, seglen, X, log_a, B, seq_idx, seg_states, seg_decay, st);
+            if (e != cudaSuccess) return cuda_status(e);
+            e = ssd::launch_segment_passing(d, seglen, seg_states, seg_decay, init_states, seq_idx, st);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+        e = ssd::launch_fused_scan(d, seglen, X, log_a, B, C, D, nseg > 1 ? seg_states : nullptr, init_states,
+                                   seq_idx, Y, final_states, st);
+        return cuda_status(e);
+    }
     float* cs = static_cast<float*>(workspace);
     float* states = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(cs_bytes(p)));
     cudaError_t e = ssd::launch_chunk_cumsum(d, log_a, cs, st);
     if (e != cudaSuccess) return cuda_status(e);
-    const bool tc = use_tc(p);
+    const bool tc = (fam == SSD_PATH_TCGEN05);
     e = tc ? ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, final_states, st)
            : ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st);
     if (e != cudaSuccess) return cuda_status(e);

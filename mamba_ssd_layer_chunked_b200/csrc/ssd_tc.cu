@@ -550,6 +550,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
 
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes, int slot) {
+    return ensure_smem_attr(reinterpret_cast<const void*>(kernel), bytes, slot);
+}
+
+}  // namespace
+
 // ---------------------------------------------------------------------------
 // host: tensor maps
 // ---------------------------------------------------------------------------
@@ -597,12 +604,7 @@ cudaError_t bc_map(CUtensorMap* m, const Dims& d, const void* Bp, uint32_t box_t
     return make_map(m, Bp, d.dstate, d.ngroups, d.seqlen, d.batch, box_tok);
 }
 
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes, int slot) {
-    return ensure_smem_attr(reinterpret_cast<const void*>(kernel), bytes, slot);
-}
 
-}  // namespace
 
 bool tc_supported(const ssd_problem* p) {
     if (p->dtype != SSD_DTYPE_BF16) return false;

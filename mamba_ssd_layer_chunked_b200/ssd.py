@@ -22,7 +22,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "ssd.h")
 
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA = range(5)
 SSD_DTYPE_F32, SSD_DTYPE_BF16 = 0, 1
-PATHS = {"auto": 0, "simt": 1, "tcgen05": 2}
+PATHS = {"auto": 0, "simt": 1, "tcgen05": 2, "fused": 3}
 
 
 class SSDError(RuntimeError):
@@ -61,6 +61,10 @@ def _declare(lib):
         "ssd_chunk_state": ([P, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "ssd_state_passing": ([P, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "ssd_chunk_scan": ([P] + [vp] * 9 + [vp], ctypes.c_int),
+        "ssd_fused_segment_length": ([P], ctypes.c_int64),
+        "ssd_segment_state": ([P, ctypes.c_int64] + [vp] * 7, ctypes.c_int),
+        "ssd_segment_passing": ([P, ctypes.c_int64] + [vp] * 5, ctypes.c_int),
+        "ssd_fused_scan": ([P, ctypes.c_int64] + [vp] * 11, ctypes.c_int),
     }
     for name, (argtypes, restype) in sig.items():
         f = getattr(lib, name)
@@ -267,4 +271,48 @@ def chunk_scan(X, B, C, cs, incoming, chunk, D=None, init_states=None, seq_idx=N
     Y = torch.empty_like(X)
     _check(lib().ssd_chunk_scan(ctypes.byref(p), _ptr(X), _ptr(B), _ptr(C), _ptr(cs), _ptr(D), _ptr(incoming),
                                 _ptr(init_states), _ptr(seq_idx), _ptr(Y), _stream(stream)), "ssd_chunk_scan")
+    return Y
+
+
+# ---- the fused path, one call per kernel -------------------------------------
+
+def fused_segment_length(p: Problem) -> int:
+    """Segment length ssd_fwd uses on the fused path (-1 outside its domain)."""
+    return int(lib().ssd_fused_segment_length(ctypes.byref(p)))
+
+
+def _fused_problem(X, B, nseq, chunk):
+    return problem_from(X, B, chunk, nseq, "fused")
+
+
+def segment_state(X, log_a, B, seglen, seq_idx=None, nseq=1, chunk=64, stream=None):
+    """Right factor per segment: (seg_states [b, nseg, H, N, P], seg_decay [b, nseg, H])."""
+    p = _fused_problem(X, B, nseq, chunk)
+    b, T, H, P = X.shape
+    N = B.shape[3]
+    nseg = (T + seglen - 1) // seglen
+    st = torch.empty((b, nseg, H, N, P), dtype=torch.float32, device=X.device)
+    dec = torch.empty((b, nseg, H), dtype=torch.float32, device=X.device)
+    _check(lib().ssd_segment_state(ctypes.byref(p), seglen, _ptr(X), _ptr(log_a), _ptr(B), _ptr(seq_idx), _ptr(st),
+                                   _ptr(dec), _stream(stream)), "ssd_segment_state")
+    return st, dec
+
+
+def segment_passing(seg_states, seg_decay, X, B, seglen, init_states=None, seq_idx=None, nseq=1, chunk=64,
+                    stream=None):
+    """State entering each segment, written over seg_states (returned)."""
+    p = _fused_problem(X, B, nseq, chunk)
+    _check(lib().ssd_segment_passing(ctypes.byref(p), seglen, _ptr(seg_states), _ptr(seg_decay), _ptr(init_states),
+                                     _ptr(seq_idx), _stream(stream)), "ssd_segment_passing")
+    return seg_states
+
+
+def fused_scan(X, log_a, B, C, seglen, seg_incoming=None, D=None, init_states=None, seq_idx=None, nseq=1,
+               final_states: Optional[torch.Tensor] = None, chunk=64, stream=None) -> torch.Tensor:
+    """Y from the incoming segment states (and final states into final_states)."""
+    p = _fused_problem(X, B, nseq, chunk)
+    Y = torch.empty_like(X)
+    _check(lib().ssd_fused_scan(ctypes.byref(p), seglen, _ptr(X), _ptr(log_a), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(seg_incoming), _ptr(init_states), _ptr(seq_idx), _ptr(Y), _ptr(final_states),
+                                _stream(stream)), "ssd_fused_scan")
     return Y

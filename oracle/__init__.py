@@ -13,6 +13,7 @@ Contents
                        localise errors in the chunked path.
 ``chunk_cumsum``       the within-chunk inclusive cumulative sum of log a (a
                        NumPy one-liner: the definition of the quantity).
+``segment_decay``      the product of a over each chunk's last sequence piece.
 ``dual_matrix``        brute-force matrix form M = L * (C B^T) (+ init and D
                        terms), Y = M X, in NumPy fp64, tiny sizes only.
 ``blockwise``          the pages' four-step block algorithm in NumPy fp64
@@ -28,6 +29,7 @@ from .ssd_oracle import (  # noqa: F401
     ssd_reference,
     chunk_states,
     chunk_cumsum,
+    segment_decay,
     dual_matrix,
     blockwise,
     recurrence_numpy,

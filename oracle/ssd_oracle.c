@@ -138,17 +138,17 @@ int ssd_oracle_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdi
  *   local[b,c,h]    = the state at the end of the chunk of a recurrence that
  *       starts from zero at the first token of the chunk's last sequence piece
  *       (max(cQ, start of that sequence)).
- * Both are [batch, nchunks, nheads, dstate, headdim]; either may be NULL.
- * seqlen must be a multiple of chunk. */
+ * Both are [batch, nchunks, nheads, dstate, headdim], nchunks = ceil(seqlen /
+ * chunk) (the last chunk may be shorter); either may be NULL. */
 int ssd_oracle_chunk_states(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                             int64_t dstate, int64_t ngroups, int64_t nseq, int64_t chunk,
                             const double* X, const double* log_a, const double* B,
                             const double* init_states, const int32_t* seq_idx,
                             double* incoming, double* local, int nthreads) {
     if (check_dims(batch, seqlen, nheads, headdim, dstate, ngroups, nseq)) return 1;
-    if (chunk <= 0 || seqlen % chunk != 0 || !X || !log_a || !B) return 1;
+    if (chunk <= 0 || !X || !log_a || !B) return 1;
     if (!seq_idx && nseq != 1) return 1;
-    const int64_t P = headdim, N = dstate, NP = dstate * headdim, nchunks = seqlen / chunk;
+    const int64_t P = headdim, N = dstate, NP = dstate * headdim, nchunks = (seqlen + chunk - 1) / chunk;
     const int64_t heads_per_group = nheads / ngroups;
     int failed = 0;
 #ifdef _OPENMP
@@ -164,9 +164,10 @@ int ssd_oracle_chunk_states(int64_t batch, int64_t seqlen, int64_t nheads, int64
         load_state(H, init_states, b, cur, h, nseq, nheads, NP);
         for (int64_t c = 0; c < nchunks; ++c) {
             const int64_t t0 = c * chunk;
-            const int64_t s_last = seq_of(seq_idx, b, seqlen, t0 + chunk - 1, nseq);
+            const int64_t t1 = (t0 + chunk < seqlen) ? t0 + chunk : seqlen;
+            const int64_t s_last = seq_of(seq_idx, b, seqlen, t1 - 1, nseq);
             memset(L, 0, (size_t)NP * sizeof(double));
-            for (int64_t t = t0; t < t0 + chunk; ++t) {
+            for (int64_t t = t0; t < t1; ++t) {
                 const int64_t s = seq_of(seq_idx, b, seqlen, t, nseq);
                 if (t > 0 && s != cur) {
                     cur = s;

@@ -121,7 +121,7 @@ def chunk_states(X, log_a, B, chunk, init_states=None, seq_idx=None, nseq=None,
     X, log_a, B, init = (_f64(v) for v in (X, log_a, B, init_states))
     si = None if seq_idx is None else np.ascontiguousarray(np.asarray(seq_idx, dtype=np.int32))
     batch, seqlen, nheads, headdim, dstate, ngroups, ns = _dims(X, B, si, nseq)
-    nchunks = seqlen // chunk
+    nchunks = (seqlen + chunk - 1) // chunk  # the last chunk may be shorter
     inc = np.empty((batch, nchunks, nheads, dstate, headdim), dtype=np.float64)
     loc = np.empty_like(inc)
     rc = _load().ssd_oracle_chunk_states(batch, seqlen, nheads, headdim, dstate, ngroups, ns, chunk,
@@ -143,6 +143,25 @@ def chunk_cumsum(log_a, chunk) -> np.ndarray:
     nchunks = seqlen // chunk
     la = la.reshape(batch, nchunks, chunk, nheads).transpose(0, 3, 1, 2)
     return np.cumsum(la, axis=-1)
+
+
+def segment_decay(log_a, chunk, seq_idx=None) -> np.ndarray:
+    """Product of a_t over the last sequence piece of each chunk (the block decay
+    of wq-win 088 section 3 for a block that may hold a sequence start):
+    [batch, nchunks, nheads], nchunks = ceil(seqlen / chunk)."""
+    la = np.asarray(log_a, dtype=np.float64)
+    batch, seqlen, nheads = la.shape
+    nch = (seqlen + chunk - 1) // chunk
+    seq = np.zeros((batch, seqlen), dtype=np.int64) if seq_idx is None else np.asarray(seq_idx, np.int64)
+    out = np.zeros((batch, nch, nheads))
+    for b in range(batch):
+        for c in range(nch):
+            t1 = min(seqlen, (c + 1) * chunk)
+            st = t1 - 1
+            while st > c * chunk and seq[b, st - 1] == seq[b, t1 - 1]:
+                st -= 1
+            out[b, c] = np.exp(la[b, st:t1].sum(axis=0))
+    return out
 
 
 def _group_of(h, nheads, ngroups):

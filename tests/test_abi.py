@@ -28,7 +28,8 @@ def test_library_exports_every_declared_function():
         assert hasattr(lib, n), n
     assert set(names) >= {"ssd_status_string", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
                           "ssd_chunk_scan", "ssd_check_problem", "ssd_path_supported", "ssd_states_bytes",
-                          "ssd_last_cuda_error_string"}
+                          "ssd_last_cuda_error_string", "ssd_segment_state", "ssd_segment_passing",
+                          "ssd_fused_scan", "ssd_fused_segment_length"}
 
 
 def test_problem_struct_layout():
@@ -43,11 +44,19 @@ def test_status_strings():
 
 def test_workspace_bytes_formula():
     p = prob()
+    align = lambda x: (x + 255) // 256 * 256
     cs = 2 * 512 * 4 * 4
     st = 2 * (512 // 256) * 4 * 128 * 64 * 4
-    align = lambda x: (x + 255) // 256 * 256
-    assert ssd.workspace_bytes(p) == align(cs) + align(st)
+    L = ssd.fused_segment_length(p)
+    assert L % 128 == 0 and 128 <= L <= 2048
+    nseg = -(-512 // L)
+    fused = align(2 * nseg * 4 * 128 * 64 * 4) + align(2 * nseg * 4 * 4)
+    assert ssd.workspace_bytes(p) == max(align(cs) + align(st), fused)
     assert ssd.states_bytes(p) == st
+    # outside the fused domain (fp32) only the chunked need counts
+    q = prob(dtype=ssd.ssd.SSD_DTYPE_F32)
+    assert ssd.fused_segment_length(q) == -1
+    assert ssd.workspace_bytes(q) == align(cs) + align(st)
 
 
 @pytest.mark.parametrize("field,value,expect", [
@@ -110,6 +119,15 @@ def test_step_entry_points_validate_on_host():
                               None) == INVALID
     q = prob(nseq=2)
     assert lib.ssd_state_passing(ctypes.byref(q), FAKE, FAKE, FAKE, None, None, None, None) == INVALID
+    # fused steps: bad segment lengths and null pointers are rejected on the host
+    for L in (0, 100, 4096):
+        assert lib.ssd_segment_state(ctypes.byref(p), L, FAKE, FAKE, FAKE, None, FAKE, FAKE, None) == INVALID
+        assert lib.ssd_segment_passing(ctypes.byref(p), L, FAKE, FAKE, None, None, None) == INVALID
+        assert lib.ssd_fused_scan(ctypes.byref(p), L, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, FAKE, None,
+                                  None) == INVALID
+    assert lib.ssd_segment_state(ctypes.byref(p), 256, None, FAKE, FAKE, None, FAKE, FAKE, None) == INVALID
+    assert lib.ssd_fused_scan(ctypes.byref(p), 256, FAKE, FAKE, FAKE, FAKE, None, None, None, None, FAKE, None,
+                              None) == INVALID  # two segments need the incoming states
 
 
 def test_binding_rejects_host_tensors_and_bad_shapes():

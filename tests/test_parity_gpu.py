@@ -16,7 +16,7 @@ from workloads import WORKLOADS, make_custom, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["simt", "tcgen05"]
+PATHS = ["simt", "tcgen05", "fused"]
 
 
 def _ssd():
@@ -126,6 +126,61 @@ def test_steps(name, path):
     Y = ssd.chunk_scan(g["X"], g["B"], g["C"], cs, torch.from_numpy(np.ascontiguousarray(inc_ref, dtype=np.float32)).cuda(), Q,
                        D=g["D"], init_states=g["init_states"], seq_idx=g["seq_idx"], nseq=nseq, path=path)
     assert_close(Y.float().cpu().numpy().astype(np.float64), Yr, tau, "chunk_scan Y")
+
+
+# --------------------------------------------------------------------------- #
+# The fused path, kernel by kernel, against the oracle's quantities at segment
+# level (a segment is a chunk of the block algorithm)
+# --------------------------------------------------------------------------- #
+
+FUSED_CASES = [
+    # (name, seglen)
+    ("bf16_varlen_N128_Q256", 256),
+    ("bf16_varlen_N128_Q256", 384),   # ragged last segment
+    ("bf16_single_N64_Q128", 128),
+    ("bf16_short_seqs", 256),
+    ("bf16_init_N128_Q128", 1024),    # one segment
+    ("bf16_groups2", 256),
+]
+
+
+@pytest.mark.parametrize("name,seglen", FUSED_CASES)
+def test_fused_steps(name, seglen):
+    ssd = _ssd()
+    b, T, H, P, N, G, Q, dtype, lengths, D, init = SMALL[name]
+    nseq = 1 if lengths is None else max(len(r) for r in lengths)
+    d = make_custom(b, T, H, P, N, ngroups=G, dtype=dtype, seed=31 + seglen, has_D=D, has_init=init,
+                    lengths=lengths, nseq=nseq if lengths else None)
+    _skip_unsupported(d, dtype, Q, "fused")
+    g = to_device(d, dtype)
+    tau = TAU[dtype]
+    X, B, C = g["X"], g["B"], g["C"]
+    inc_ref, loc_ref = oracle.chunk_states(d["X"], d["log_a"], d["B"], seglen, d["init_states"], d["seq_idx"],
+                                           nseq=nseq)
+    dec_ref = oracle.segment_decay(d["log_a"], seglen, d["seq_idx"])
+    Yr, Fr = run_oracle(d)
+    nseg = -(-T // seglen)
+    if nseg > 1:
+        st, dec = ssd.segment_state(X, g["log_a"], B, seglen, g["seq_idx"], nseq)
+        assert_close(st.cpu().numpy().astype(np.float64), loc_ref, tau, "segment states")
+        assert_close(dec.cpu().numpy().astype(np.float64), dec_ref, 1e-5, "segment decay")
+        inc = ssd.segment_passing(st, dec, X, B, seglen, g["init_states"], g["seq_idx"], nseq)
+        assert_close(inc.cpu().numpy().astype(np.float64), inc_ref, tau, "segment incoming states")
+        # segment_passing alone, fed the oracle's states and decays: fp32 arithmetic
+        st2 = torch.from_numpy(np.ascontiguousarray(loc_ref, dtype=np.float32)).cuda()
+        dec2 = torch.from_numpy(np.ascontiguousarray(dec_ref, dtype=np.float32)).cuda()
+        inc2 = ssd.segment_passing(st2, dec2, X, B, seglen, g["init_states"], g["seq_idx"], nseq)
+        assert_close(inc2.cpu().numpy().astype(np.float64), inc_ref, 1e-5, "segment incoming (oracle inputs)")
+        seg_in = torch.from_numpy(np.ascontiguousarray(inc_ref, dtype=np.float32)).cuda()
+    else:
+        seg_in = None
+    # fused_scan fed the oracle's incoming segment states
+    F = torch.full((b, nseq, H, N, P), float("nan"), dtype=torch.float32, device="cuda")
+    Y = ssd.fused_scan(X, g["log_a"], B, C, seglen, seg_in, D=g["D"], init_states=g["init_states"],
+                       seq_idx=g["seq_idx"], nseq=nseq, final_states=F)
+    torch.cuda.synchronize()
+    assert_close(Y.float().cpu().numpy().astype(np.float64), Yr, tau, "fused_scan Y")
+    assert_close(F.cpu().numpy().astype(np.float64), Fr, tau, "fused_scan final states")
 
 
 # --------------------------------------------------------------------------- #
