@@ -124,9 +124,18 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     float tail = 0.f;  // sum of log a after the current tile, this thread's head
     bool cut = false;
     int done = 0;
+    // log a of this thread's (row, head) in a tile; unconditional (clamped row)
+    // so that the prefetch does not stall until the value is used
+    auto load_la = [&](int i) -> float {
+        const int ts = st + 128 * i;
+        const int v = min(128, s1 - ts);
+        return log_a[(row + ts + min(rr, v - 1)) * d.nheads + h0 + hh];
+    };
+    float la_cur = load_la(ntiles - 1);
     for (int i = ntiles - 1; i >= 0; --i) {
         const int ts = st + 128 * i;
         const int v = min(128, s1 - ts);
+        const float la_nxt = i > 0 ? load_la(i - 1) : 0.f;
         if (tid == 0) {
             mbar_arrive_expect_tx(&bar_load, kXB + kBB);
             tma_load_4d(Xs, &tm_x, &bar_load, 0, h0, ts, b);
@@ -135,8 +144,8 @@ __global__ void __launch_bounds__(kSegThreads, 1)
             for (int q = 0; q < N / 64; ++q) tma_load_4d(Bs + q * kBox, &tm_b, &bar_load, 64 * q, g, ts, b);
         }
         // within-tile inclusive cumsum of log a (one row per thread, one head per 4 warps)
-        const float la = rr < v ? log_a[(row + ts + rr) * d.nheads + h0 + hh] : 0.f;
-        float x = la;
+        float x = rr < v ? la_cur : 0.f;
+        la_cur = la_nxt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -155,11 +164,13 @@ __global__ void __launch_bounds__(kSegThreads, 1)
         // weight of row rr: prod of a over (rr, segment end] = exp(tail + tot - cs)
         const float wgt = rr < v ? ex2_approx((tail + tot - cs) * kLog2e) : 0.f;
         mbar_wait(&bar_load, done & 1);
-        // scale row rr of head hh in place
+        // scale row rr of head hh in place; the chunk order is rotated by row so
+        // that the 32 rows of a warp spread over all banks
         {
             uint8_t* rowp = Xs + hh * kBox + rr * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int cc = 0; cc < 8; ++cc) {
+                const int c = (cc + rr) & 7;
                 uint4 vv = *reinterpret_cast<uint4*>(rowp + 16 * c);
                 uint32_t* u = reinterpret_cast<uint32_t*>(&vv);
 #pragma unroll
@@ -269,7 +280,8 @@ __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, int seglen
 // ===========================================================================
 // fused_scan
 // ===========================================================================
-constexpr int kComputeThreads = 256;
+constexpr int kComputeWarps = 16;
+constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kFusedThreads = kComputeThreads + 32;  // + one control warp
 
 template <int N>
@@ -278,8 +290,8 @@ struct FusedSmem {
     static constexpr uint32_t kB = (N / 64) * kBox;  // per stage
     static constexpr uint32_t kX = 2 * kBox;         // per stage, two heads
     static constexpr uint32_t kH = (N / 64) * kBox;  // carried state, bf16, rows (h,p), K = n
-    static constexpr uint32_t kHY = kH > kX ? kH : kX;
-    static constexpr uint32_t oC = 0, oB = kC, oX = oB + 2 * kB, oHY = oX + 2 * kX, oTail = oHY + kHY;
+    static constexpr uint32_t kHY = kH > 2 * kBox ? kH : 2 * kBox;  // ... and the Y staging of a tile
+    static constexpr uint32_t oC = 0, oB = kC, oX = oB + 2 * kB, oH = oX + 2 * kX, oTail = oH + kHY;
 };
 
 // One tile: first token, valid rows, and flags.
@@ -299,6 +311,20 @@ __device__ __forceinline__ Tile unpack_tile(int2 e) {
     return t;
 }
 
+// Thread layout of the 16 compute warps: warp w owns the TMEM lane quarter
+// w % 4 (rows 32 (w % 4) .. +31) and the column quarter w / 4 of every
+// 128-column accumulator it touches; the four warps of a lane quarter split
+// the columns.
+//
+// Per tile t the compute warps run, in this order,
+//   epilogue(t):  Y = Y_diag + rscale Y_off + D x, staged (bf16) in the buffer
+//                 of the carried state, which Y_off(t) has finished reading, for
+//                 the TMA store; X' = w X in place in the tile's X buffer;
+//   L o G(t+1):   the next tile's masked C B^T into TMEM (while the tile state
+//                 MMA of tile t runs and Y(t) drains);
+//   state(t):     H <- a H + S and its bf16 copy for the next C H.
+// Tensor memory: G [0,128), L o G [128,256), Y_diag [256,384), and
+// [384,512) holds Y_off, then the tile state S once Y_off has been read.
 template <int N>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
@@ -308,13 +334,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                       const int32_t* __restrict__ seq_idx, __nv_bfloat16* __restrict__ Y,
                       float* __restrict__ final_states) {
     using S = FusedSmem<N>;
+    constexpr int NQ = N / 4;  // state columns per thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* Cs = smem + S::oC;
-    uint8_t* HY = smem + S::oHY;
-    int* seq_s = reinterpret_cast<int*>(smem + S::oTail);   // [seglen] ids of the segment (varlen only)
+    uint8_t* Hs = smem + S::oH;
+    int* seq_s = reinterpret_cast<int*>(smem + S::oTail);  // [seglen] ids of the segment (varlen only)
     int2* tiles = reinterpret_cast<int2*>(seq_s + (seq_idx ? seglen : 0));  // tile list
-    __shared__ float cs2[2][2][128];  // [buffer][head][row]: log2-scaled within-tile cumsum
+    __shared__ __align__(16) float cs2[2][2][128];  // [buffer][head][row]: log2-scaled within-tile cumsum
+    __shared__ __align__(16) float colf[kComputeWarps][2][32];  // per-warp column factors
     __shared__ float wsum[8];
     __shared__ int ntiles_s, lastid_s;
     __shared__ __align__(8) uint64_t bar_c, bar_bx[2], bar_g, bar_yo, bar_yd, bar_s, bar_lg, bar_epi, bar_st,
@@ -341,14 +369,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         mbar_init(&bar_c, 1);
         mbar_init(&bar_bx[0], 1);
         mbar_init(&bar_bx[1], 1);
+        mbar_init(&bar_free, 1);
         mbar_init(&bar_g, 1);
         mbar_init(&bar_yo, 1);
         mbar_init(&bar_yd, 1);
         mbar_init(&bar_s, 1);
-        mbar_init(&bar_lg, 8);
-        mbar_init(&bar_epi, 8);
-        mbar_init(&bar_st, 8);
-        mbar_init(&bar_free, 1);
+        mbar_init(&bar_lg, kComputeWarps);
+        mbar_init(&bar_epi, kComputeWarps);
+        mbar_init(&bar_st, kComputeWarps);
         mbar_fence_init();
     }
     if (warp == 0) {
@@ -386,9 +414,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
     __syncthreads();
     const int ntiles = ntiles_s;
-    const uint32_t tm_g = tmem_base, tm_ls = tmem_base + 128, tm_yd = tmem_base + 256, tm_yo = tmem_base + 384;
+    const uint32_t tm_g = tmem_base, tm_lg = tmem_base + 128, tm_yd = tmem_base + 256, tm_yos = tmem_base + 384;
 
-    if (warp == 8) {
+    if (warp == kComputeWarps) {
         // =================== control warp: TMA and MMA issue ===================
         if (lane == 0) {
             const uint32_t idesc_nn = idesc_bf16(128, 128, false, false);   // K-major A and B
@@ -411,8 +439,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 #pragma unroll
                 for (int q = 0; q < N / 64; ++q) tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, tl.ts, b);
             };
+            const uint32_t ca = smem_u32(Cs), ha = smem_u32(Hs);
             auto issue_g = [&](int t) {
-                const uint32_t ca = smem_u32(Cs), ba = smem_u32(smem + S::oB + (t & 1) * S::kB);
+                const uint32_t ba = smem_u32(smem + S::oB + (t & 1) * S::kB);
 #pragma unroll
                 for (int k = 0; k < N / 16; ++k) {
                     const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
@@ -432,120 +461,188 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const int st = t & 1;
                 const uint32_t par = t & 1;
                 const Tile tl = unpack_tile(tiles[t]);
-                // Y_off = C Hs (Hs: the state before this tile, written by the compute warps)
+                const uint32_t xa = smem_u32(smem + S::oX + st * S::kX);
+                const uint32_t ba = smem_u32(smem + S::oB + st * S::kB);
+                // Y_off = C Hs once the state before this tile is in Hs
                 mbar_wait(&bar_st, par);
                 tc_fence_after();
-                {
-                    const uint32_t ca = smem_u32(Cs), ha = smem_u32(HY);
 #pragma unroll
-                    for (int k = 0; k < N / 16; ++k) {
-                        const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                        mma_bf16_ss(tm_yo, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ha + off, 16, 1024),
-                                    idesc_nn, k > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&bar_yo);
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
+                    mma_bf16_ss(tm_yos, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ha + off, 16, 1024),
+                                idesc_nn, k > 0 ? 1u : 0u);
                 }
-                // C is free once G and Y_off have read it
-                if (t + 1 < ntiles) {
-                    mbar_wait(&bar_g, par);
-                    mbar_wait(&bar_yo, par);
-                    load_c(t + 1);
-                }
+                mma_commit(&bar_yo);
                 // Y_diag = (L o G) X, A operand from TMEM
                 mbar_wait(&bar_lg, par);
                 tc_fence_after();
-                {
-                    const uint32_t xa = smem_u32(smem + S::oX + st * S::kX);
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            mma_bf16_ts(tm_yd + 64 * hh, tm_ls + 64 * hh + 8 * k,
-                                        smem_desc_sw128(xa + hh * kBox + k * 2048, kBox, 1024), idesc_ts,
-                                        k > 0 ? 1u : 0u);
-                    mma_commit(&bar_yd);
-                }
-                // tile state S = X'^T B after the epilogue scaled X in place
-                mbar_wait(&bar_epi, par);
-                tc_fence_after();
-                const bool full = tl.v == 128;
-                if (full) {
-                    tma_store_4d(&tm_y, HY, 0, h0, tl.ts, b);
-                    tma_store_4d(&tm_y, HY + kBox, 0, h0 + 1, tl.ts, b);
-                    tma_store_commit();
-                }
-                {
-                    const uint32_t xa = smem_u32(smem + S::oX + st * S::kX);
-                    const uint32_t ba = smem_u32(smem + S::oB + st * S::kB);
+                for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_bf16_ss(tm_ls, smem_desc_sw128(xa + k * 2048, kBox, 1024),
-                                    smem_desc_sw128(ba + k * 2048, kBox, 1024), idesc_st, k > 0 ? 1u : 0u);
-                    mma_commit(&bar_s);
-                }
-                // next tile's G as soon as its operands are in
+                        mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 64 * hh + 8 * k,
+                                    smem_desc_sw128(xa + hh * kBox + k * 2048, kBox, 1024), idesc_ts, k > 0 ? 1u : 0u);
+                mma_commit(&bar_yd);
+                // C is free once G(t) and Y_off(t) have read it; G(t+1) as soon as its operands are in
                 if (t + 1 < ntiles) {
+                    mbar_wait(&bar_yo, par);
+                    load_c(t + 1);
                     mbar_wait(&bar_c, (t + 1) & 1);
                     mbar_wait(&bar_bx[st ^ 1], ((t + 1) >> 1) & 1);
                     tc_fence_after();
                     issue_g(t + 1);
                 }
+                // epilogue done: store Y(t) from the staging buffer; tile state S = X'^T B
+                mbar_wait(&bar_epi, par);
+                tc_fence_after();
+                const bool full = tl.v == 128;
+                if (full) {
+                    tma_store_4d(&tm_y, Hs, 0, h0, tl.ts, b);
+                    tma_store_4d(&tm_y, Hs + kBox, 0, h0 + 1, tl.ts, b);
+                    tma_store_commit();
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ss(tm_yos, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
+                                idesc_st, k > 0 ? 1u : 0u);
+                mma_commit(&bar_s);
                 if (full) tma_store_wait_read0();
                 mbar_arrive(&bar_free);
                 // this stage is free once the tile state has been computed
-                mbar_wait(&bar_s, par);
-                if (t + 2 < ntiles) load_bx(t + 2);
+                if (t + 2 < ntiles) {
+                    mbar_wait(&bar_s, par);
+                    load_bx(t + 2);
+                }
             }
         }
         __syncwarp();
     } else {
         // =================== compute warps ===================
-        const int q4 = warp & 3, half = warp >> 2;
+        const int q4 = warp & 3, cq = warp >> 2;
         const int m = 32 * q4 + lane;           // TMEM lane: token row, or (head, p) for states
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
         const int sh = m >> 6, sp = m & 63;     // state row (head, p) of lane m
-        constexpr int NH = N / 2;               // state columns per thread
-        float Hreg[NH];
+        float Hreg[NQ];
 
         auto load_state = [&](const float* src) {  // src: [N][P] of head sh, or null for zero
 #pragma unroll
-            for (int i = 0; i < NH; ++i) Hreg[i] = src ? src[(int64_t)(half * NH + i) * kP + sp] : 0.f;
+            for (int i = 0; i < NQ; ++i) Hreg[i] = src ? src[(int64_t)(cq * NQ + i) * kP + sp] : 0.f;
         };
         auto write_hs = [&]() {  // bf16 state, row m, K-major over n
 #pragma unroll
-            for (int c8 = 0; c8 < NH / 8; ++c8) {
-                const int n = half * NH + 8 * c8;
+            for (int c8 = 0; c8 < NQ / 8; ++c8) {
+                const int n = cq * NQ + 8 * c8;
                 const uint4 u = make_uint4(pack_bf16(Hreg[8 * c8], Hreg[8 * c8 + 1]), pack_bf16(Hreg[8 * c8 + 2], Hreg[8 * c8 + 3]),
                                            pack_bf16(Hreg[8 * c8 + 4], Hreg[8 * c8 + 5]), pack_bf16(Hreg[8 * c8 + 6], Hreg[8 * c8 + 7]));
-                *reinterpret_cast<uint4*>(HY + (n >> 6) * kBox + sw128_off(m, (n & 63) >> 3)) = u;
+                *reinterpret_cast<uint4*>(Hs + (n >> 6) * kBox + sw128_off(m, (n & 63) >> 3)) = u;
             }
         };
         auto signal = [&](uint64_t* bar) {
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
+        // log a of tile t for (head warp/4, row 32 (warp%4) + lane), warps 0..7; the
+        // load is unconditional (clamped row) so that it does not stall until used
+        auto load_la = [&](int t) -> float {
+            if (warp >= 8 || t >= ntiles) return 0.f;
+            const Tile tl = unpack_tile(tiles[t]);
+            const int hh = warp >> 2, rr = min(32 * (warp & 3) + lane, tl.v - 1);
+            return log_a[(row + tl.ts + rr) * d.nheads + h0 + hh];
+        };
         // within-tile cumsum of log a * log2(e) for tile t into buffer t & 1
-        auto tile_cumsum = [&](int t, float la) {
-            const int hh = warp >> 2, rr = 32 * (warp & 3) + lane;
-            float x = la * kLog2e;
+        auto tile_cumsum = [&](int t, float la_raw) {
+            const int hh = (warp >> 2) & 1, rr = 32 * (warp & 3) + lane;
+            float x = 0.f;
+            if (warp < 8) {
+                const Tile tl = unpack_tile(tiles[t]);
+                x = rr < tl.v ? la_raw * kLog2e : 0.f;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                if (lane == 31) wsum[warp] = x;
             }
-            if (lane == 31) wsum[warp] = x;
             named_bar_sync(1, kComputeThreads);
-            float pre = 0.f;
+            if (warp < 8) {
+                float pre = 0.f;
 #pragma unroll
-            for (int w = 0; w < 3; ++w)
-                if (w < (warp & 3)) pre += wsum[4 * hh + w];
-            cs2[t & 1][hh][rr] = x + pre;
+                for (int w = 0; w < 3; ++w)
+                    if (w < (warp & 3)) pre += wsum[4 * hh + w];
+                cs2[t & 1][hh][rr] = x + pre;
+            }
             named_bar_sync(1, kComputeThreads);
         };
-        auto load_la = [&](int t) -> float {
-            const Tile tl = unpack_tile(tiles[t]);
-            const int hh = warp >> 2, rr = 32 * (warp & 3) + lane;
-            return rr < tl.v ? log_a[(row + tl.ts + rr) * d.nheads + h0 + hh] : 0.f;
+        // L o G of tile t into TMEM (bf16): row m, columns [32 cq, 32 cq + 32), both heads.
+        // Above the diagonal block 0; on it exp(c_m - c_l) for l <= m; below it
+        // exp(c_m - c_r0) * exp(c_r0 - c_l) with r0 = 32 q4 (both factors <= 1).
+        auto build_lg = [&](int t) {
+            const float* c2 = &cs2[t & 1][0][0];
+            const int r0 = 32 * q4, cb = 32 * cq;
+            const float ck0 = c2[m], ck1 = c2[128 + m];
+            float rf0 = 0.f, rf1 = 0.f;
+            if (cq < q4) {
+                const float cr0 = c2[r0], cr1 = c2[128 + r0];
+                rf0 = ex2_approx(ck0 - cr0);
+                rf1 = ex2_approx(ck1 - cr1);
+                colf[warp][0][lane] = ex2_approx(cr0 - c2[cb + lane]);  // column cb + lane
+                colf[warp][1][lane] = ex2_approx(cr1 - c2[128 + cb + lane]);
+                __syncwarp();
+            }
+            mbar_wait(&bar_g, t & 1);
+            tc_fence_after();
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time
+                uint32_t w0[8], w1[8];
+                if (cq > q4) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) w0[i] = w1[i] = 0u;
+                } else {
+                    uint32_t gr[16];
+                    tmem_ld16_async(tm_g + lane_off + cb + 16 * hf, gr);
+                    // the 16 column values of both heads, as broadcast vector loads
+                    float cl0[16], cl1[16];
+                    const float* src0 = (cq == q4) ? c2 + cb + 16 * hf : &colf[warp][0][16 * hf];
+                    const float* src1 = (cq == q4) ? c2 + 128 + cb + 16 * hf : &colf[warp][1][16 * hf];
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const float4 a = *reinterpret_cast<const float4*>(src0 + 4 * v4);
+                        const float4 bq = *reinterpret_cast<const float4*>(src1 + 4 * v4);
+                        cl0[4 * v4] = a.x; cl0[4 * v4 + 1] = a.y; cl0[4 * v4 + 2] = a.z; cl0[4 * v4 + 3] = a.w;
+                        cl1[4 * v4] = bq.x; cl1[4 * v4 + 1] = bq.y; cl1[4 * v4 + 2] = bq.z; cl1[4 * v4 + 3] = bq.w;
+                    }
+                    tmem_wait_ld();
+                    if (cq == q4) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float a0[2], a1[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int l = cb + 16 * hf + 2 * i + e;
+                                const bool ok = l <= m;
+                                const float gg = __uint_as_float(gr[2 * i + e]);
+                                a0[e] = ok ? gg * ex2_approx(ck0 - cl0[2 * i + e]) : 0.f;
+                                a1[e] = ok ? gg * ex2_approx(ck1 - cl1[2 * i + e]) : 0.f;
+                            }
+                            w0[i] = pack_bf16(a0[0], a0[1]);
+                            w1[i] = pack_bf16(a1[0], a1[1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
+                            w0[i] = pack_bf16(g0 * rf0 * cl0[2 * i], g1 * rf0 * cl0[2 * i + 1]);
+                            w1[i] = pack_bf16(g0 * rf1 * cl1[2 * i], g1 * rf1 * cl1[2 * i + 1]);
+                        }
+                    }
+                }
+                // head h's packed L o G occupies columns [64 h, 64 h + 64) of the region
+                tmem_st8(tm_lg + lane_off + 16 * cq + 8 * hf, w0);
+                tmem_st8(tm_lg + lane_off + 64 + 16 * cq + 8 * hf, w1);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            signal(&bar_lg);
         };
         auto piece_id = [&](int ts) -> int { return seq_idx ? seq_s[ts - s0] : 0; };
         auto seq_ends_at = [&](int pend) -> bool {  // does the sequence of token pend-1 end there?
@@ -554,7 +651,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             return seq_idx ? seq_clamped(seq_idx, row, pend, d.nseq) != seq_s[pend - 1 - s0] : false;
         };
 
-        // initial state of the first piece
+        // ---- prologue: the first piece's state, tile 0's cumsum and L o G ----
         {
             const Tile t0 = unpack_tile(tiles[0]);
             const int sid = piece_id(t0.ts);
@@ -564,114 +661,59 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             load_state(src);
             write_hs();
         }
+        float la_next = load_la(1);
         tile_cumsum(0, load_la(0));
         fence_async_shared();
+        tc_fence_before();
         signal(&bar_st);
+        build_lg(0);
 
-        const float dh0 = Dv ? Dv[h0] : 0.f, dh1 = Dv ? Dv[h0 + 1] : 0.f;
+        const int eh = cq >> 1, p0 = 32 * (cq & 1);  // epilogue: head and first p of this thread
+        const float dh = Dv ? Dv[h0 + eh] : 0.f;
         for (int t = 0; t < ntiles; ++t) {
             const uint32_t par = t & 1;
             const int st = t & 1;
             const Tile tl = unpack_tile(tiles[t]);
             const float* c2 = &cs2[t & 1][0][0];
-            const float la_next = (t + 1 < ntiles) ? load_la(t + 1) : 0.f;  // prefetch
+            uint8_t* Xst = smem + S::oX + st * S::kX + eh * kBox;
 
-            // ---- L o G into TMEM (bf16): row m, columns [64 half, 64 half + 64) ----
-            // Per 32x32 sub-block of (rows of this warp) x (columns): above the
-            // diagonal it is 0; on the diagonal exp(c_m - c_l) for l <= m; below
-            // it exp(c_m - c_r0) * exp(c_r0 - c_l) with r0 the warp's first row
-            // (both factors <= 1), so only the diagonal needs one exp per element.
-            mbar_wait(&bar_g, par);
-            tc_fence_after();
-            {
-                const int r0 = 32 * q4;
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int cb = 64 * half + 32 * q;  // first column of this sub-block
-                    uint32_t w0[16], w1[16];
-                    if (cb > r0) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) w0[i] = w1[i] = 0u;
-                    } else {
-                        float gv[32];
-                        tmem_ld32(tm_g + lane_off + cb, gv);
-                        const float ck0 = c2[m], ck1 = c2[128 + m];
-                        if (cb == r0) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                float a0[2], a1[2];
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int l = cb + 2 * i + e;
-                                    const bool ok = l <= m;
-                                    a0[e] = ok ? gv[2 * i + e] * ex2_approx(ck0 - c2[l]) : 0.f;
-                                    a1[e] = ok ? gv[2 * i + e] * ex2_approx(ck1 - c2[128 + l]) : 0.f;
-                                }
-                                w0[i] = pack_bf16(a0[0], a0[1]);
-                                w1[i] = pack_bf16(a1[0], a1[1]);
-                            }
-                        } else {
-                            const float cr0 = c2[r0], cr1 = c2[128 + r0];
-                            const float rf0 = ex2_approx(ck0 - cr0), rf1 = ex2_approx(ck1 - cr1);
-                            const float cf0 = ex2_approx(cr0 - c2[cb + lane]);  // column cb + lane
-                            const float cf1 = ex2_approx(cr1 - c2[128 + cb + lane]);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float f00 = __shfl_sync(0xffffffffu, cf0, 2 * i);
-                                const float f01 = __shfl_sync(0xffffffffu, cf0, 2 * i + 1);
-                                const float f10 = __shfl_sync(0xffffffffu, cf1, 2 * i);
-                                const float f11 = __shfl_sync(0xffffffffu, cf1, 2 * i + 1);
-                                w0[i] = pack_bf16(gv[2 * i] * rf0 * f00, gv[2 * i + 1] * rf0 * f01);
-                                w1[i] = pack_bf16(gv[2 * i] * rf1 * f10, gv[2 * i + 1] * rf1 * f11);
-                            }
-                        }
-                    }
-                    // head h's packed L o G occupies columns [64 h, 64 h + 64) of the
-                    // region (element l at column l / 2): columns cb/2 .. cb/2 + 15
-                    tmem_st16(tm_ls + lane_off + cb / 2, w0);
-                    tmem_st16(tm_ls + lane_off + 64 + cb / 2, w1);
-                }
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            signal(&bar_lg);
-
-            // ---- epilogue: Y = Y_diag + rscale Y_off + D x, and X' = w X in place ----
+            // ---- epilogue(t): Y staged in Hs (or stored), X' = w X in place ----
             mbar_wait(&bar_yd, par);
             mbar_wait(&bar_yo, par);
             tc_fence_after();
             {
-                const int hh = half;  // this warp's head
-                const float ck = c2[128 * hh + m];
-                const float cend = c2[128 * hh + tl.v - 1];
+                const float ck = c2[128 * eh + m];
+                const float cend = c2[128 * eh + tl.v - 1];
                 const float rs = ex2_approx(ck);                           // decay from the tile start
                 const float wx = m < tl.v ? ex2_approx(cend - ck) : 0.f;  // decay to the tile end
-                const float dh = hh ? dh1 : dh0;
-                uint8_t* Xst = smem + S::oX + st * S::kX + hh * kBox;
-                __nv_bfloat16* yrow = Y + ((row + tl.ts + m) * d.nheads + h0 + hh) * (int64_t)kP;
+                const __nv_bfloat162 wx2 = __floats2bfloat162_rn(wx, wx);
+                __nv_bfloat16* yrow = Y + ((row + tl.ts + m) * d.nheads + h0 + eh) * (int64_t)kP + p0;
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float yd[32], yo[32];
-                    tmem_ld32(tm_yd + lane_off + 64 * hh + 32 * q, yd);
-                    tmem_ld32(tm_yo + lane_off + 64 * hh + 32 * q, yo);
+                for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time
+                    uint32_t yd[16], yo[16];
+                    tmem_ld16_async(tm_yd + lane_off + 32 * cq + 16 * hf, yd);
+                    tmem_ld16_async(tm_yos + lane_off + 32 * cq + 16 * hf, yo);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int c16 = 4 * q + c;
+                    for (int c = 0; c < 2; ++c) {
+                        const int c16 = (p0 >> 3) + 2 * hf + c;
                         const uint32_t off = sw128_off(m, c16);
                         uint4 xv = *reinterpret_cast<const uint4*>(Xst + off);
                         uint32_t* xu = reinterpret_cast<uint32_t*>(&xv);
                         uint32_t out[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xu[i]));
+                            const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&xu[i]);
+                            const float2 xf = __bfloat1622float2(xb);
                             const int e0 = 8 * c + 2 * i;
-                            out[i] = pack_bf16(fmaf(dh, xf.x, fmaf(rs, yo[e0], yd[e0])),
-                                               fmaf(dh, xf.y, fmaf(rs, yo[e0 + 1], yd[e0 + 1])));
-                            xu[i] = pack_bf16(xf.x * wx, xf.y * wx);
+                            out[i] = pack_bf16(fmaf(dh, xf.x, fmaf(rs, __uint_as_float(yo[e0]), __uint_as_float(yd[e0]))),
+                                               fmaf(dh, xf.y, fmaf(rs, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1]))));
+                            const __nv_bfloat162 xs = __hmul2(xb, wx2);
+                            xu[i] = *reinterpret_cast<const uint32_t*>(&xs);
                         }
                         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
-                        if (tl.v == 128) *reinterpret_cast<uint4*>(HY + hh * kBox + off) = ov;
-                        else if (m < tl.v) *reinterpret_cast<uint4*>(yrow + 8 * c16) = ov;
+                        if (tl.v == 128) *reinterpret_cast<uint4*>(Hs + eh * kBox + off) = ov;  // Y_off(t) has read Hs
+                        else if (m < tl.v) *reinterpret_cast<uint4*>(yrow + 8 * (c16 - (p0 >> 3))) = ov;
                         *reinterpret_cast<uint4*>(Xst + off) = xv;
                     }
                 }
@@ -680,18 +722,31 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             tc_fence_before();
             signal(&bar_epi);
 
-            // ---- state update: H = a(tile) H + S; final states; next piece ----
+            // ---- L o G(t+1) while S(t) runs ----
+            if (t + 1 < ntiles) {
+                tile_cumsum(t + 1, la_next);
+                la_next = load_la(t + 2);
+                build_lg(t + 1);
+            }
+
+            // ---- state(t): H = a(tile) H + S, final states, next piece; Hs once Y(t) has left ----
             mbar_wait(&bar_s, par);
             mbar_wait(&bar_free, par);
             tc_fence_after();
             {
                 const float dec = ex2_approx(c2[128 * sh + tl.v - 1]);
+                if constexpr (NQ == 32) {
+                    uint32_t sv[32];
+                    tmem_ld32_async(tm_yos + lane_off + NQ * cq, sv);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int n0 = 0; n0 < NH; n0 += 32) {
-                    float sv[32];
-                    tmem_ld32(tm_ls + lane_off + half * NH + n0, sv);
+                    for (int i = 0; i < 32; ++i) Hreg[i] = fmaf(dec, Hreg[i], __uint_as_float(sv[i]));
+                } else {
+                    uint32_t sv[16];
+                    tmem_ld16_async(tm_yos + lane_off + NQ * cq, sv);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) Hreg[n0 + i] = fmaf(dec, Hreg[n0 + i], sv[i]);
+                    for (int i = 0; i < 16; ++i) Hreg[i] = fmaf(dec, Hreg[i], __uint_as_float(sv[i]));
                 }
                 if (tl.last) {
                     const int pend = tl.ts + tl.v;
@@ -699,7 +754,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     if (final_states && seq_ends_at(pend)) {
                         float* f = final_states + seqst_off(d, b, sid, h0 + sh);
 #pragma unroll
-                        for (int i = 0; i < NH; ++i) f[(int64_t)(half * NH + i) * kP + sp] = Hreg[i];
+                        for (int i = 0; i < NQ; ++i) f[(int64_t)(cq * NQ + i) * kP + sp] = Hreg[i];
                     }
                     if (t + 1 < ntiles) {  // the next piece starts a new sequence
                         const Tile tn = unpack_tile(tiles[t + 1]);
@@ -708,19 +763,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
                 write_hs();
             }
-            if (t + 1 < ntiles) tile_cumsum(t + 1, la_next);
             fence_async_shared();
             tc_fence_before();
             signal(&bar_st);
         }
         // ids after the row's last sequence never occur: they keep their initial state
         if (final_states && s1 == d.seqlen && seq_idx) {
-            for (int s = lastid_s + 1; s < d.nseq; ++s) {
-                float* f = final_states + seqst_off(d, b, s, h0 + sh);
-                const float* src = init_states ? init_states + seqst_off(d, b, s, h0 + sh) : nullptr;
+            for (int sq = lastid_s + 1; sq < d.nseq; ++sq) {
+                float* f = final_states + seqst_off(d, b, sq, h0 + sh);
+                const float* src = init_states ? init_states + seqst_off(d, b, sq, h0 + sh) : nullptr;
 #pragma unroll
-                for (int i = 0; i < NH; ++i) {
-                    const int64_t o = (int64_t)(half * NH + i) * kP + sp;
+                for (int i = 0; i < NQ; ++i) {
+                    const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
                     f[o] = src ? src[o] : 0.f;
                 }
             }
@@ -731,6 +785,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
 
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// host
+// ---------------------------------------------------------------------------
+namespace {
 
 template <typename K>
 cudaError_t set_smem_attr(K kernel, int bytes, int slot) {
