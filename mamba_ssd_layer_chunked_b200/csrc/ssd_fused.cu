@@ -320,11 +320,13 @@ __device__ __forceinline__ Tile unpack_tile(int2 e) {
 //   epilogue(t):  Y = Y_diag + rscale Y_off + D x, staged (bf16) in the buffer
 //                 of the carried state, which Y_off(t) has finished reading, for
 //                 the TMA store; X' = w X in place in the tile's X buffer;
-//   L o G(t+1):   the next tile's masked C B^T into TMEM (while the tile state
-//                 MMA of tile t runs and Y(t) drains);
-//   state(t):     H <- a H + S and its bf16 copy for the next C H.
-// Tensor memory: G [0,128), L o G [128,256), Y_diag [256,384), and
-// [384,512) holds Y_off, then the tile state S once Y_off has been read.
+//   L o G(t+1):   the next tile's masked C B^T, written over G in TMEM (while
+//                 the tile state MMA of tile t runs and Y(t) drains);
+//   state(t):     the carried state H(t) (in TMEM: the tile state MMA adds
+//                 X'^T B onto it) to bf16 for the next C H and to the final
+//                 states, then pre-scaled by the next tile's decay.
+// Tensor memory: G, then L o G in place [0,128); Y_diag [128,256);
+// Y_off [256,384); the carried state H [384,512) (rows (head, p), N columns).
 template <int N>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
@@ -414,7 +416,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
     __syncthreads();
     const int ntiles = ntiles_s;
-    const uint32_t tm_g = tmem_base, tm_lg = tmem_base + 128, tm_yd = tmem_base + 256, tm_yos = tmem_base + 384;
+    const uint32_t tm_g = tmem_base, tm_lg = tmem_base, tm_yd = tmem_base + 128, tm_yo = tmem_base + 256,
+                   tm_h = tmem_base + 384;
 
     if (warp == kComputeWarps) {
         // =================== control warp: TMA and MMA issue ===================
@@ -463,17 +466,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const Tile tl = unpack_tile(tiles[t]);
                 const uint32_t xa = smem_u32(smem + S::oX + st * S::kX);
                 const uint32_t ba = smem_u32(smem + S::oB + st * S::kB);
-                // Y_off = C Hs once the state before this tile is in Hs
-                mbar_wait(&bar_st, par);
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                    mma_bf16_ss(tm_yos, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ha + off, 16, 1024),
-                                idesc_nn, k > 0 ? 1u : 0u);
-                }
-                mma_commit(&bar_yo);
-                // Y_diag = (L o G) X, A operand from TMEM
+                // Y_diag = (L o G) X, A operand from TMEM: L o G(t) is built before
+                // state(t-1), so this runs while the state update does
                 mbar_wait(&bar_lg, par);
                 tc_fence_after();
 #pragma unroll
@@ -483,16 +477,28 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 64 * hh + 8 * k,
                                     smem_desc_sw128(xa + hh * kBox + k * 2048, kBox, 1024), idesc_ts, k > 0 ? 1u : 0u);
                 mma_commit(&bar_yd);
-                // C is free once G(t) and Y_off(t) have read it; G(t+1) as soon as its operands are in
+                // Y_off = C Hs once the state before this tile is in Hs
+                mbar_wait(&bar_st, par);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
+                    mma_bf16_ss(tm_yo, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ha + off, 16, 1024),
+                                idesc_nn, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&bar_yo);
+                // C is free once G(t) and Y_off(t) have read it; G(t+1) once its
+                // operands are in and Y_diag(t) has read L o G(t) from the same columns
                 if (t + 1 < ntiles) {
                     mbar_wait(&bar_yo, par);
                     load_c(t + 1);
                     mbar_wait(&bar_c, (t + 1) & 1);
                     mbar_wait(&bar_bx[st ^ 1], ((t + 1) >> 1) & 1);
+                    mbar_wait(&bar_yd, par);
                     tc_fence_after();
                     issue_g(t + 1);
                 }
-                // epilogue done: store Y(t) from the staging buffer; tile state S = X'^T B
+                // epilogue done: store Y(t) from the staging buffer; H += X'^T B
                 mbar_wait(&bar_epi, par);
                 tc_fence_after();
                 const bool full = tl.v == 128;
@@ -503,12 +509,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_bf16_ss(tm_yos, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
-                                idesc_st, k > 0 ? 1u : 0u);
+                    mma_bf16_ss(tm_h, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
+                                idesc_st, 1u);
                 mma_commit(&bar_s);
                 if (full) tma_store_wait_read0();
                 mbar_arrive(&bar_free);
-                // this stage is free once the tile state has been computed
+                // this stage is free once the tile state has been added
                 if (t + 2 < ntiles) {
                     mbar_wait(&bar_s, par);
                     load_bx(t + 2);
@@ -522,21 +528,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const int m = 32 * q4 + lane;           // TMEM lane: token row, or (head, p) for states
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
         const int sh = m >> 6, sp = m & 63;     // state row (head, p) of lane m
-        float Hreg[NQ];
 
-        auto load_state = [&](const float* src) {  // src: [N][P] of head sh, or null for zero
-#pragma unroll
-            for (int i = 0; i < NQ; ++i) Hreg[i] = src ? src[(int64_t)(cq * NQ + i) * kP + sp] : 0.f;
-        };
-        auto write_hs = [&]() {  // bf16 state, row m, K-major over n
-#pragma unroll
-            for (int c8 = 0; c8 < NQ / 8; ++c8) {
-                const int n = cq * NQ + 8 * c8;
-                const uint4 u = make_uint4(pack_bf16(Hreg[8 * c8], Hreg[8 * c8 + 1]), pack_bf16(Hreg[8 * c8 + 2], Hreg[8 * c8 + 3]),
-                                           pack_bf16(Hreg[8 * c8 + 4], Hreg[8 * c8 + 5]), pack_bf16(Hreg[8 * c8 + 6], Hreg[8 * c8 + 7]));
-                *reinterpret_cast<uint4*>(Hs + (n >> 6) * kBox + sw128_off(m, (n & 63) >> 3)) = u;
-            }
-        };
         auto signal = [&](uint64_t* bar) {
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
@@ -581,64 +573,100 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int r0 = 32 * q4, cb = 32 * cq;
             const float ck0 = c2[m], ck1 = c2[128 + m];
             float rf0 = 0.f, rf1 = 0.f;
-            if (cq < q4) {
+            if (cq < q4) {  // below the diagonal: ref r0, column factors of this warp's 32 columns
                 const float cr0 = c2[r0], cr1 = c2[128 + r0];
                 rf0 = ex2_approx(ck0 - cr0);
                 rf1 = ex2_approx(ck1 - cr1);
-                colf[warp][0][lane] = ex2_approx(cr0 - c2[cb + lane]);  // column cb + lane
+                colf[warp][0][lane] = ex2_approx(cr0 - c2[cb + lane]);
                 colf[warp][1][lane] = ex2_approx(cr1 - c2[128 + cb + lane]);
+                __syncwarp();
+            } else if (cq == q4) {  // diagonal: lower-left 16x16 quarter, ref = r0 + 15
+                const float cref0 = c2[r0 + 15], cref1 = c2[128 + r0 + 15];
+                rf0 = lane >= 16 ? ex2_approx(ck0 - cref0) : 0.f;
+                rf1 = lane >= 16 ? ex2_approx(ck1 - cref1) : 0.f;
+                if (lane < 16) {
+                    colf[warp][0][lane] = ex2_approx(cref0 - c2[r0 + lane]);
+                    colf[warp][1][lane] = ex2_approx(cref1 - c2[128 + r0 + lane]);
+                }
                 __syncwarp();
             }
             mbar_wait(&bar_g, t & 1);
             tc_fence_after();
+            // this warp's 32 G columns, read by all warps of the lane quarter before
+            // any of them writes L o G over the same columns
+            uint32_t ga[16], gb[16];
+            if (cq <= q4) {
+                tmem_ld16_async(tm_g + lane_off + cb, ga);
+                tmem_ld16_async(tm_g + lane_off + cb + 16, gb);
+                tmem_wait_ld();
+            }
+            named_bar_sync(2 + q4, 128);
+            if (cq > q4) {
+                uint32_t z[8];
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time
-                uint32_t w0[8], w1[8];
-                if (cq > q4) {
+                for (int i = 0; i < 8; ++i) z[i] = 0u;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) w0[i] = w1[i] = 0u;
-                } else {
-                    uint32_t gr[16];
-                    tmem_ld16_async(tm_g + lane_off + cb + 16 * hf, gr);
-                    // the 16 column values of both heads, as broadcast vector loads
-                    float cl0[16], cl1[16];
-                    const float* src0 = (cq == q4) ? c2 + cb + 16 * hf : &colf[warp][0][16 * hf];
-                    const float* src1 = (cq == q4) ? c2 + 128 + cb + 16 * hf : &colf[warp][1][16 * hf];
+                for (int hf = 0; hf < 2; ++hf) {
+                    tmem_st8(tm_lg + lane_off + 16 * cq + 8 * hf, z);
+                    tmem_st8(tm_lg + lane_off + 64 + 16 * cq + 8 * hf, z);
+                }
+            } else if (cq < q4) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time
+                    uint32_t w0[8], w1[8];
+                    const uint32_t* gr = hf ? gb : ga;
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
-                        const float4 a = *reinterpret_cast<const float4*>(src0 + 4 * v4);
-                        const float4 bq = *reinterpret_cast<const float4*>(src1 + 4 * v4);
-                        cl0[4 * v4] = a.x; cl0[4 * v4 + 1] = a.y; cl0[4 * v4 + 2] = a.z; cl0[4 * v4 + 3] = a.w;
-                        cl1[4 * v4] = bq.x; cl1[4 * v4 + 1] = bq.y; cl1[4 * v4 + 2] = bq.z; cl1[4 * v4 + 3] = bq.w;
+                        const float4 a = *reinterpret_cast<const float4*>(&colf[warp][0][16 * hf + 4 * v4]);
+                        const float4 bq = *reinterpret_cast<const float4*>(&colf[warp][1][16 * hf + 4 * v4]);
+                        const float g0 = __uint_as_float(gr[4 * v4]), g1 = __uint_as_float(gr[4 * v4 + 1]);
+                        const float g2 = __uint_as_float(gr[4 * v4 + 2]), g3 = __uint_as_float(gr[4 * v4 + 3]);
+                        w0[2 * v4] = pack_bf16(g0 * rf0 * a.x, g1 * rf0 * a.y);
+                        w0[2 * v4 + 1] = pack_bf16(g2 * rf0 * a.z, g3 * rf0 * a.w);
+                        w1[2 * v4] = pack_bf16(g0 * rf1 * bq.x, g1 * rf1 * bq.y);
+                        w1[2 * v4 + 1] = pack_bf16(g2 * rf1 * bq.z, g3 * rf1 * bq.w);
                     }
-                    tmem_wait_ld();
-                    if (cq == q4) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float a0[2], a1[2];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int l = cb + 16 * hf + 2 * i + e;
-                                const bool ok = l <= m;
-                                const float gg = __uint_as_float(gr[2 * i + e]);
-                                a0[e] = ok ? gg * ex2_approx(ck0 - cl0[2 * i + e]) : 0.f;
-                                a1[e] = ok ? gg * ex2_approx(ck1 - cl1[2 * i + e]) : 0.f;
-                            }
-                            w0[i] = pack_bf16(a0[0], a0[1]);
-                            w1[i] = pack_bf16(a1[0], a1[1]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
-                            w0[i] = pack_bf16(g0 * rf0 * cl0[2 * i], g1 * rf0 * cl0[2 * i + 1]);
-                            w1[i] = pack_bf16(g0 * rf1 * cl1[2 * i], g1 * rf1 * cl1[2 * i + 1]);
-                        }
-                    }
+                    // head h's packed L o G occupies columns [64 h, 64 h + 64) of the region
+                    tmem_st8(tm_lg + lane_off + 16 * cq + 8 * hf, w0);
+                    tmem_st8(tm_lg + lane_off + 64 + 16 * cq + 8 * hf, w1);
                 }
-                // head h's packed L o G occupies columns [64 h, 64 h + 64) of the region
-                tmem_st8(tm_lg + lane_off + 16 * cq + 8 * hf, w0);
-                tmem_st8(tm_lg + lane_off + 64 + 16 * cq + 8 * hf, w1);
+            } else {
+                // Diagonal block. Lanes 0..15 (rows r0..r0+15) own columns r0..r0+15,
+                // lanes 16..31 own r0+16..r0+31: direct exps there (16 per lane and
+                // head, issued as 16 instructions for the whole warp). Lanes 16..31
+                // x columns r0..r0+15: exp(c_m - c_ref) exp(c_ref - c_l); lanes 0..15
+                // x columns r0+16..: above the diagonal.
+                const bool upper = lane < 16;
+                const int own0 = cb + (upper ? 0 : 16);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const float ck = hh ? ck1 : ck0, rf = hh ? rf1 : rf0;
+                    const float* crow = c2 + 128 * hh;
+                    uint32_t o0[8], o1[8];
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const float4 cv = *reinterpret_cast<const float4*>(crow + own0 + 4 * v4);
+                        const float4 fv = *reinterpret_cast<const float4*>(&colf[warp][hh][4 * v4]);
+                        const float cvs[4] = {cv.x, cv.y, cv.z, cv.w};
+                        const float fvs[4] = {fv.x, fv.y, fv.z, fv.w};
+                        float lo[4], hi[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int jj = 4 * v4 + e;
+                            const float gown = __uint_as_float(upper ? ga[jj] : gb[jj]);
+                            const float a = (own0 + jj <= m) ? gown * ex2_approx(ck - cvs[e]) : 0.f;
+                            const float bq = upper ? 0.f : __uint_as_float(ga[jj]) * rf * fvs[e];
+                            lo[e] = upper ? a : bq;  // column cb + jj
+                            hi[e] = upper ? 0.f : a;  // column cb + 16 + jj
+                        }
+                        o0[2 * v4] = pack_bf16(lo[0], lo[1]);
+                        o0[2 * v4 + 1] = pack_bf16(lo[2], lo[3]);
+                        o1[2 * v4] = pack_bf16(hi[0], hi[1]);
+                        o1[2 * v4 + 1] = pack_bf16(hi[2], hi[3]);
+                    }
+                    tmem_st8(tm_lg + lane_off + 64 * hh + 16 * cq, o0);
+                    tmem_st8(tm_lg + lane_off + 64 * hh + 16 * cq + 8, o1);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -651,6 +679,50 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             return seq_idx ? seq_clamped(seq_idx, row, pend, d.nseq) != seq_s[pend - 1 - s0] : false;
         };
 
+        // the state columns [NQ cq, NQ cq + NQ) of lane m, to/from TMEM
+        auto ld_state = [&](float (&v)[NQ]) {
+            if constexpr (NQ == 32) {
+                uint32_t r[32];
+                tmem_ld32_async(tm_h + lane_off + NQ * cq, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+            } else {
+                uint32_t r[16];
+                tmem_ld16_async(tm_h + lane_off + NQ * cq, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+            }
+        };
+        auto st_state_scaled = [&](const float (&v)[NQ], float a) {
+#pragma unroll
+            for (int h16 = 0; h16 < NQ / 16; ++h16) {
+                float w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) w[i] = a * v[16 * h16 + i];
+                tmem_st16f(tm_h + lane_off + NQ * cq + 16 * h16, w);
+            }
+        };
+        auto load_state = [&](float (&v)[NQ], const float* src) {  // src: [N][P] of head sh, or null
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) v[i] = src ? src[(int64_t)(cq * NQ + i) * kP + sp] : 0.f;
+        };
+        auto write_hs = [&](const float (&v)[NQ]) {  // bf16 state, row m, K-major over n
+#pragma unroll
+            for (int c8 = 0; c8 < NQ / 8; ++c8) {
+                const int n = cq * NQ + 8 * c8;
+                const uint4 u = make_uint4(pack_bf16(v[8 * c8], v[8 * c8 + 1]), pack_bf16(v[8 * c8 + 2], v[8 * c8 + 3]),
+                                           pack_bf16(v[8 * c8 + 4], v[8 * c8 + 5]), pack_bf16(v[8 * c8 + 6], v[8 * c8 + 7]));
+                *reinterpret_cast<uint4*>(Hs + (n >> 6) * kBox + sw128_off(m, (n & 63) >> 3)) = u;
+            }
+        };
+        // decay of a whole tile for the head of state lane m (cs2 of that tile must be in)
+        auto tile_decay = [&](int t) -> float {
+            const Tile tl = unpack_tile(tiles[t]);
+            return ex2_approx(cs2[t & 1][sh][tl.v - 1]);
+        };
+
         // ---- prologue: the first piece's state, tile 0's cumsum and L o G ----
         {
             const Tile t0 = unpack_tile(tiles[0]);
@@ -658,11 +730,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const float* src = nullptr;
             if (seg_incoming) src = seg_incoming + (((int64_t)b * nseg + j) * d.nheads + h0 + sh) * (int64_t)N * kP;
             else if (init_states) src = init_states + seqst_off(d, b, sid, h0 + sh);
-            load_state(src);
-            write_hs();
+            float hv[NQ];
+            load_state(hv, src);
+            write_hs(hv);
+            tile_cumsum(0, load_la(0));
+            st_state_scaled(hv, tile_decay(0));
+            tmem_wait_st();
         }
         float la_next = load_la(1);
-        tile_cumsum(0, load_la(0));
         fence_async_shared();
         tc_fence_before();
         signal(&bar_st);
@@ -677,6 +752,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const float* c2 = &cs2[t & 1][0][0];
             uint8_t* Xst = smem + S::oX + st * S::kX + eh * kBox;
 
+            // the next tile's cumsum while Y(t) is computed
+            if (t + 1 < ntiles) {
+                tile_cumsum(t + 1, la_next);
+                la_next = load_la(t + 2);
+            }
             // ---- epilogue(t): Y staged in Hs (or stored), X' = w X in place ----
             mbar_wait(&bar_yd, par);
             mbar_wait(&bar_yo, par);
@@ -692,7 +772,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time
                     uint32_t yd[16], yo[16];
                     tmem_ld16_async(tm_yd + lane_off + 32 * cq + 16 * hf, yd);
-                    tmem_ld16_async(tm_yos + lane_off + 32 * cq + 16 * hf, yo);
+                    tmem_ld16_async(tm_yo + lane_off + 32 * cq + 16 * hf, yo);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
@@ -722,46 +802,34 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             tc_fence_before();
             signal(&bar_epi);
 
-            // ---- L o G(t+1) while S(t) runs ----
-            if (t + 1 < ntiles) {
-                tile_cumsum(t + 1, la_next);
-                la_next = load_la(t + 2);
-                build_lg(t + 1);
-            }
+            // ---- L o G(t+1) while H += X'^T B runs ----
+            if (t + 1 < ntiles) build_lg(t + 1);
 
-            // ---- state(t): H = a(tile) H + S, final states, next piece; Hs once Y(t) has left ----
+            // ---- state(t): H(t) to Hs (bf16) and to the final states; pre-scale for t+1 ----
             mbar_wait(&bar_s, par);
             mbar_wait(&bar_free, par);
             tc_fence_after();
             {
-                const float dec = ex2_approx(c2[128 * sh + tl.v - 1]);
-                if constexpr (NQ == 32) {
-                    uint32_t sv[32];
-                    tmem_ld32_async(tm_yos + lane_off + NQ * cq, sv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) Hreg[i] = fmaf(dec, Hreg[i], __uint_as_float(sv[i]));
-                } else {
-                    uint32_t sv[16];
-                    tmem_ld16_async(tm_yos + lane_off + NQ * cq, sv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) Hreg[i] = fmaf(dec, Hreg[i], __uint_as_float(sv[i]));
-                }
+                float hv[NQ];
+                ld_state(hv);
                 if (tl.last) {
                     const int pend = tl.ts + tl.v;
                     const int sid = piece_id(tl.ts);
                     if (final_states && seq_ends_at(pend)) {
                         float* f = final_states + seqst_off(d, b, sid, h0 + sh);
 #pragma unroll
-                        for (int i = 0; i < NQ; ++i) f[(int64_t)(cq * NQ + i) * kP + sp] = Hreg[i];
+                        for (int i = 0; i < NQ; ++i) f[(int64_t)(cq * NQ + i) * kP + sp] = hv[i];
                     }
                     if (t + 1 < ntiles) {  // the next piece starts a new sequence
                         const Tile tn = unpack_tile(tiles[t + 1]);
-                        load_state(init_states ? init_states + seqst_off(d, b, piece_id(tn.ts), h0 + sh) : nullptr);
+                        load_state(hv, init_states ? init_states + seqst_off(d, b, piece_id(tn.ts), h0 + sh) : nullptr);
                     }
                 }
-                write_hs();
+                if (t + 1 < ntiles) {
+                    write_hs(hv);
+                    st_state_scaled(hv, tile_decay(t + 1));
+                    tmem_wait_st();
+                }
             }
             fence_async_shared();
             tc_fence_before();
