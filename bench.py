@@ -72,7 +72,28 @@ def algorithmic_bytes(w) -> float:
     return by
 
 
-def kernel_model(w, seglen=None):
+def fused_plan(w, wt):
+    """The fused path's work ranges for tiles-per-range wt: (nwork, cut_tokens,
+    ncuts). cut_tokens: tokens x head pairs that segment_state walks (the last
+    piece of every range that ends inside its row); ncuts: ranges that start
+    inside a row (each needs one incoming state per head of its pair)."""
+    b, T, H = w.batch, w.seqlen, w.nheads
+    npairs, nt = H // 2, -(-T // 128)
+    total = b * npairs * nt
+    nwork = -(-total // wt)
+    cut_tokens = ncuts = 0
+    for i in range(nwork):
+        fb, fe = i * wt, min((i + 1) * wt, total)
+        r = (fe - 1) // nt
+        s0, s1 = 128 * max(fb - r * nt, 0), min(128 * (fe - r * nt), T)
+        if s1 < T:
+            cut_tokens += s1 - s0
+        if fb % nt:
+            ncuts += 1
+    return nwork, cut_tokens, ncuts
+
+
+def kernel_model(w, wt=None):
     """Algorithmic bytes and flops per launch of each kernel.
 
     Chunked path (chunk Q):
@@ -83,14 +104,16 @@ def kernel_model(w, seglen=None):
                     final states; 2 N P flops per (b, chunk, h).
       chunk_scan    reads X, B, C, cs, D and the incoming states; writes Y;
                     Q(Q+1)P + 2QNP flops per (b, chunk, h) + Q(Q+1)N per (b, chunk, g).
-    Fused path (segments of `seglen`, tiles of 128):
-      segment_state   reads X, B, log a; writes one fp32 state and one decay per
-                      (b, segment, h); 2 N P flops per token and head.
-      segment_passing reads and writes the segment states; 2 N P flops per
-                      (b, segment, h).
-      fused_scan      reads X, B, C, log a, D, the segment incoming states and
-                      initial states; writes Y and the final states; per (b, tile, h)
-                      128*129 P + 4*128 N P flops, per (b, tile, g) 128*129 N.
+    Fused path (work ranges of wt tiles of 128 over the (batch row, head pair)
+    rows; see fused_plan):
+      segment_state   reads X, B, log a of the last piece of every range that
+                      ends inside a row; writes one fp32 state and one decay per
+                      such range and head; 2 N P flops per token and head walked.
+      segment_passing reads those states and decays, writes one incoming state
+                      per range start inside a row and head; 2 N P flops each.
+      fused_scan      reads X, B, C, log a, D, the incoming states at the cuts and
+                      the initial states; writes Y and the final states; per
+                      (b, tile, h) 128*129 P + 4*128 N P flops, per (b, tile, g) 128*129 N.
     """
     e = _esize(w)
     b, T, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
@@ -109,14 +132,16 @@ def kernel_model(w, seglen=None):
         "chunk_scan": dict(bytes=2 * xb + 2 * bcb + csb + st + init,
                            flops=b * cn * (H * (Q * (Q + 1) * P + 2 * Q * N * P) + G * Q * (Q + 1) * N)),
     }
-    if seglen:
-        nseg = -(-T // seglen)
-        sst = b * nseg * H * N * P * 4
+    if wt:
+        nwork, cut_tokens, ncuts = fused_plan(w, wt)
         ntile = -(-T // 128)
+        st2 = 2 * N * P * 4  # the two heads of a pair
+        walked = cut_tokens * 2  # token x head
         out.update({
-            "segment_state": dict(bytes=xb + bcb + csb + sst + b * nseg * H * 4, flops=b * T * H * 2 * N * P),
-            "segment_passing": dict(bytes=2 * sst + b * nseg * H * 4 + init, flops=b * nseg * H * 2 * N * P),
-            "fused_scan": dict(bytes=2 * xb + 2 * bcb + csb + (sst if nseg > 1 else 0) + init + fin,
+            "segment_state": dict(bytes=walked * (P * e + 4) + cut_tokens * N * e + ncuts * (st2 + 8),
+                                  flops=walked * 2 * N * P),
+            "segment_passing": dict(bytes=ncuts * (2 * st2 + 8), flops=ncuts * 2 * 2 * N * P),
+            "fused_scan": dict(bytes=2 * xb + 2 * bcb + csb + ncuts * st2 + init + fin,
                                flops=b * ntile * (H * (128 * 129 * P + 4 * 128 * N * P) + G * 128 * 129 * N)),
         })
     return out
@@ -381,23 +406,25 @@ def run_ours(args, w):
     sp = ctypes.c_void_p(stream.cuda_stream)
     vp = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
     pr = ctypes.byref(p)
-    seglen = None
+    wt = nwork = None
     if fam == "fused":
-        seglen = ssd.fused_segment_length(p)
-        nseg = -(-T // seglen)
-        sst = wsp[: b * nseg * H * N * P * 4].view(torch.float32)
-        soff = (b * nseg * H * N * P * 4 + 255) // 256 * 256
-        sdec = wsp[soff: soff + b * nseg * H * 4].view(torch.float32)
+        wt = ssd.fused_work_tiles(p)
+        nwork = ssd.fused_work_count(p, wt)
+        stb = nwork * 2 * N * P * 4
+        al = lambda x: (x + 255) // 256 * 256
+        wloc = wsp[:stb].view(torch.float32)
+        win = wsp[al(stb): al(stb) + stb].view(torch.float32)
+        wdec = wsp[2 * al(stb): 2 * al(stb) + nwork * 2 * 4].view(torch.float32)
+        cuts = nwork > 1 and wt % -(-T // 128) != 0
         names, launches = [], []
-        if nseg > 1:
+        if cuts:
             names += ["segment_state", "segment_passing"]
             launches += [
-                lambda: lib.ssd_segment_state(pr, seglen, vp(X), vp(la), vp(B), vp(seq), vp(sst), vp(sdec), sp),
-                lambda: lib.ssd_segment_passing(pr, seglen, vp(sst), vp(sdec), vp(init), vp(seq), sp)]
+                lambda: lib.ssd_segment_state(pr, wt, vp(X), vp(la), vp(B), vp(seq), vp(wloc), vp(wdec), sp),
+                lambda: lib.ssd_segment_passing(pr, wt, vp(wloc), vp(wdec), vp(init), vp(seq), vp(win), sp)]
         names.append("fused_scan")
-        launches.append(lambda: lib.ssd_fused_scan(pr, seglen, vp(X), vp(la), vp(B), vp(C), vp(D),
-                                                   vp(sst) if nseg > 1 else None, vp(init), vp(seq), vp(Y), vp(F),
-                                                   sp))
+        launches.append(lambda: lib.ssd_fused_scan(pr, wt, vp(X), vp(la), vp(B), vp(C), vp(D),
+                                                   vp(win) if cuts else None, vp(init), vp(seq), vp(Y), vp(F), sp))
     else:
         pk = ssd.problem_from(X, B, w.chunk, inputs["nseq"], "tcgen05" if fam == "tcgen05" else "simt")
         pr = ctypes.byref(pk)
@@ -458,7 +485,7 @@ def run_ours(args, w):
     e2e_value, _ = aggregate(units, e0.elapsed_time(e1) / 1e3, dev if ws > 1 else None)
 
     # roofline of the dominant kernel
-    model = kernel_model(w, seglen)
+    model = kernel_model(w, wt)
     dom = max(per_kernel, key=per_kernel.get)
     peaks = load_peaks()
     km = model[dom]
@@ -485,7 +512,8 @@ def run_ours(args, w):
         "pct_bf16_peak": flops / step_s / 1e12 / peaks["bf16_tflops"],
         "pct_hbm": algorithmic_bytes(w) / step_s / 1e9 / peaks["hbm_gbs"],
         "path": fam,
-        "segment_length": seglen,
+        "work_tiles": wt,
+        "work_ranges": nwork,
         "per_kernel_us": {k: v * 1e6 for k, v in per_kernel.items()},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

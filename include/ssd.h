@@ -79,8 +79,8 @@ typedef enum {
  *            number of heads per group);
  *   FUSED    the two-level path of ssd_segment_state / ssd_segment_passing /
  *            ssd_fused_scan (bf16, headdim 64, dstate 64 or 128, an even number
- *            of heads per group; any chunk): the state crosses HBM once per
- *            segment instead of once per chunk.
+ *            of heads per group; any chunk): the state stays on chip within a
+ *            work range and crosses HBM only where a range boundary cuts a row.
  * AUTO picks FUSED, else TCGEN05, else SIMT, by what the problem allows. An
  * explicit family outside its domain returns SSD_ERR_UNSUPPORTED. */
 typedef enum {
@@ -120,8 +120,8 @@ int ssd_path_supported(const ssd_problem* p, ssd_path path);
 /* Bytes of workspace ssd_fwd needs, or (size_t)-1 if p is invalid: the larger
  * of the chunked paths' need (the chunk cumulative sums, batch*seqlen*nheads
  * fp32, and one state per chunk, batch*nchunks*nheads*dstate*headdim fp32) and
- * the fused path's need (one state and one decay per segment), each part
- * 256-byte aligned. */
+ * the fused path's need (two states and two decays per work range, see
+ * ssd_fused_work_tiles), each part 256-byte aligned. */
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p);
 
 /*
@@ -222,49 +222,62 @@ ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, co
                           void* stream);
 
 /* ---- the fused path: the same block decomposition at two levels ----
- * The sequence axis is cut into segments of `seglen` tokens (a multiple of 128,
- * at most 2048; the last segment may be shorter). Inside a segment the state is
- * carried on chip across 128-token tiles aligned to the sequence starts, so a
- * state goes through HBM once per segment. nseg = ceil(seqlen / seglen); a
- * "segment state buffer" is [batch, nseg, nheads, dstate, headdim] fp32 and a
- * "segment decay buffer" [batch, nseg, nheads] fp32. These entry points cover
- * the FUSED family's domain only (SSD_ERR_UNSUPPORTED elsewhere). */
+ * Each batch row is split into head pairs (heads 2j, 2j+1) and each (batch
+ * row, head pair) "row" into ceil(seqlen / 128) tiles of 128 tokens (the last
+ * may be shorter). The rows' tiles, laid end to end in the order (batch row,
+ * head pair, tile), are cut into `nwork` work ranges of `work_tiles` tiles (the
+ * last may be shorter): nwork = ceil(batch * nheads/2 * ceil(seqlen/128) /
+ * work_tiles). One CTA walks one range and carries the state on chip from
+ * tile to tile; a range may start or end inside a row, and only the states at
+ * those cuts go through HBM. Buffers indexed by range i:
+ *   work_local / work_incoming  [nwork, 2, dstate, headdim] fp32 (the two heads
+ *                               of the row the range ends / starts in)
+ *   work_decay                  [nwork, 2] fp32
+ * These entry points cover the FUSED family's domain only
+ * (SSD_ERR_UNSUPPORTED elsewhere); 1 <= work_tiles <= the number of tiles,
+ * else SSD_ERR_INVALID_ARG. */
 
-/* Segment length ssd_fwd uses for p on the current device (-1 if p is invalid
- * or outside the fused domain). */
-int64_t ssd_fused_segment_length(const ssd_problem* p);
+/* Tiles per range ssd_fwd uses for p on the current device (about one range
+ * per SM), or -1 if p is invalid or outside the fused domain. */
+int64_t ssd_fused_work_tiles(const ssd_problem* p);
 
-/* Right factors per segment: for the segment's last sequence piece [st, s1),
- *   seg_states[b, j, h] = sum_{l in [st, s1)} (prod_{k=l+1..s1-1} a_k) B_l x_l^T
- *   seg_decay[b, j, h]  = prod_{k in [st, s1)} a_k
- * (wq-win section 3, "local_end_state" and "block_decay", for a block that is a
- * segment). */
-ssd_status ssd_segment_state(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a,
-                             const void* B, const int32_t* seq_idx, float* seg_states, float* seg_decay,
+/* nwork for p and work_tiles, or -1 if either is invalid. */
+int64_t ssd_fused_work_count(const ssd_problem* p, int64_t work_tiles);
+
+/* Right factors at the cuts: for every range i whose last piece [s0, s1) ends
+ * inside its row (s1 < seqlen), over the last sequence piece [st, s1) of it:
+ *   work_local[i, j]  = sum_{l in [st, s1)} (prod_{k=l+1..s1-1} a_k) B_l x_l^T
+ *   work_decay[i, j]  = prod_{k in [st, s1)} a_k        (head 2 hp + j)
+ * (wq-win section 3, "local_end_state" and "block_decay", for a block that is
+ * a range's piece). Entries of ranges that end at a row end are not written. */
+ssd_status ssd_segment_state(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a,
+                             const void* B, const int32_t* seq_idx, float* work_local, float* work_decay,
                              void* stream);
 
-/* Centre factors: H_end(j) = seg_decay(j) * H_start(j) + seg_states(j), with
- * H_start(j) = H_end(j-1) when the last piece of segment j continues the
- * sequence of segment j-1, else that sequence's initial state (or zero).
- * Overwrites seg_states[b, j, h] with the state entering segment j for the
- * sequence of its first token: H_end(j-1) when that token continues the
- * sequence of the previous token, else that sequence's initial state (or
- * zero). */
-ssd_status ssd_segment_passing(const ssd_problem* p, int64_t seglen, float* seg_states,
-                               const float* seg_decay, const float* init_states,
-                               const int32_t* seq_idx, void* stream);
+/* Centre factors: over the pieces of each row in order, H_end = decay *
+ * H_start + local for every piece that ends inside the row, with H_start =
+ * H_end of the previous piece when the piece's last sequence continues from
+ * it, else that sequence's initial state (or zero). For every range i whose
+ * first piece starts inside its row, writes work_incoming[i, j]: the state
+ * entering that piece for the sequence of its first token (H_end of the
+ * previous piece when that token continues the previous token's sequence,
+ * else its initial state or zero). Other entries are not written. */
+ssd_status ssd_segment_passing(const ssd_problem* p, int64_t work_tiles, const float* work_local,
+                               const float* work_decay, const float* init_states,
+                               const int32_t* seq_idx, float* work_incoming, void* stream);
 
-/* Per segment: walks 128-token tiles aligned to sequence starts; per tile
+/* Per range: walks 128-token tiles aligned to sequence starts; per tile
  *   y_k = sum_{l <= k in tile} exp(cs_k - cs_l) (C_k . B_l) x_l + exp(cs_k) C_k^T H + D_h x_k
  *   H  <- exp(cs_end) H + sum_{l in tile} exp(cs_end - cs_l) B_l x_l^T
- * starting from seg_incoming[b, j, h] (the output of ssd_segment_passing) for
- * the segment's first sequence and from the initial state (or zero) for every
- * sequence that starts later in the segment;
- * writes Y and, when non-NULL, final_states for every sequence that ends in
- * the segment (and the initial state for ids after the row's last sequence).
- * seg_incoming may be NULL when seqlen <= seglen. */
-ssd_status ssd_fused_scan(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a,
-                          const void* B, const void* C, const float* D, const float* seg_incoming,
+ * starting from work_incoming[i] (the output of ssd_segment_passing) when the
+ * range starts inside a row, and from the initial state (or zero) for every
+ * sequence that starts in the range; writes Y and, when non-NULL,
+ * final_states for every sequence that ends in the range (and the initial
+ * state for ids after a row's last sequence). work_incoming may be NULL when
+ * no range starts inside a row (nwork == 1, or work_tiles a multiple of
+ * ceil(seqlen / 128)). */
+ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a,
+                          const void* B, const void* C, const float* D, const float* work_incoming,
                           const float* init_states, const int32_t* seq_idx, void* Y,
                           float* final_states, void* stream);
 

@@ -18,7 +18,8 @@ from .ssd import (  # noqa: F401
     chunk_state,
     declared_functions,
     fused_scan,
-    fused_segment_length,
+    fused_work_count,
+    fused_work_tiles,
     segment_passing,
     segment_state,
     lib,

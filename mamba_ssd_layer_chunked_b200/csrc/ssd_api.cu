@@ -169,60 +169,68 @@ size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
     size_t need = chunked_workspace_bytes(p);
     if (ssd::fused_supported(p)) {
         const ssd::Dims d = make_dims(p);
-        const size_t f = ssd::fused_workspace_bytes(d, ssd::fused_default_seglen(d));
+        const size_t f = ssd::fused_workspace_bytes(d, ssd::fused_default_work_tiles(d));
         if (f > need) need = f;
     }
     return need;
 }
 
-int64_t ssd_fused_segment_length(const ssd_problem* p) {
+int64_t ssd_fused_work_tiles(const ssd_problem* p) {
     if (check_dims(p) != SSD_OK || !ssd::fused_supported(p)) return -1;
-    return ssd::fused_default_seglen(make_dims(p));
+    return ssd::fused_default_work_tiles(make_dims(p));
 }
 
-ssd_status ssd_segment_state(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a,
-                             const void* B, const int32_t* seq_idx, float* seg_states, float* seg_decay,
+int64_t ssd_fused_work_count(const ssd_problem* p, int64_t work_tiles) {
+    if (check_dims(p) != SSD_OK) return -1;
+    const ssd::Dims d = make_dims(p);
+    if (!ssd::fused_work_ok(d, work_tiles)) return -1;
+    return ssd::fused_work_count(d, work_tiles);
+}
+
+ssd_status ssd_segment_state(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a,
+                             const void* B, const int32_t* seq_idx, float* work_local, float* work_decay,
                              void* stream) {
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
-    if (!X || !log_a || !B || !seg_states || !seg_decay) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, seq_idx, seg_states, seg_decay)) return SSD_ERR_INVALID_ARG;
+    if (!X || !log_a || !B || !work_local || !work_decay) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, log_a, B, seq_idx, work_local, work_decay)) return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = make_dims(p);
-    if (!ssd::fused_seglen_ok(d, seglen)) return SSD_ERR_INVALID_ARG;
+    if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
     if ((s = check_device()) != SSD_OK) return s;
     if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
-    return cuda_status(ssd::launch_segment_state(d, (int)seglen, X, log_a, B, seq_idx, seg_states, seg_decay,
+    return cuda_status(ssd::launch_segment_state(d, work_tiles, X, log_a, B, seq_idx, work_local, work_decay,
                                                  (cudaStream_t)stream));
 }
 
-ssd_status ssd_segment_passing(const ssd_problem* p, int64_t seglen, float* seg_states, const float* seg_decay,
-                               const float* init_states, const int32_t* seq_idx, void* stream) {
+ssd_status ssd_segment_passing(const ssd_problem* p, int64_t work_tiles, const float* work_local,
+                               const float* work_decay, const float* init_states, const int32_t* seq_idx,
+                               float* work_incoming, void* stream) {
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
-    if (!seg_states || !seg_decay) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(seg_states, seg_decay, init_states, seq_idx)) return SSD_ERR_INVALID_ARG;
+    if (!work_local || !work_decay || !work_incoming) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(work_local, work_decay, init_states, seq_idx, work_incoming)) return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = make_dims(p);
-    if (!ssd::fused_seglen_ok(d, seglen)) return SSD_ERR_INVALID_ARG;
+    if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
     if ((s = check_device()) != SSD_OK) return s;
     if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
-    return cuda_status(ssd::launch_segment_passing(d, (int)seglen, seg_states, seg_decay, init_states, seq_idx,
-                                                   (cudaStream_t)stream));
+    return cuda_status(ssd::launch_segment_passing(d, work_tiles, work_local, work_decay, init_states, seq_idx,
+                                                   work_incoming, (cudaStream_t)stream));
 }
 
-ssd_status ssd_fused_scan(const ssd_problem* p, int64_t seglen, const void* X, const float* log_a, const void* B,
-                          const void* C, const float* D, const float* seg_incoming, const float* init_states,
+ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a, const void* B,
+                          const void* C, const float* D, const float* work_incoming, const float* init_states,
                           const int32_t* seq_idx, void* Y, float* final_states, void* stream) {
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
-    if (p->seqlen > seglen && !seg_incoming) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, C, D, seg_incoming, init_states, seq_idx, Y, final_states))
+    if (!all_aligned(X, log_a, B, C, D, work_incoming, init_states, seq_idx, Y, final_states))
         return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = make_dims(p);
-    if (!ssd::fused_seglen_ok(d, seglen)) return SSD_ERR_INVALID_ARG;
+    if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
+    if (ssd::fused_needs_cut_states(d, work_tiles) && !work_incoming) return SSD_ERR_INVALID_ARG;
     if ((s = check_device()) != SSD_OK) return s;
     if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
-    return cuda_status(ssd::launch_fused_scan(d, (int)seglen, X, log_a, B, C, D, seg_incoming, init_states, seq_idx,
+    return cuda_status(ssd::launch_fused_scan(d, work_tiles, X, log_a, B, C, D, work_incoming, init_states, seq_idx,
                                               Y, final_states, (cudaStream_t)stream));
 }
 
@@ -291,20 +299,22 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
     cudaStream_t st = (cudaStream_t)stream;
     const ssd_path fam = fwd_family(p);
     if (fam == SSD_PATH_FUSED) {
-        const int seglen = ssd::fused_default_seglen(d);
-        const int nseg = (d.seqlen + seglen - 1) / seglen;
-        float* seg_states = static_cast<float*>(workspace);
-        const size_t stb = (size_t)d.batch * nseg * d.nheads * d.dstate * d.headdim * sizeof(float);
-        float* seg_decay = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(stb));
+        const int64_t wt = ssd::fused_default_work_tiles(d);
+        const size_t nwork = (size_t)ssd::fused_work_count(d, wt);
+        const size_t stb = nwork * 2 * d.dstate * d.headdim * sizeof(float);
+        float* work_local = static_cast<float*>(workspace);
+        float* work_in = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(stb));
+        float* work_decay = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * align256(stb));
+        const bool cuts = ssd::fused_needs_cut_states(d, wt);
         cudaError_t e = cudaSuccess;
-        if (nseg > 1) {
-            e = ssd::launch_segment_state(d, seglen, X, log_a, B, seq_idx, seg_states, seg_decay, st);
+        if (cuts) {
+            e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st);
             if (e != cudaSuccess) return cuda_status(e);
-            e = ssd::launch_segment_passing(d, seglen, seg_states, seg_decay, init_states, seq_idx, st);
+            e = ssd::launch_segment_passing(d, wt, work_local, work_decay, init_states, seq_idx, work_in, st);
             if (e != cudaSuccess) return cuda_status(e);
         }
-        e = ssd::launch_fused_scan(d, seglen, X, log_a, B, C, D, nseg > 1 ? seg_states : nullptr, init_states,
-                                   seq_idx, Y, final_states, st);
+        e = ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, cuts ? work_in : nullptr, init_states, seq_idx, Y,
+                                   final_states, st);
         return cuda_status(e);
     }
     float* cs = static_cast<float*>(workspace);

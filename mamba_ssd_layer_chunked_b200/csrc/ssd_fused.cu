@@ -1,19 +1,23 @@
 // ssd_fused.cu -- the fused tensor-core path of the SSD forward (bf16 in, fp32
 // state): the block decomposition applied at two levels.
 //
-// The sequence is cut into segments of L tokens (a multiple of 128). Within a
-// segment a CTA walks 128-token tiles and carries the state on chip from tile
-// to tile; only one state per segment goes through HBM. Three kernels:
+// The rows (batch row, head pair) are laid end to end, each cut into 128-token
+// tiles, and the resulting line of tiles is cut into equal work ranges, one
+// per CTA (about one per SM, so the ranges finish together). Within a range a
+// CTA walks its tiles and carries the state on chip from tile to tile; a range
+// may start or end inside a row, and only the states at those cuts go through
+// HBM. Three kernels:
 //
-//   segment_state    per (batch row, head pair, segment): the end state of the
-//                    segment's last sequence piece from a zero start,
+//   segment_state    per range ending inside a row: the end state of the
+//                    range's last sequence piece from a zero start,
 //                    accumulated over its tiles in TMEM (the right factors of
-//                    the block algorithm at segment level);
-//   segment_passing  the short recurrence over segments (centre factors);
-//   fused_scan       per (batch row, head pair, segment): for each tile the
-//                    masked quadratic term (L o C B^T) X, the carried state read
-//                    out by C, D x, and the carried state update
-//                    H <- a(tile) H + sum_l a(l..end) B_l x_l^T.
+//                    the block algorithm at range level);
+//   segment_passing  the short recurrence over the cuts of each row (centre
+//                    factors), giving the state entering each range that
+//                    starts inside a row;
+//   fused_scan       per range: for each tile the masked quadratic term
+//                    (L o C B^T) X, the carried state read out by C, D x, and
+//                    the carried state update H <- a(tile) H + sum_l a(l..end) B_l x_l^T.
 //
 // Source: "Mamba-2: writing the recurrent state as a structured matrix"
 // (wq-win.github.io/llm/088-mamba2.html), section 3 (block algorithm: local
@@ -24,13 +28,15 @@
 // change the output), so the tiles here are aligned to sequence starts: no tile
 // mixes two sequences.
 //
-// fused_scan is warp-specialised: 8 compute warps (the TMEM lane quarters are
-// shared by warps w and w+4, which split the columns) and one control warp that
-// issues TMA loads/stores and tcgen05.mma, handshaking through mbarriers.
-// Tensor memory (512 columns): G = C B^T [0,128), L o G (bf16, the A operand of
-// a TS-MMA) and later the tile state S [128,256), Y_diag [256,384), Y_off [384,512).
+// fused_scan is warp-specialised: 16 compute warps (warp w reaches the TMEM
+// lane quarter w % 4), one control warp that issues TMA copies and tcgen05.mma,
+// and one decay warp that walks the range ahead of the others and publishes,
+// per tile, its coordinates and the within-tile cumsum of log a; the roles
+// handshake through mbarriers.
 
 #include <cuda.h>
+
+#include <algorithm>
 
 #include "ssd_tc.cuh"
 #include "tc_ptx.cuh"
@@ -63,6 +69,26 @@ __device__ int lower_bound_global(const int32_t* seq_idx, int64_t row, int lo, i
     return lo;
 }
 
+// ---------------------------------------------------------------------------
+// work ranges: rows r = b * npairs + hp, each of nt tiles of 128 tokens; the
+// tiles of all rows in a line, cut into ranges of wt tiles (the last shorter)
+// ---------------------------------------------------------------------------
+struct Work {
+    int npairs, nt, wt, nwork;
+    int64_t total;  // rows * nt
+};
+
+__device__ __forceinline__ int64_t work_begin(const Work& w, int i) { return (int64_t)i * w.wt; }
+__device__ __forceinline__ int64_t work_end(const Work& w, int i) {
+    return min((int64_t)(i + 1) * w.wt, w.total);
+}
+// tokens [s0, s1) of row r that tiles [fb, fe) of the line cover
+__device__ __forceinline__ void row_piece(const Work& w, int seqlen, int64_t fb, int64_t fe, int r, int& s0, int& s1) {
+    const int64_t rb = (int64_t)r * w.nt;
+    s0 = (int)(128 * max(fb - rb, (int64_t)0));
+    s1 = (int)min((int64_t)128 * (fe - rb), (int64_t)seqlen);
+}
+
 // ===========================================================================
 // segment_state
 // ===========================================================================
@@ -71,8 +97,8 @@ constexpr int kSegThreads = 256;
 template <int N>
 __global__ void __launch_bounds__(kSegThreads, 1)
     segment_state_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b, Dims d,
-                         int seglen, int nseg, const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
-                         float* __restrict__ seg_states, float* __restrict__ seg_decay) {
+                         Work wk, const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
+                         float* __restrict__ work_local, float* __restrict__ work_decay) {
     constexpr uint32_t kXB = 2 * kBox, kBB = (N / 64) * kBox;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -85,13 +111,15 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int npairs = d.nheads / 2;
-    int r = blockIdx.x;
-    const int j = r % nseg;
-    r /= nseg;
-    const int hp = r % npairs, b = r / npairs;
+    // the last piece of range i, when it ends inside its row
+    const int i_work = blockIdx.x;
+    const int64_t fe = work_end(wk, i_work);
+    const int r = (int)((fe - 1) / wk.nt);
+    int s0, s1;
+    row_piece(wk, d.seqlen, work_begin(wk, i_work), fe, r, s0, s1);
+    if (s1 >= d.seqlen) return;  // ends at the row end: nothing feeds a next range
+    const int hp = r % wk.npairs, b = r / wk.npairs;
     const int h0 = 2 * hp, g = h0 / d.heads_per_group;
-    const int s0 = j * seglen, s1 = min(d.seqlen, s0 + seglen);
     const int64_t row = (int64_t)b * d.seqlen;
 
     if (tid == 0) {
@@ -207,7 +235,7 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     // epilogue: lane m = (head, p); warps w and w+4 split the N columns
     const int m = 32 * (warp & 3) + lane, half = warp >> 2;
     const int eh = m >> 6, p = m & 63;
-    float* dst = seg_states + (((int64_t)b * nseg + j) * d.nheads + h0 + eh) * (int64_t)N * kP;
+    float* dst = work_local + ((int64_t)i_work * 2 + eh) * N * kP;
     const uint32_t lane_addr = tacc + ((uint32_t)(32 * (warp & 3)) << 16);
 #pragma unroll
     for (int n0 = 0; n0 < N / 2; n0 += 32) {
@@ -218,7 +246,7 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     }
     if (tid < 2) {
         const float t = tail_s[tid];
-        seg_decay[((int64_t)b * nseg + j) * d.nheads + h0 + tid] = cut ? 0.f : ex2_approx(t * kLog2e);
+        work_decay[(int64_t)i_work * 2 + tid] = cut ? 0.f : ex2_approx(t * kLog2e);
     }
     tc_fence_before();
     __syncthreads();
@@ -226,18 +254,22 @@ __global__ void __launch_bounds__(kSegThreads, 1)
 }
 
 // ===========================================================================
-// segment_passing: H_end(j) = decay(j) * H_start(j) + S(j) over segments, and
-// over S(j), in place, the state entering segment j for the sequence of its
-// first token: H_end(j-1) when that sequence continues from segment j-1, else
-// its initial state (or zero).
+// segment_passing: per (batch row, head), over the ranges that cover the row
+// in order, H_end = decay * H_start + local for each piece that ends inside
+// the row, with H_start = H_end of the previous piece when the piece's last
+// sequence continues from it, else that sequence's initial state (or zero);
+// and, for each piece that starts inside the row, the state entering it for
+// the sequence of its first token into work_in.
 // ===========================================================================
-__global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, int seglen, int nseg, float* seg_states,
-                                                              const float* __restrict__ seg_decay,
+__global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, Work wk, const float* __restrict__ work_local,
+                                                              const float* __restrict__ work_decay,
                                                               const float* __restrict__ init_states,
-                                                              const int32_t* __restrict__ seq_idx) {
+                                                              const int32_t* __restrict__ seq_idx,
+                                                              float* __restrict__ work_in) {
     __shared__ int info[4];  // last id, last piece continues, first id, first token continues
     const int bh = blockIdx.x;
     const int h = bh % d.nheads, b = bh / d.nheads;
+    const int r = b * wk.npairs + h / 2, hh = h & 1;
     const int NP = d.dstate * d.headdim;
     const int idx = (blockIdx.y * 256 + threadIdx.x) * 4;
     const bool active = idx < NP;
@@ -247,12 +279,15 @@ __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, int seglen
         if (!init_states) return zero;
         return *reinterpret_cast<const float4*>(init_states + seqst_off(d, b, sq, h) + idx);
     };
+    const int64_t rb = (int64_t)r * wk.nt;
+    const int i0 = (int)(rb / wk.wt), i1 = (int)((rb + wk.nt - 1) / wk.wt);
     float4 H = zero;
-    for (int j = 0; j < nseg; ++j) {
-        const int s0 = j * seglen, s1 = min(d.seqlen, s0 + seglen);
+    for (int i = i0; i <= i1; ++i) {
+        int s0, s1;
+        row_piece(wk, d.seqlen, work_begin(wk, i), work_end(wk, i), r, s0, s1);
         __syncthreads();
         if (threadIdx.x == 0) {
-            int sl = 0, cont_last = (j > 0), sf = 0, cont_first = (j > 0);
+            int sl = 0, cont_last = (s0 > 0), sf = 0, cont_first = (s0 > 0);
             if (seq_idx) {
                 sl = seq_clamped(seq_idx, row, s1 - 1, d.nseq);
                 sf = seq_clamped(seq_idx, row, s0, d.nseq);
@@ -267,13 +302,15 @@ __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, int seglen
             info[3] = cont_first;
         }
         __syncthreads();
-        float* S = seg_states + ((int64_t)b * nseg + j) * d.nheads * (int64_t)NP + (int64_t)h * NP;
-        const float dec = seg_decay[((int64_t)b * nseg + j) * d.nheads + h];
         if (!active) continue;
-        const float4 s = *reinterpret_cast<const float4*>(S + idx);
-        *reinterpret_cast<float4*>(S + idx) = info[3] ? H : init_of(info[2]);
-        const float4 st = info[1] ? H : init_of(info[0]);
-        H = make_float4(fmaf(dec, st.x, s.x), fmaf(dec, st.y, s.y), fmaf(dec, st.z, s.z), fmaf(dec, st.w, s.w));
+        const int64_t o = ((int64_t)i * 2 + hh) * NP + idx;
+        if (s0 > 0) *reinterpret_cast<float4*>(work_in + o) = info[3] ? H : init_of(info[2]);
+        if (s1 < d.seqlen) {
+            const float dec = work_decay[(int64_t)i * 2 + hh];
+            const float4 sv = *reinterpret_cast<const float4*>(work_local + o);
+            const float4 st = info[1] ? H : init_of(info[0]);
+            H = make_float4(fmaf(dec, st.x, sv.x), fmaf(dec, st.y, sv.y), fmaf(dec, st.z, sv.z), fmaf(dec, st.w, sv.w));
+        }
     }
 }
 
@@ -282,7 +319,9 @@ __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, int seglen
 // ===========================================================================
 constexpr int kComputeWarps = 16;
 constexpr int kComputeThreads = 32 * kComputeWarps;
-constexpr int kFusedThreads = kComputeThreads + 32;  // + one control warp
+constexpr int kFusedThreads = kComputeThreads + 64;  // + the MMA/TMA control warp and the decay warp
+constexpr int kCsBufs = 4;                           // decay buffers in flight
+constexpr bool kPermRows = false;                     // balanced row order of C (see row_token)
 
 template <int N>
 struct FusedSmem {
@@ -294,27 +333,51 @@ struct FusedSmem {
     static constexpr uint32_t oC = 0, oB = kC, oX = oB + 2 * kB, oH = oX + 2 * kX, oTail = oH + kHY;
 };
 
-// One tile: first token, valid rows, and flags.
-struct Tile {
-    int ts, v;
-    int first;     // first tile of its sequence piece
-    int last;      // last tile of its sequence piece
+// One tile of a range, as the decay warp publishes it: batch row, head pair,
+// first token, valid rows, the sequence id of its tokens and flags.
+struct TileDesc {
+    int b, hp, ts, v, sid, flags;
+};
+enum : int {
+    kTileLast = 1,      // last tile of its sequence piece in this range
+    kTileSeqEnd = 2,    // ... and the sequence ends there (its final state is due)
+    kTileRowEnd = 4,    // the tile ends its row
+    kTileFinal = 8,     // last tile of the range
+    kTileFromWork = 16  // first tile of a range that starts inside its row
 };
 
-__device__ __forceinline__ Tile unpack_tile(int2 e) {
-    Tile t;
-    t.ts = e.x;
-    t.v = e.y & 0xFF;
-    if (t.v == 0) t.v = 128;
-    t.first = (e.y >> 8) & 1;
-    t.last = (e.y >> 9) & 1;
-    return t;
+// Token of the tile held by TMEM lane m in G, L o G and the Y accumulators.
+// With kPermRows, C is loaded as eight 16-row blocks so that lane quarter q
+// holds tokens [16 q, 16 q + 16) and [112 - 16 q, 128 - 16 q): every quarter
+// then gets the same share of the causal triangle (tensor memory lane quarter
+// q can only be reached from SM sub-partition q).
+__device__ __forceinline__ int row_token(int m) {
+    if (!kPermRows) return m;
+    const int q = m >> 5, i = m & 15;
+    return (m & 16) ? 112 - 16 * q + i : 16 * q + i;
 }
 
+// 16-row block of the tokens held by lane half hi (lanes 16 hi .. 16 hi + 15) of quarter q
+__device__ __forceinline__ int row_block(int q, int hi) {
+    if (!kPermRows) return 2 * q + hi;
+    return hi ? 7 - q : q;
+}
+
+// Per-tile data, written by the decay warp: c[h][k] = log2(e) * the
+// within-tile inclusive cumsum of log a for head h, the whole-tile decays and
+// the tile's descriptor.
+struct __align__(16) CsBuf {
+    float c[2][128];
+    float dec[2];
+    int pad[2];
+    TileDesc td;
+};
+// every buffer's c rows are read and written as float4
+static_assert(sizeof(CsBuf) % 16 == 0, "CsBuf must keep 16-byte alignment in an array");
+
 // Thread layout of the 16 compute warps: warp w owns the TMEM lane quarter
-// w % 4 (rows 32 (w % 4) .. +31) and the column quarter w / 4 of every
-// 128-column accumulator it touches; the four warps of a lane quarter split
-// the columns.
+// w % 4 and the column quarter w / 4 of every 128-column accumulator it
+// touches; the four warps of a lane quarter split the columns.
 //
 // Per tile t the compute warps run, in this order,
 //   epilogue(t):  Y = Y_diag + rscale Y_off + D x, staged (bf16) in the buffer
@@ -325,14 +388,16 @@ __device__ __forceinline__ Tile unpack_tile(int2 e) {
 //   state(t):     the carried state H(t) (in TMEM: the tile state MMA adds
 //                 X'^T B onto it) to bf16 for the next C H and to the final
 //                 states, then pre-scaled by the next tile's decay.
+// The decay warp runs ahead, filling the decay buffers; the control warp
+// issues the TMA copies and the MMAs.
 // Tensor memory: G, then L o G in place [0,128); Y_diag [128,256);
 // Y_off [256,384); the carried state H [384,512) (rows (head, p), N columns).
 template <int N>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, Dims d,
-                      int seglen, int nseg, const float* __restrict__ log_a, const float* __restrict__ Dv,
-                      const float* __restrict__ seg_incoming, const float* __restrict__ init_states,
+                      Work wk, const float* __restrict__ log_a, const float* __restrict__ Dv,
+                      const float* __restrict__ work_in, const float* __restrict__ init_states,
                       const int32_t* __restrict__ seq_idx, __nv_bfloat16* __restrict__ Y,
                       float* __restrict__ final_states) {
     using S = FusedSmem<N>;
@@ -341,28 +406,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     uint8_t* smem = align1024(smem_raw);
     uint8_t* Cs = smem + S::oC;
     uint8_t* Hs = smem + S::oH;
-    int* seq_s = reinterpret_cast<int*>(smem + S::oTail);  // [seglen] ids of the segment (varlen only)
-    int2* tiles = reinterpret_cast<int2*>(seq_s + (seq_idx ? seglen : 0));  // tile list
-    __shared__ __align__(16) float cs2[2][2][128];  // [buffer][head][row]: log2-scaled within-tile cumsum
-    __shared__ __align__(16) float colf[kComputeWarps][2][32];  // per-warp column factors
-    __shared__ float wsum[8];
-    __shared__ int ntiles_s, lastid_s;
+    __shared__ __align__(16) CsBuf csb[kCsBufs];
+    // per-warp column factors of the full L o G blocks, [warp][head][row half][column]
+    // (the second half's 32 entries XOR-swizzled by 4 so that both halves' float4
+    // reads fall in different banks)
+    __shared__ __align__(16) float colf[kComputeWarps][2][2][32];
+    // per-warp factors exp2(c_{r+8} - c_{r+e}), e < 8, of the diagonal blocks [warp][row half][head][e]
+    __shared__ __align__(16) float cf8[kComputeWarps][2][2][8];
     __shared__ __align__(8) uint64_t bar_c, bar_bx[2], bar_g, bar_yo, bar_yd, bar_s, bar_lg, bar_epi, bar_st,
-        bar_free;
+        bar_free, bar_csfull[kCsBufs], bar_csfree[kCsBufs];
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int npairs = d.nheads / 2;
-    int r = blockIdx.x;
-    const int j = r % nseg;
-    r /= nseg;
-    const int hp = r % npairs, b = r / npairs;
-    const int h0 = 2 * hp, g = h0 / d.heads_per_group;
-    const int s0 = j * seglen, s1 = min(d.seqlen, s0 + seglen);
-    const int64_t row = (int64_t)b * d.seqlen;
-    const int L = s1 - s0;
+    const int i_work = blockIdx.x;
 
-    // ---- setup: barriers, TMEM, the segment's ids and tile list ----
+    // ---- setup: barriers, TMEM ----
     if (tid == 0) {
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_b);
@@ -379,43 +437,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         mbar_init(&bar_lg, kComputeWarps);
         mbar_init(&bar_epi, kComputeWarps);
         mbar_init(&bar_st, kComputeWarps);
+        for (int i = 0; i < kCsBufs; ++i) {
+            mbar_init(&bar_csfull[i], 1);
+            mbar_init(&bar_csfree[i], kComputeWarps);
+        }
         mbar_fence_init();
     }
     if (warp == 0) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
-    if (seq_idx)
-        for (int k = tid; k < L; k += kFusedThreads) seq_s[k] = seq_clamped(seq_idx, row, s0 + k, d.nseq);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0) {
-        // tiles aligned to the starts of the sequence pieces of [s0, s1)
-        int n = 0, pos = s0;
-        while (pos < s1) {
-            int pend = s1;
-            if (seq_idx) {  // end of the piece containing pos
-                const int v = seq_s[pos - s0];
-                int lo = pos - s0, hi = L;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (seq_s[mid] <= v) lo = mid + 1;
-                    else hi = mid;
-                }
-                pend = s0 + lo;
-            }
-            for (int ts = pos; ts < pend; ts += 128) {
-                const int v = min(128, pend - ts);
-                tiles[n++] = make_int2(ts, (v & 0xFF) | ((ts == pos) << 8) | ((ts + v == pend) << 9));
-            }
-            pos = pend;
-        }
-        ntiles_s = n;
-        lastid_s = seq_idx ? seq_s[L - 1] : 0;
-    }
-    __syncthreads();
-    const int ntiles = ntiles_s;
     const uint32_t tm_g = tmem_base, tm_lg = tmem_base, tm_yd = tmem_base + 128, tm_yo = tmem_base + 256,
                    tm_h = tmem_base + 384;
 
@@ -425,22 +459,37 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const uint32_t idesc_nn = idesc_bf16(128, 128, false, false);   // K-major A and B
             const uint32_t idesc_ts = idesc_bf16(128, 64, false, true);     // TMEM A, MN-major B
             const uint32_t idesc_st = idesc_bf16(128, N, true, true);       // MN-major A and B
-            auto load_bx = [&](int t) {
-                const Tile tl = unpack_tile(tiles[t]);
-                const int st = t & 1;
+            auto desc = [&](int t) -> TileDesc {
+                mbar_wait(&bar_csfull[t & (kCsBufs - 1)], (t / kCsBufs) & 1);
+                return csb[t & (kCsBufs - 1)].td;
+            };
+            auto load_bx = [&](const TileDesc& td, int st) {
+                const int h0 = 2 * td.hp, g = h0 / d.heads_per_group;
                 uint8_t* Bsg = smem + S::oB + st * S::kB;
                 uint8_t* Xsg = smem + S::oX + st * S::kX;
                 mbar_arrive_expect_tx(&bar_bx[st], S::kB + S::kX);
 #pragma unroll
-                for (int q = 0; q < N / 64; ++q) tma_load_4d(Bsg + q * kBox, &tm_b, &bar_bx[st], 64 * q, g, tl.ts, b);
-                tma_load_4d(Xsg, &tm_x, &bar_bx[st], 0, h0, tl.ts, b);
-                tma_load_4d(Xsg + kBox, &tm_x, &bar_bx[st], 0, h0 + 1, tl.ts, b);
+                for (int q = 0; q < N / 64; ++q)
+                    tma_load_4d(Bsg + q * kBox, &tm_b, &bar_bx[st], 64 * q, g, td.ts, td.b);
+                tma_load_4d(Xsg, &tm_x, &bar_bx[st], 0, h0, td.ts, td.b);
+                tma_load_4d(Xsg + kBox, &tm_x, &bar_bx[st], 0, h0 + 1, td.ts, td.b);
             };
-            auto load_c = [&](int t) {
-                const Tile tl = unpack_tile(tiles[t]);
+            // C rows in the order of row_token: with kPermRows smem rows
+            // [16 s, 16 s + 16) hold the tokens of row_block(s / 2, s % 2)
+            auto load_c = [&](const TileDesc& td) {
+                const int g = 2 * td.hp / d.heads_per_group;
                 mbar_arrive_expect_tx(&bar_c, S::kC);
 #pragma unroll
-                for (int q = 0; q < N / 64; ++q) tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, tl.ts, b);
+                for (int q = 0; q < N / 64; ++q) {
+                    if (kPermRows) {
+#pragma unroll
+                        for (int sblk = 0; sblk < 8; ++sblk)
+                            tma_load_4d(Cs + q * kBox + sblk * 2048, &tm_c, &bar_c, 64 * q, g,
+                                        td.ts + 16 * row_block(sblk >> 1, sblk & 1), td.b);
+                    } else {
+                        tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, td.ts, td.b);
+                    }
+                }
             };
             const uint32_t ca = smem_u32(Cs), ha = smem_u32(Hs);
             auto issue_g = [&](int t) {
@@ -453,17 +502,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
                 mma_commit(&bar_g);
             };
-            load_c(0);
-            load_bx(0);
-            if (ntiles > 1) load_bx(1);
+            TileDesc cur = desc(0), nx = cur;
+            bool has_nx = !(cur.flags & kTileFinal);
+            load_c(cur);
+            load_bx(cur, 0);
+            if (has_nx) {
+                nx = desc(1);
+                load_bx(nx, 1);
+            }
             mbar_wait(&bar_c, 0);
             mbar_wait(&bar_bx[0], 0);
             tc_fence_after();
             issue_g(0);
-            for (int t = 0; t < ntiles; ++t) {
+            for (int t = 0;; ++t) {
                 const int st = t & 1;
                 const uint32_t par = t & 1;
-                const Tile tl = unpack_tile(tiles[t]);
                 const uint32_t xa = smem_u32(smem + S::oX + st * S::kX);
                 const uint32_t ba = smem_u32(smem + S::oB + st * S::kB);
                 // Y_diag = (L o G) X, A operand from TMEM: L o G(t) is built before
@@ -474,7 +527,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 64 * hh + 8 * k,
+                        mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 16 * k + 8 * hh,
                                     smem_desc_sw128(xa + hh * kBox + k * 2048, kBox, 1024), idesc_ts, k > 0 ? 1u : 0u);
                 mma_commit(&bar_yd);
                 // Y_off = C Hs once the state before this tile is in Hs
@@ -489,9 +542,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 mma_commit(&bar_yo);
                 // C is free once G(t) and Y_off(t) have read it; G(t+1) once its
                 // operands are in and Y_diag(t) has read L o G(t) from the same columns
-                if (t + 1 < ntiles) {
+                if (has_nx) {
                     mbar_wait(&bar_yo, par);
-                    load_c(t + 1);
+                    load_c(nx);
                     mbar_wait(&bar_c, (t + 1) & 1);
                     mbar_wait(&bar_bx[st ^ 1], ((t + 1) >> 1) & 1);
                     mbar_wait(&bar_yd, par);
@@ -501,10 +554,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 // epilogue done: store Y(t) from the staging buffer; H += X'^T B
                 mbar_wait(&bar_epi, par);
                 tc_fence_after();
-                const bool full = tl.v == 128;
+                const bool full = cur.v == 128;
                 if (full) {
-                    tma_store_4d(&tm_y, Hs, 0, h0, tl.ts, b);
-                    tma_store_4d(&tm_y, Hs + kBox, 0, h0 + 1, tl.ts, b);
+                    tma_store_4d(&tm_y, Hs, 0, 2 * cur.hp, cur.ts, cur.b);
+                    tma_store_4d(&tm_y, Hs + kBox, 0, 2 * cur.hp + 1, cur.ts, cur.b);
                     tma_store_commit();
                 }
 #pragma unroll
@@ -514,18 +567,144 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 mma_commit(&bar_s);
                 if (full) tma_store_wait_read0();
                 mbar_arrive(&bar_free);
+                if (!has_nx) break;
                 // this stage is free once the tile state has been added
-                if (t + 2 < ntiles) {
+                TileDesc nx2 = nx;
+                const bool has_nx2 = !(nx.flags & kTileFinal);
+                if (has_nx2) {
+                    nx2 = desc(t + 2);
                     mbar_wait(&bar_s, par);
-                    load_bx(t + 2);
+                    load_bx(nx2, st);
                 }
+                cur = nx;
+                nx = nx2;
+                has_nx = has_nx2;
             }
         }
         __syncwarp();
+    } else if (warp == kComputeWarps + 1) {
+        // =================== decay warp ===================
+        // Walks the range's pieces (one per row it covers) in tiles of at most
+        // 128 tokens that never cross a sequence start, one tile ahead of the
+        // buffers it fills. Lane j holds tokens 4j .. 4j+3 of a tile.
+        const int64_t fb = work_begin(wk, i_work), fe = work_end(wk, i_work);
+        int r = (int)(fb / wk.nt);
+        int s0, s1;
+        row_piece(wk, d.seqlen, fb, fe, r, s0, s1);
+        int pos = s0;
+        bool first = true;
+        auto next_tile = [&](TileDesc& td) {
+            const int b = r / wk.npairs, hp = r % wk.npairs;
+            const int64_t row = (int64_t)b * d.seqlen;
+            int v = min(128, s1 - pos);
+            int sid = 0;
+            bool change = false;  // the sequence changes right after the tile
+            if (seq_idx) {
+                sid = seq_clamped(seq_idx, row, pos, d.nseq);
+                // first offset j in [1, min(128, s1 - pos - 1)] whose id differs
+                const int jmax = min(128, s1 - pos - 1);
+                int jm = 1 << 30;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int jj = 4 * lane + 1 + e;
+                    if (jj <= jmax && seq_clamped(seq_idx, row, pos + jj, d.nseq) != sid) jm = min(jm, jj);
+                }
+                jm = __reduce_min_sync(0xffffffffu, jm);
+                if (jm <= jmax) {
+                    v = jm;
+                    change = true;
+                }
+            }
+            const int pend = pos + v;
+            const bool piece_end = pend == s1;
+            const bool last_piece = (int64_t)(r + 1) * wk.nt >= fe;
+            bool seq_end = false;
+            if (pend == d.seqlen) seq_end = true;
+            else if (change) seq_end = true;
+            else if (piece_end && seq_idx) seq_end = seq_clamped(seq_idx, row, pend, d.nseq) != sid;
+            int flags = 0;
+            if (piece_end || change) flags |= kTileLast;
+            if ((piece_end || change) && seq_end) flags |= kTileSeqEnd;
+            if (pend == d.seqlen) flags |= kTileRowEnd;
+            if (piece_end && last_piece) flags |= kTileFinal;
+            if (first && s0 > 0) flags |= kTileFromWork;
+            td.b = b;
+            td.hp = hp;
+            td.ts = pos;
+            td.v = v;
+            td.sid = sid;
+            td.flags = flags;
+            first = false;
+            pos = pend;
+            if (piece_end && !last_piece) {
+                ++r;
+                row_piece(wk, d.seqlen, fb, fe, r, s0, s1);
+                pos = s0;
+            }
+        };
+        auto load4 = [&](const TileDesc& td, float (&v)[2][4]) {
+            const int64_t row = (int64_t)td.b * d.seqlen;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = 4 * lane + e;
+                    v[hh][e] = tok < td.v ? log_a[(row + td.ts + tok) * d.nheads + 2 * td.hp + hh] : 0.f;
+                }
+        };
+        TileDesc cur;
+        next_tile(cur);
+        float lcur[2][4];
+        load4(cur, lcur);
+        for (int t = 0;; ++t) {
+            const bool fin = (cur.flags & kTileFinal) != 0;
+            TileDesc nxt = cur;
+            float lnxt[2][4];
+            if (!fin) {
+                next_tile(nxt);
+                load4(nxt, lnxt);
+            }
+            const int bi = t & (kCsBufs - 1);
+            if (t >= kCsBufs) mbar_wait(&bar_csfree[bi], ((t / kCsBufs) - 1) & 1);
+            const int last = cur.v - 1;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float x0 = lcur[hh][0] * kLog2e;
+                float x1 = fmaf(lcur[hh][1], kLog2e, x0);
+                float x2 = fmaf(lcur[hh][2], kLog2e, x1);
+                float x3 = fmaf(lcur[hh][3], kLog2e, x2);
+                float tot = x3;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, tot, o);
+                    if (lane >= o) tot += y;
+                }
+                const float pre = tot - x3;
+                x0 += pre;
+                x1 += pre;
+                x2 += pre;
+                x3 += pre;
+                *reinterpret_cast<float4*>(&csb[bi].c[hh][4 * lane]) = make_float4(x0, x1, x2, x3);
+                const int el = last & 3;
+                const float mine = el == 0 ? x0 : el == 1 ? x1 : el == 2 ? x2 : x3;
+                const float cend = __shfl_sync(0xffffffffu, mine, last >> 2);
+                if (lane == 0) csb[bi].dec[hh] = ex2_approx(cend);
+            }
+            if (lane == 0) csb[bi].td = cur;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_csfull[bi]);
+            if (fin) break;
+            cur = nxt;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) lcur[hh][e] = lnxt[hh][e];
+        }
     } else {
         // =================== compute warps ===================
         const int q4 = warp & 3, cq = warp >> 2;
-        const int m = 32 * q4 + lane;           // TMEM lane: token row, or (head, p) for states
+        const int m = 32 * q4 + lane;           // TMEM lane
+        const int k = row_token(m);             // its token in G, L o G and Y
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
         const int sh = m >> 6, sp = m & 63;     // state row (head, p) of lane m
 
@@ -533,152 +712,102 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
-        // log a of tile t for (head warp/4, row 32 (warp%4) + lane), warps 0..7; the
-        // load is unconditional (clamped row) so that it does not stall until used
-        auto load_la = [&](int t) -> float {
-            if (warp >= 8 || t >= ntiles) return 0.f;
-            const Tile tl = unpack_tile(tiles[t]);
-            const int hh = warp >> 2, rr = min(32 * (warp & 3) + lane, tl.v - 1);
-            return log_a[(row + tl.ts + rr) * d.nheads + h0 + hh];
-        };
-        // within-tile cumsum of log a * log2(e) for tile t into buffer t & 1
-        auto tile_cumsum = [&](int t, float la_raw) {
-            const int hh = (warp >> 2) & 1, rr = 32 * (warp & 3) + lane;
-            float x = 0.f;
-            if (warp < 8) {
-                const Tile tl = unpack_tile(tiles[t]);
-                x = rr < tl.v ? la_raw * kLog2e : 0.f;
+        auto wait_cs = [&](int t) { mbar_wait(&bar_csfull[t & (kCsBufs - 1)], (t / kCsBufs) & 1); };
+        // L o G of tile t into TMEM over G (bf16 pairs; the 16-token K block k of
+        // head h in columns [16 k + 8 h, 16 k + 8 h + 8)), so that warp w reads its
+        // 32 G columns [32 (w / 4), +32) and writes L o G back over the same columns.
+        // Lane half hi holds the 16-row block rb of tokens; column block c (16
+        // tokens) is zero above rb, exp2(c_k - c_l) masked on the diagonal block, and
+        // below it exp2(c_k - c_{16 rb}) * exp2(c_{16 rb} - c_l), both factors <= 1.
+        // the per-warp column factor tables of tile t (before the wait for Y(t-1))
+        auto lg_tables = [&](int t) {
+            const CsBuf& cs = csb[t & (kCsBufs - 1)];
+            const int l = 32 * cq + lane;
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, o);
-                    if (lane >= o) x += y;
-                }
-                if (lane == 31) wsum[warp] = x;
+            for (int hh = 0; hh < 2; ++hh) {
+                const float cl = cs.c[hh][l];
+                // only columns l < 16 rb are read back (full blocks)
+                colf[warp][hh][0][lane] = ex2_approx(cs.c[hh][16 * row_block(q4, 0)] - cl);
+                colf[warp][hh][1][lane ^ 4] = ex2_approx(cs.c[hh][16 * row_block(q4, 1)] - cl);
             }
-            named_bar_sync(1, kComputeThreads);
-            if (warp < 8) {
-                float pre = 0.f;
-#pragma unroll
-                for (int w = 0; w < 3; ++w)
-                    if (w < (warp & 3)) pre += wsum[4 * hh + w];
-                cs2[t & 1][hh][rr] = x + pre;
+            {
+                const int hf = lane >> 4, hh = (lane >> 3) & 1, e = lane & 7;
+                const int r = 16 * row_block(q4, hf);
+                cf8[warp][hf][hh][e] = ex2_approx(cs.c[hh][r + 8] - cs.c[hh][r + e]);
             }
-            named_bar_sync(1, kComputeThreads);
         };
-        // L o G of tile t into TMEM (bf16): row m, columns [32 cq, 32 cq + 32), both heads.
-        // Above the diagonal block 0; on it exp(c_m - c_l) for l <= m; below it
-        // exp(c_m - c_r0) * exp(c_r0 - c_l) with r0 = 32 q4 (both factors <= 1).
         auto build_lg = [&](int t) {
-            const float* c2 = &cs2[t & 1][0][0];
-            const int r0 = 32 * q4, cb = 32 * cq;
-            const float ck0 = c2[m], ck1 = c2[128 + m];
-            float rf0 = 0.f, rf1 = 0.f;
-            if (cq < q4) {  // below the diagonal: ref r0, column factors of this warp's 32 columns
-                const float cr0 = c2[r0], cr1 = c2[128 + r0];
-                rf0 = ex2_approx(ck0 - cr0);
-                rf1 = ex2_approx(ck1 - cr1);
-                colf[warp][0][lane] = ex2_approx(cr0 - c2[cb + lane]);
-                colf[warp][1][lane] = ex2_approx(cr1 - c2[128 + cb + lane]);
-                __syncwarp();
-            } else if (cq == q4) {  // diagonal: lower-left 16x16 quarter, ref = r0 + 15
-                const float cref0 = c2[r0 + 15], cref1 = c2[128 + r0 + 15];
-                rf0 = lane >= 16 ? ex2_approx(ck0 - cref0) : 0.f;
-                rf1 = lane >= 16 ? ex2_approx(ck1 - cref1) : 0.f;
-                if (lane < 16) {
-                    colf[warp][0][lane] = ex2_approx(cref0 - c2[r0 + lane]);
-                    colf[warp][1][lane] = ex2_approx(cref1 - c2[128 + r0 + lane]);
-                }
-                __syncwarp();
-            }
+            const CsBuf& cs = csb[t & (kCsBufs - 1)];
+            const int hi = lane >> 4, i = lane & 15;
+            const int rb = row_block(q4, hi);
+            const float ck0 = cs.c[0][k], ck1 = cs.c[1][k];
+            const float rf0 = ex2_approx(ck0 - cs.c[0][16 * rb]), rf1 = ex2_approx(ck1 - cs.c[1][16 * rb]);
+            const float rg0 = ex2_approx(ck0 - cs.c[0][16 * rb + 8]), rg1 = ex2_approx(ck1 - cs.c[1][16 * rb + 8]);
+            __syncwarp();
             mbar_wait(&bar_g, t & 1);
             tc_fence_after();
-            // this warp's 32 G columns, read by all warps of the lane quarter before
-            // any of them writes L o G over the same columns
-            uint32_t ga[16], gb[16];
-            if (cq <= q4) {
-                tmem_ld16_async(tm_g + lane_off + cb, ga);
-                tmem_ld16_async(tm_g + lane_off + cb + 16, gb);
+            uint32_t gw[32];  // G columns [32 cq, 32 cq + 32), then L o G over them
+            if (2 * cq <= row_block(q4, 1)) {
+                tmem_ld32_async(tm_g + lane_off + 32 * cq, gw);
                 tmem_wait_ld();
             }
-            named_bar_sync(2 + q4, 128);
-            if (cq > q4) {
-                uint32_t z[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) z[i] = 0u;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    tmem_st8(tm_lg + lane_off + 16 * cq + 8 * hf, z);
-                    tmem_st8(tm_lg + lane_off + 64 + 16 * cq + 8 * hf, z);
-                }
-            } else if (cq < q4) {
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time
-                    uint32_t w0[8], w1[8];
-                    const uint32_t* gr = hf ? gb : ga;
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        const float4 a = *reinterpret_cast<const float4*>(&colf[warp][0][16 * hf + 4 * v4]);
-                        const float4 bq = *reinterpret_cast<const float4*>(&colf[warp][1][16 * hf + 4 * v4]);
-                        const float g0 = __uint_as_float(gr[4 * v4]), g1 = __uint_as_float(gr[4 * v4 + 1]);
-                        const float g2 = __uint_as_float(gr[4 * v4 + 2]), g3 = __uint_as_float(gr[4 * v4 + 3]);
-                        w0[2 * v4] = pack_bf16(g0 * rf0 * a.x, g1 * rf0 * a.y);
-                        w0[2 * v4 + 1] = pack_bf16(g2 * rf0 * a.z, g3 * rf0 * a.w);
-                        w1[2 * v4] = pack_bf16(g0 * rf1 * bq.x, g1 * rf1 * bq.y);
-                        w1[2 * v4 + 1] = pack_bf16(g2 * rf1 * bq.z, g3 * rf1 * bq.w);
-                    }
-                    // head h's packed L o G occupies columns [64 h, 64 h + 64) of the region
-                    tmem_st8(tm_lg + lane_off + 16 * cq + 8 * hf, w0);
-                    tmem_st8(tm_lg + lane_off + 64 + 16 * cq + 8 * hf, w1);
-                }
-            } else {
-                // Diagonal block. Lanes 0..15 (rows r0..r0+15) own columns r0..r0+15,
-                // lanes 16..31 own r0+16..r0+31: direct exps there (16 per lane and
-                // head, issued as 16 instructions for the whole warp). Lanes 16..31
-                // x columns r0..r0+15: exp(c_m - c_ref) exp(c_ref - c_l); lanes 0..15
-                // x columns r0+16..: above the diagonal.
-                const bool upper = lane < 16;
-                const int own0 = cb + (upper ? 0 : 16);
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * cq + cc;  // columns [16 c, 16 c + 16)
+                const uint32_t* g = gw + 16 * cc;
+                uint32_t o[16];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const float ck = hh ? ck1 : ck0, rf = hh ? rf1 : rf0;
-                    const float* crow = c2 + 128 * hh;
-                    uint32_t o0[8], o1[8];
+                    uint32_t* w = o + 8 * hh;
+                    if (c < rb) {
+                        const float rf = hh ? rf1 : rf0;
+                        const float* cf = &colf[warp][hh][hi][0];
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        const float4 cv = *reinterpret_cast<const float4*>(crow + own0 + 4 * v4);
-                        const float4 fv = *reinterpret_cast<const float4*>(&colf[warp][hh][4 * v4]);
-                        const float cvs[4] = {cv.x, cv.y, cv.z, cv.w};
-                        const float fvs[4] = {fv.x, fv.y, fv.z, fv.w};
-                        float lo[4], hi[4];
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            const float4 f = *reinterpret_cast<const float4*>(cf + ((16 * cc + 4 * v4) ^ (4 * hi)));
+                            const uint32_t* g4 = g + 4 * v4;
+                            w[2 * v4] = pack_bf16(__uint_as_float(g4[0]) * rf * f.x, __uint_as_float(g4[1]) * rf * f.y);
+                            w[2 * v4 + 1] = pack_bf16(__uint_as_float(g4[2]) * rf * f.z, __uint_as_float(g4[3]) * rf * f.w);
+                        }
+                    } else if (c == rb) {
+                        // diagonal block as 8x8 quadrants: row i < 8 has columns [0, 8)
+                        // direct (masked); row i >= 8 has [8, 16) direct and [0, 8) as
+                        // exp2(c_k - c_{r+8}) exp2(c_{r+8} - c_l), both factors <= 1
+                        const float ck = hh ? ck1 : ck0, rg = hh ? rg1 : rg0;
+                        const bool lo = i < 8;
+                        const int own = lo ? 0 : 8;
+                        const float* cr = &cs.c[hh][16 * c + own];
+                        const float4 ca = *reinterpret_cast<const float4*>(cr);
+                        const float4 cb = *reinterpret_cast<const float4*>(cr + 4);
+                        const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                        const float4 fa = *reinterpret_cast<const float4*>(&cf8[warp][hi][hh][0]);
+                        const float4 fb = *reinterpret_cast<const float4*>(&cf8[warp][hi][hh][4]);
+                        const float fv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+                        float dv[8], lv[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float gd = __uint_as_float(lo ? g[e] : g[8 + e]);
+                            dv[e] = own + e <= i ? gd * ex2_approx(ck - cv[e]) : 0.f;
+                            lv[e] = lo ? dv[e] : __uint_as_float(g[e]) * rg * fv[e];
+                        }
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int jj = 4 * v4 + e;
-                            const float gown = __uint_as_float(upper ? ga[jj] : gb[jj]);
-                            const float a = (own0 + jj <= m) ? gown * ex2_approx(ck - cvs[e]) : 0.f;
-                            const float bq = upper ? 0.f : __uint_as_float(ga[jj]) * rf * fvs[e];
-                            lo[e] = upper ? a : bq;  // column cb + jj
-                            hi[e] = upper ? 0.f : a;  // column cb + 16 + jj
+                            w[e] = pack_bf16(lv[2 * e], lv[2 * e + 1]);
+                            w[4 + e] = lo ? 0u : pack_bf16(dv[2 * e], dv[2 * e + 1]);
                         }
-                        o0[2 * v4] = pack_bf16(lo[0], lo[1]);
-                        o0[2 * v4 + 1] = pack_bf16(lo[2], lo[3]);
-                        o1[2 * v4] = pack_bf16(hi[0], hi[1]);
-                        o1[2 * v4 + 1] = pack_bf16(hi[2], hi[3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) w[e] = 0u;
                     }
-                    tmem_st8(tm_lg + lane_off + 64 * hh + 16 * cq, o0);
-                    tmem_st8(tm_lg + lane_off + 64 * hh + 16 * cq + 8, o1);
                 }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) gw[16 * cc + e] = o[e];
             }
+            tmem_st32(tm_lg + lane_off + 32 * cq, gw);
             tmem_wait_st();
             tc_fence_before();
             signal(&bar_lg);
         };
-        auto piece_id = [&](int ts) -> int { return seq_idx ? seq_s[ts - s0] : 0; };
-        auto seq_ends_at = [&](int pend) -> bool {  // does the sequence of token pend-1 end there?
-            if (pend < s1) return true;
-            if (pend >= d.seqlen) return true;
-            return seq_idx ? seq_clamped(seq_idx, row, pend, d.nseq) != seq_s[pend - 1 - s0] : false;
-        };
-
         // the state columns [NQ cq, NQ cq + NQ) of lane m, to/from TMEM
         auto ld_state = [&](float (&v)[NQ]) {
             if constexpr (NQ == 32) {
@@ -695,14 +824,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
             }
         };
-        auto st_state_scaled = [&](const float (&v)[NQ], float a) {
+        // scales v in place, then stores it
+        auto st_state_scaled = [&](float (&v)[NQ], float a) {
 #pragma unroll
-            for (int h16 = 0; h16 < NQ / 16; ++h16) {
-                float w[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) w[i] = a * v[16 * h16 + i];
-                tmem_st16f(tm_h + lane_off + NQ * cq + 16 * h16, w);
-            }
+            for (int i = 0; i < NQ; ++i) v[i] *= a;
+            if constexpr (NQ == 32) tmem_st32(tm_h + lane_off + NQ * cq, reinterpret_cast<const uint32_t(&)[32]>(v));
+            else tmem_st16(tm_h + lane_off + NQ * cq, reinterpret_cast<const uint32_t(&)[16]>(v));
         };
         auto load_state = [&](float (&v)[NQ], const float* src) {  // src: [N][P] of head sh, or null
 #pragma unroll
@@ -717,59 +844,60 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 *reinterpret_cast<uint4*>(Hs + (n >> 6) * kBox + sw128_off(m, (n & 63) >> 3)) = u;
             }
         };
-        // decay of a whole tile for the head of state lane m (cs2 of that tile must be in)
-        auto tile_decay = [&](int t) -> float {
-            const Tile tl = unpack_tile(tiles[t]);
-            return ex2_approx(cs2[t & 1][sh][tl.v - 1]);
+
+        // the initial state (or zero) of sequence sid of batch row b for head pair hp
+        auto init_src = [&](int b, int hp, int sid) -> const float* {
+            return init_states ? init_states + seqst_off(d, b, sid, 2 * hp + sh) : nullptr;
         };
 
-        // ---- prologue: the first piece's state, tile 0's cumsum and L o G ----
+        // ---- prologue: the first piece's state and tile 0's L o G ----
+        wait_cs(0);
+        TileDesc cur = csb[0].td;
         {
-            const Tile t0 = unpack_tile(tiles[0]);
-            const int sid = piece_id(t0.ts);
-            const float* src = nullptr;
-            if (seg_incoming) src = seg_incoming + (((int64_t)b * nseg + j) * d.nheads + h0 + sh) * (int64_t)N * kP;
-            else if (init_states) src = init_states + seqst_off(d, b, sid, h0 + sh);
+            const float* src = (cur.flags & kTileFromWork) ? work_in + ((int64_t)i_work * 2 + sh) * N * kP
+                                                           : init_src(cur.b, cur.hp, cur.sid);
             float hv[NQ];
             load_state(hv, src);
             write_hs(hv);
-            tile_cumsum(0, load_la(0));
-            st_state_scaled(hv, tile_decay(0));
+            st_state_scaled(hv, csb[0].dec[sh]);
             tmem_wait_st();
         }
-        float la_next = load_la(1);
         fence_async_shared();
         tc_fence_before();
         signal(&bar_st);
+        lg_tables(0);
         build_lg(0);
 
         const int eh = cq >> 1, p0 = 32 * (cq & 1);  // epilogue: head and first p of this thread
-        const float dh = Dv ? Dv[h0 + eh] : 0.f;
-        for (int t = 0; t < ntiles; ++t) {
+        for (int t = 0;; ++t) {
             const uint32_t par = t & 1;
             const int st = t & 1;
-            const Tile tl = unpack_tile(tiles[t]);
-            const float* c2 = &cs2[t & 1][0][0];
+            const bool fin = (cur.flags & kTileFinal) != 0;
+            const float* ct = csb[t & (kCsBufs - 1)].c[eh];
             uint8_t* Xst = smem + S::oX + st * S::kX + eh * kBox;
+            const int64_t rowt = (int64_t)cur.b * d.seqlen;
+            const float dh = Dv ? Dv[2 * cur.hp + eh] : 0.f;
 
-            // the next tile's cumsum while Y(t) is computed
-            if (t + 1 < ntiles) {
-                tile_cumsum(t + 1, la_next);
-                la_next = load_la(t + 2);
+            // the next tile's column factor tables while Y(t) is computed
+            TileDesc nx = cur;
+            if (!fin) {
+                wait_cs(t + 1);
+                nx = csb[(t + 1) & (kCsBufs - 1)].td;
+                lg_tables(t + 1);
             }
             // ---- epilogue(t): Y staged in Hs (or stored), X' = w X in place ----
             mbar_wait(&bar_yd, par);
             mbar_wait(&bar_yo, par);
             tc_fence_after();
             {
-                const float ck = c2[128 * eh + m];
-                const float cend = c2[128 * eh + tl.v - 1];
-                const float rs = ex2_approx(ck);                           // decay from the tile start
-                const float wx = m < tl.v ? ex2_approx(cend - ck) : 0.f;  // decay to the tile end
+                const float ck = ct[k];
+                const float cend = ct[cur.v - 1];
+                const float rs = ex2_approx(ck);                            // decay from the tile start
+                const float wx = k < cur.v ? ex2_approx(cend - ck) : 0.f;  // decay to the tile end
                 const __nv_bfloat162 wx2 = __floats2bfloat162_rn(wx, wx);
-                __nv_bfloat16* yrow = Y + ((row + tl.ts + m) * d.nheads + h0 + eh) * (int64_t)kP + p0;
+                __nv_bfloat16* yrow = Y + ((rowt + cur.ts + k) * d.nheads + 2 * cur.hp + eh) * (int64_t)kP + p0;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {  // 16 columns at a time
+                for (int hf = 0; hf < 2; ++hf) {
                     uint32_t yd[16], yo[16];
                     tmem_ld16_async(tm_yd + lane_off + 32 * cq + 16 * hf, yd);
                     tmem_ld16_async(tm_yo + lane_off + 32 * cq + 16 * hf, yo);
@@ -777,7 +905,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         const int c16 = (p0 >> 3) + 2 * hf + c;
-                        const uint32_t off = sw128_off(m, c16);
+                        const uint32_t off = sw128_off(k, c16);
                         uint4 xv = *reinterpret_cast<const uint4*>(Xst + off);
                         uint32_t* xu = reinterpret_cast<uint32_t*>(&xv);
                         uint32_t out[4];
@@ -785,15 +913,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         for (int i = 0; i < 4; ++i) {
                             const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&xu[i]);
                             const float2 xf = __bfloat1622float2(xb);
-                            const int e0 = 8 * c + 2 * i;
+                            const int e0 = 8 * c + 2 * i;  // of this half
                             out[i] = pack_bf16(fmaf(dh, xf.x, fmaf(rs, __uint_as_float(yo[e0]), __uint_as_float(yd[e0]))),
                                                fmaf(dh, xf.y, fmaf(rs, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1]))));
                             const __nv_bfloat162 xs = __hmul2(xb, wx2);
                             xu[i] = *reinterpret_cast<const uint32_t*>(&xs);
                         }
                         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
-                        if (tl.v == 128) *reinterpret_cast<uint4*>(Hs + eh * kBox + off) = ov;  // Y_off(t) has read Hs
-                        else if (m < tl.v) *reinterpret_cast<uint4*>(yrow + 8 * (c16 - (p0 >> 3))) = ov;
+                        if (cur.v == 128) *reinterpret_cast<uint4*>(Hs + eh * kBox + off) = ov;  // Y_off(t) has read Hs
+                        else if (k < cur.v) *reinterpret_cast<uint4*>(yrow + 8 * (c16 - (p0 >> 3))) = ov;
                         *reinterpret_cast<uint4*>(Xst + off) = xv;
                     }
                 }
@@ -803,7 +931,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             signal(&bar_epi);
 
             // ---- L o G(t+1) while H += X'^T B runs ----
-            if (t + 1 < ntiles) build_lg(t + 1);
+            if (!fin) build_lg(t + 1);
 
             // ---- state(t): H(t) to Hs (bf16) and to the final states; pre-scale for t+1 ----
             mbar_wait(&bar_s, par);
@@ -812,40 +940,39 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             {
                 float hv[NQ];
                 ld_state(hv);
-                if (tl.last) {
-                    const int pend = tl.ts + tl.v;
-                    const int sid = piece_id(tl.ts);
-                    if (final_states && seq_ends_at(pend)) {
-                        float* f = final_states + seqst_off(d, b, sid, h0 + sh);
+                if (cur.flags & kTileLast) {
+                    if (final_states && (cur.flags & kTileSeqEnd)) {
+                        float* f = final_states + seqst_off(d, cur.b, cur.sid, 2 * cur.hp + sh);
 #pragma unroll
                         for (int i = 0; i < NQ; ++i) f[(int64_t)(cq * NQ + i) * kP + sp] = hv[i];
                     }
-                    if (t + 1 < ntiles) {  // the next piece starts a new sequence
-                        const Tile tn = unpack_tile(tiles[t + 1]);
-                        load_state(hv, init_states ? init_states + seqst_off(d, b, piece_id(tn.ts), h0 + sh) : nullptr);
+                    // the next tile starts a new sequence or a new row
+                    if (!fin) load_state(hv, init_src(nx.b, nx.hp, nx.sid));
+                }
+                // ids after the row's last sequence never occur: they keep their initial state
+                if ((cur.flags & kTileRowEnd) && final_states && seq_idx) {
+                    for (int sq = cur.sid + 1; sq < d.nseq; ++sq) {
+                        float* f = final_states + seqst_off(d, cur.b, sq, 2 * cur.hp + sh);
+                        const float* src = init_src(cur.b, cur.hp, sq);
+#pragma unroll
+                        for (int i = 0; i < NQ; ++i) {
+                            const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
+                            f[o] = src ? src[o] : 0.f;
+                        }
                     }
                 }
-                if (t + 1 < ntiles) {
+                if (!fin) {
                     write_hs(hv);
-                    st_state_scaled(hv, tile_decay(t + 1));
+                    st_state_scaled(hv, csb[(t + 1) & (kCsBufs - 1)].dec[sh]);
                     tmem_wait_st();
                 }
             }
             fence_async_shared();
             tc_fence_before();
             signal(&bar_st);
-        }
-        // ids after the row's last sequence never occur: they keep their initial state
-        if (final_states && s1 == d.seqlen && seq_idx) {
-            for (int sq = lastid_s + 1; sq < d.nseq; ++sq) {
-                float* f = final_states + seqst_off(d, b, sq, h0 + sh);
-                const float* src = init_states ? init_states + seqst_off(d, b, sq, h0 + sh) : nullptr;
-#pragma unroll
-                for (int i = 0; i < NQ; ++i) {
-                    const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
-                    f[o] = src ? src[o] : 0.f;
-                }
-            }
+            signal(&bar_csfree[t & (kCsBufs - 1)]);  // done with tile t's decay data
+            if (fin) break;
+            cur = nx;
         }
     }
     tc_fence_before();
@@ -865,11 +992,9 @@ cudaError_t set_smem_attr(K kernel, int bytes, int slot) {
     return ensure_smem_attr(reinterpret_cast<const void*>(kernel), bytes, slot);
 }
 
-int max_tiles(int seglen, bool varlen) { return varlen ? seglen + seglen / 128 + 2 : seglen / 128 + 2; }
-
 template <int N>
-int fused_smem_bytes(int seglen, bool varlen) {
-    return (int)FusedSmem<N>::oTail + (varlen ? seglen * 4 : 0) + max_tiles(seglen, varlen) * 8 + 1024;
+int fused_smem_bytes() {
+    return (int)FusedSmem<N>::oTail + 1024;
 }
 
 int num_sms() {
@@ -890,6 +1015,16 @@ int num_sms() {
     return n[dev];
 }
 
+Work make_work(const Dims& d, int64_t work_tiles) {
+    Work w;
+    w.npairs = d.nheads / 2;
+    w.nt = (d.seqlen + 127) / 128;
+    w.total = (int64_t)d.batch * w.npairs * w.nt;
+    w.wt = (int)work_tiles;
+    w.nwork = (int)((w.total + work_tiles - 1) / work_tiles);
+    return w;
+}
+
 }  // namespace
 
 bool fused_supported(const ssd_problem* p) {
@@ -899,96 +1034,89 @@ bool fused_supported(const ssd_problem* p) {
     return true;
 }
 
-bool fused_seglen_ok(const Dims& d, int64_t seglen) {
-    (void)d;
-    return seglen >= 128 && seglen <= 2048 && seglen % 128 == 0;
+bool fused_work_ok(const Dims& d, int64_t work_tiles) {
+    const int64_t total = (int64_t)d.batch * (d.nheads / 2) * ((d.seqlen + 127) / 128);
+    if (work_tiles < 1 || work_tiles > total) return false;
+    return (total + work_tiles - 1) / work_tiles <= (int64_t)1 << 30;
 }
 
-// Segment length: balance the waves of fused_scan (one CTA per SM, time per
-// wave proportional to the tiles of a segment) against the per-segment state
-// traffic (about four tiles' worth of bytes per segment, spread over the SMs).
-int fused_default_seglen(const Dims& d) {
-    const int nsm = num_sms();
-    const int64_t pairs = (int64_t)d.batch * (d.nheads / 2);
-    int best = 128;
-    double best_cost = 1e300;
-    for (int L = 128; L <= 2048; L *= 2) {
-        const int64_t nseg = (d.seqlen + L - 1) / L;
-        const int64_t items = pairs * nseg;
-        const double waves = (double)((items + nsm - 1) / nsm);
-        const double tiles = (double)(L < d.seqlen ? L : ((d.seqlen + 127) / 128) * 128) / 128.0;
-        const double cost = waves * tiles + (nseg > 1 ? 4.0 * (double)items / nsm : 0.0);
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = L;
-        }
-        if (L >= d.seqlen) break;
-    }
-    return best;
+int64_t fused_work_count(const Dims& d, int64_t work_tiles) { return make_work(d, work_tiles).nwork; }
+
+bool fused_needs_cut_states(const Dims& d, int64_t work_tiles) {
+    const Work w = make_work(d, work_tiles);
+    return w.nwork > 1 && work_tiles % w.nt != 0;
 }
 
-size_t fused_workspace_bytes(const Dims& d, int seglen) {
-    const size_t nseg = (d.seqlen + seglen - 1) / seglen;
-    const size_t st = (size_t)d.batch * nseg * d.nheads * d.dstate * d.headdim * sizeof(float);
-    const size_t dec = (size_t)d.batch * nseg * d.nheads * sizeof(float);
-    return ((st + 255) & ~size_t(255)) + ((dec + 255) & ~size_t(255));
+// Tiles per work range: the line of tiles split evenly over the SMs (one CTA
+// per SM), so that every CTA has the same number of tiles to walk.
+int fused_default_work_tiles(const Dims& d) {
+    const int64_t total = (int64_t)d.batch * (d.nheads / 2) * ((d.seqlen + 127) / 128);
+    const int64_t g = std::min<int64_t>(num_sms(), total);
+    return (int)((total + g - 1) / g);
 }
 
-cudaError_t launch_segment_state(const Dims& d, int seglen, const void* X, const float* log_a, const void* B,
-                                 const int32_t* seq_idx, float* seg_states, float* seg_decay, cudaStream_t st) {
+size_t fused_workspace_bytes(const Dims& d, int64_t work_tiles) {
+    const size_t nwork = (size_t)make_work(d, work_tiles).nwork;
+    const size_t st = nwork * 2 * d.dstate * d.headdim * sizeof(float);
+    const size_t dec = nwork * 2 * sizeof(float);
+    const auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+    return 2 * al(st) + al(dec);
+}
+
+cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
+                                 const int32_t* seq_idx, float* work_local, float* work_decay, cudaStream_t st) {
     CUtensorMap mx, mb;
     cudaError_t e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
     if ((e = bc_map(&mb, d, B, 128)) != cudaSuccess) return e;
-    const int nseg = (d.seqlen + seglen - 1) / seglen;
-    const dim3 grid(d.batch * (d.nheads / 2) * nseg);
+    const Work w = make_work(d, work_tiles);
+    const dim3 grid(w.nwork);
     const int smem = 2 * (int)kBox + (d.dstate / 64) * (int)kBox + 1024;
     if (d.dstate == 64) {
         auto k = segment_state_kernel<64>;
         if ((e = set_smem_attr(k, smem, 30)) != cudaSuccess) return e;
-        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, seglen, nseg, log_a, seq_idx, seg_states, seg_decay);
+        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay);
     } else if (d.dstate == 128) {
         auto k = segment_state_kernel<128>;
         if ((e = set_smem_attr(k, smem, 31)) != cudaSuccess) return e;
-        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, seglen, nseg, log_a, seq_idx, seg_states, seg_decay);
+        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay);
     } else {
         return cudaErrorNotSupported;
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_segment_passing(const Dims& d, int seglen, float* seg_states, const float* seg_decay,
-                                   const float* init_states, const int32_t* seq_idx, cudaStream_t st) {
-    const int nseg = (d.seqlen + seglen - 1) / seglen;
+cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const float* work_local, const float* work_decay,
+                                   const float* init_states, const int32_t* seq_idx, float* work_in, cudaStream_t st) {
+    const Work w = make_work(d, work_tiles);
     const dim3 grid(d.batch * d.nheads, (d.dstate * d.headdim + 1023) / 1024);
-    segment_passing_kernel<<<grid, 256, 0, st>>>(d, seglen, nseg, seg_states, seg_decay, init_states, seq_idx);
+    segment_passing_kernel<<<grid, 256, 0, st>>>(d, w, work_local, work_decay, init_states, seq_idx, work_in);
     return cudaGetLastError();
 }
 
-cudaError_t launch_fused_scan(const Dims& d, int seglen, const void* X, const float* log_a, const void* B,
-                              const void* C, const float* D, const float* seg_incoming, const float* init_states,
+cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
+                              const void* C, const float* D, const float* work_in, const float* init_states,
                               const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st) {
     CUtensorMap mx, mb, mc, my;
     cudaError_t e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
     if ((e = bc_map(&mb, d, B, 128)) != cudaSuccess) return e;
-    if ((e = bc_map(&mc, d, C, 128)) != cudaSuccess) return e;
+    if ((e = bc_map(&mc, d, C, kPermRows ? 16 : 128)) != cudaSuccess) return e;  // C in 16-row blocks
     if ((e = x_map(&my, d, Y, 128)) != cudaSuccess) return e;
-    const int nseg = (d.seqlen + seglen - 1) / seglen;
-    const dim3 grid(d.batch * (d.nheads / 2) * nseg);
-    const bool varlen = seq_idx != nullptr;
+    const Work w = make_work(d, work_tiles);
+    const dim3 grid(w.nwork);
     if (d.dstate == 64) {
         auto k = fused_scan_kernel<64>;
-        const int smem = fused_smem_bytes<64>(seglen, varlen);
+        const int smem = fused_smem_bytes<64>();
         if ((e = set_smem_attr(k, smem, 32)) != cudaSuccess) return e;
-        k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, seglen, nseg, log_a, D, seg_incoming, init_states,
-                                             seq_idx, (__nv_bfloat16*)Y, final_states);
+        k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx,
+                                             (__nv_bfloat16*)Y, final_states);
     } else if (d.dstate == 128) {
         auto k = fused_scan_kernel<128>;
-        const int smem = fused_smem_bytes<128>(seglen, varlen);
+        const int smem = fused_smem_bytes<128>();
         if ((e = set_smem_attr(k, smem, 33)) != cudaSuccess) return e;
-        k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, seglen, nseg, log_a, D, seg_incoming, init_states,
-                                             seq_idx, (__nv_bfloat16*)Y, final_states);
+        k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx,
+                                             (__nv_bfloat16*)Y, final_states);
     } else {
         return cudaErrorNotSupported;
     }

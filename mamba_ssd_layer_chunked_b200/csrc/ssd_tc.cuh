@@ -25,18 +25,23 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* X, const void* B, co
                                  cudaStream_t st);
 
 // ---- fused path (ssd_fused.cu) ----
+// The rows (batch row, head pair) x 128-token tiles laid end to end, cut into
+// ranges of work_tiles tiles, one CTA each.
 bool fused_supported(const ssd_problem* p);
-// segment length chosen for problem d on the current device (multiple of 128)
-int fused_default_seglen(const Dims& d);
-bool fused_seglen_ok(const Dims& d, int64_t seglen);
-size_t fused_workspace_bytes(const Dims& d, int seglen);
+// tiles per range chosen for problem d on the current device
+int fused_default_work_tiles(const Dims& d);
+bool fused_work_ok(const Dims& d, int64_t work_tiles);
+int64_t fused_work_count(const Dims& d, int64_t work_tiles);
+// true when some range starts inside a row (then the cut states are needed)
+bool fused_needs_cut_states(const Dims& d, int64_t work_tiles);
+size_t fused_workspace_bytes(const Dims& d, int64_t work_tiles);
 
-cudaError_t launch_segment_state(const Dims& d, int seglen, const void* X, const float* log_a, const void* B,
-                                 const int32_t* seq_idx, float* seg_states, float* seg_decay, cudaStream_t st);
-cudaError_t launch_segment_passing(const Dims& d, int seglen, float* seg_states, const float* seg_decay,
-                                   const float* init_states, const int32_t* seq_idx, cudaStream_t st);
-cudaError_t launch_fused_scan(const Dims& d, int seglen, const void* X, const float* log_a, const void* B,
-                              const void* C, const float* D, const float* seg_incoming, const float* init_states,
+cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
+                                 const int32_t* seq_idx, float* work_local, float* work_decay, cudaStream_t st);
+cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const float* work_local, const float* work_decay,
+                                   const float* init_states, const int32_t* seq_idx, float* work_in, cudaStream_t st);
+cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
+                              const void* C, const float* D, const float* work_in, const float* init_states,
                               const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st);
 
 }  // namespace ssd

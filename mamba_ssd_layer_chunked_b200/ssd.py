@@ -61,9 +61,10 @@ def _declare(lib):
         "ssd_chunk_state": ([P, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "ssd_state_passing": ([P, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "ssd_chunk_scan": ([P] + [vp] * 9 + [vp], ctypes.c_int),
-        "ssd_fused_segment_length": ([P], ctypes.c_int64),
+        "ssd_fused_work_tiles": ([P], ctypes.c_int64),
+        "ssd_fused_work_count": ([P, ctypes.c_int64], ctypes.c_int64),
         "ssd_segment_state": ([P, ctypes.c_int64] + [vp] * 7, ctypes.c_int),
-        "ssd_segment_passing": ([P, ctypes.c_int64] + [vp] * 5, ctypes.c_int),
+        "ssd_segment_passing": ([P, ctypes.c_int64] + [vp] * 6, ctypes.c_int),
         "ssd_fused_scan": ([P, ctypes.c_int64] + [vp] * 11, ctypes.c_int),
     }
     for name, (argtypes, restype) in sig.items():
@@ -276,43 +277,53 @@ def chunk_scan(X, B, C, cs, incoming, chunk, D=None, init_states=None, seq_idx=N
 
 # ---- the fused path, one call per kernel -------------------------------------
 
-def fused_segment_length(p: Problem) -> int:
-    """Segment length ssd_fwd uses on the fused path (-1 outside its domain)."""
-    return int(lib().ssd_fused_segment_length(ctypes.byref(p)))
+def fused_work_tiles(p: Problem) -> int:
+    """Tiles per work range ssd_fwd uses on the fused path (-1 outside its domain)."""
+    return int(lib().ssd_fused_work_tiles(ctypes.byref(p)))
+
+
+def fused_work_count(p: Problem, work_tiles: int) -> int:
+    """Number of work ranges for p and work_tiles (-1 if invalid)."""
+    return int(lib().ssd_fused_work_count(ctypes.byref(p), int(work_tiles)))
 
 
 def _fused_problem(X, B, nseq, chunk):
     return problem_from(X, B, chunk, nseq, "fused")
 
 
-def segment_state(X, log_a, B, seglen, seq_idx=None, nseq=1, chunk=64, stream=None):
-    """Right factor per segment: (seg_states [b, nseg, H, N, P], seg_decay [b, nseg, H])."""
+def segment_state(X, log_a, B, work_tiles, seq_idx=None, nseq=1, chunk=64, stream=None):
+    """Right factors at the range cuts: (work_local [nwork, 2, N, P], work_decay [nwork, 2]).
+
+    Entries of ranges that end at a row end are left as allocated (NaN here)."""
     p = _fused_problem(X, B, nseq, chunk)
-    b, T, H, P = X.shape
-    N = B.shape[3]
-    nseg = (T + seglen - 1) // seglen
-    st = torch.empty((b, nseg, H, N, P), dtype=torch.float32, device=X.device)
-    dec = torch.empty((b, nseg, H), dtype=torch.float32, device=X.device)
-    _check(lib().ssd_segment_state(ctypes.byref(p), seglen, _ptr(X), _ptr(log_a), _ptr(B), _ptr(seq_idx), _ptr(st),
-                                   _ptr(dec), _stream(stream)), "ssd_segment_state")
-    return st, dec
+    nwork = fused_work_count(p, work_tiles)
+    if nwork < 0:
+        raise ValueError(f"invalid work_tiles {work_tiles}")
+    N, P = B.shape[3], X.shape[3]
+    loc = torch.full((nwork, 2, N, P), float("nan"), dtype=torch.float32, device=X.device)
+    dec = torch.full((nwork, 2), float("nan"), dtype=torch.float32, device=X.device)
+    _check(lib().ssd_segment_state(ctypes.byref(p), int(work_tiles), _ptr(X), _ptr(log_a), _ptr(B), _ptr(seq_idx),
+                                   _ptr(loc), _ptr(dec), _stream(stream)), "ssd_segment_state")
+    return loc, dec
 
 
-def segment_passing(seg_states, seg_decay, X, B, seglen, init_states=None, seq_idx=None, nseq=1, chunk=64,
+def segment_passing(work_local, work_decay, X, B, work_tiles, init_states=None, seq_idx=None, nseq=1, chunk=64,
                     stream=None):
-    """State entering each segment, written over seg_states (returned)."""
+    """State entering each range that starts inside a row: [nwork, 2, N, P] (NaN elsewhere)."""
     p = _fused_problem(X, B, nseq, chunk)
-    _check(lib().ssd_segment_passing(ctypes.byref(p), seglen, _ptr(seg_states), _ptr(seg_decay), _ptr(init_states),
-                                     _ptr(seq_idx), _stream(stream)), "ssd_segment_passing")
-    return seg_states
+    inc = torch.full_like(work_local, float("nan"))
+    _check(lib().ssd_segment_passing(ctypes.byref(p), int(work_tiles), _ptr(work_local), _ptr(work_decay),
+                                     _ptr(init_states), _ptr(seq_idx), _ptr(inc), _stream(stream)),
+           "ssd_segment_passing")
+    return inc
 
 
-def fused_scan(X, log_a, B, C, seglen, seg_incoming=None, D=None, init_states=None, seq_idx=None, nseq=1,
+def fused_scan(X, log_a, B, C, work_tiles, work_incoming=None, D=None, init_states=None, seq_idx=None, nseq=1,
                final_states: Optional[torch.Tensor] = None, chunk=64, stream=None) -> torch.Tensor:
-    """Y from the incoming segment states (and final states into final_states)."""
+    """Y from the incoming range states (and final states into final_states)."""
     p = _fused_problem(X, B, nseq, chunk)
     Y = torch.empty_like(X)
-    _check(lib().ssd_fused_scan(ctypes.byref(p), seglen, _ptr(X), _ptr(log_a), _ptr(B), _ptr(C), _ptr(D),
-                                _ptr(seg_incoming), _ptr(init_states), _ptr(seq_idx), _ptr(Y), _ptr(final_states),
+    _check(lib().ssd_fused_scan(ctypes.byref(p), int(work_tiles), _ptr(X), _ptr(log_a), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(work_incoming), _ptr(init_states), _ptr(seq_idx), _ptr(Y), _ptr(final_states),
                                 _stream(stream)), "ssd_fused_scan")
     return Y

@@ -43,11 +43,13 @@ def rel_err(got, ref):
     return err, scale
 
 
-def assert_close(got, ref, tau, what):
+def assert_close(got, ref, tau, what, atol=0.0):
+    """max|got - ref| <= tau * max|ref| + atol (atol only for quantities that
+    fp32 cannot hold, such as decays below its smallest normal number)."""
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     assert np.isfinite(got).all(), f"{what}: non-finite values"
     err, scale = rel_err(got, ref)
-    assert err <= tau * scale, f"{what}: max|d| = {err:.3e} > {tau:g} * max|ref| = {tau * scale:.3e}"
+    assert err <= tau * scale + atol, f"{what}: max|d| = {err:.3e} > {tau:g} * max|ref| + {atol:g} = {tau * scale + atol:.3e}"
     return err / scale if scale else 0.0
 
 

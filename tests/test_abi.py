@@ -29,7 +29,7 @@ def test_library_exports_every_declared_function():
     assert set(names) >= {"ssd_status_string", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
                           "ssd_chunk_scan", "ssd_check_problem", "ssd_path_supported", "ssd_states_bytes",
                           "ssd_last_cuda_error_string", "ssd_segment_state", "ssd_segment_passing",
-                          "ssd_fused_scan", "ssd_fused_segment_length"}
+                          "ssd_fused_scan", "ssd_fused_work_tiles", "ssd_fused_work_count"}
 
 
 def test_problem_struct_layout():
@@ -47,16 +47,27 @@ def test_workspace_bytes_formula():
     align = lambda x: (x + 255) // 256 * 256
     cs = 2 * 512 * 4 * 4
     st = 2 * (512 // 256) * 4 * 128 * 64 * 4
-    L = ssd.fused_segment_length(p)
-    assert L % 128 == 0 and 128 <= L <= 2048
-    nseg = -(-512 // L)
-    fused = align(2 * nseg * 4 * 128 * 64 * 4) + align(2 * nseg * 4 * 4)
+    # fused: rows (batch, head pair) = 4, 4 tiles each; ranges of wt tiles
+    wt = ssd.fused_work_tiles(p)
+    total = 2 * 2 * 4
+    assert 1 <= wt <= total  # about one range per SM of the device (or of a 148-SM part without one)
+    nwork = -(-total // wt)
+    assert ssd.fused_work_count(p, wt) == nwork
+    fused = 2 * align(nwork * 2 * 128 * 64 * 4) + align(nwork * 2 * 4)
     assert ssd.workspace_bytes(p) == max(align(cs) + align(st), fused)
     assert ssd.states_bytes(p) == st
     # outside the fused domain (fp32) only the chunked need counts
     q = prob(dtype=ssd.ssd.SSD_DTYPE_F32)
-    assert ssd.fused_segment_length(q) == -1
+    assert ssd.fused_work_tiles(q) == -1
     assert ssd.workspace_bytes(q) == align(cs) + align(st)
+
+
+def test_fused_work_count():
+    p = prob()  # 16 tiles in all
+    assert ssd.fused_work_count(p, 3) == 6
+    assert ssd.fused_work_count(p, 16) == 1
+    for bad in (0, -2, 17):
+        assert ssd.fused_work_count(p, bad) == -1
 
 
 @pytest.mark.parametrize("field,value,expect", [
@@ -119,15 +130,16 @@ def test_step_entry_points_validate_on_host():
                               None) == INVALID
     q = prob(nseq=2)
     assert lib.ssd_state_passing(ctypes.byref(q), FAKE, FAKE, FAKE, None, None, None, None) == INVALID
-    # fused steps: bad segment lengths and null pointers are rejected on the host
-    for L in (0, 100, 4096):
-        assert lib.ssd_segment_state(ctypes.byref(p), L, FAKE, FAKE, FAKE, None, FAKE, FAKE, None) == INVALID
-        assert lib.ssd_segment_passing(ctypes.byref(p), L, FAKE, FAKE, None, None, None) == INVALID
-        assert lib.ssd_fused_scan(ctypes.byref(p), L, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, FAKE, None,
+    # fused steps: bad work range lengths and null pointers are rejected on the host
+    for wt in (0, -1, 17):
+        assert lib.ssd_segment_state(ctypes.byref(p), wt, FAKE, FAKE, FAKE, None, FAKE, FAKE, None) == INVALID
+        assert lib.ssd_segment_passing(ctypes.byref(p), wt, FAKE, FAKE, None, None, FAKE, None) == INVALID
+        assert lib.ssd_fused_scan(ctypes.byref(p), wt, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, FAKE, None,
                                   None) == INVALID
-    assert lib.ssd_segment_state(ctypes.byref(p), 256, None, FAKE, FAKE, None, FAKE, FAKE, None) == INVALID
-    assert lib.ssd_fused_scan(ctypes.byref(p), 256, FAKE, FAKE, FAKE, FAKE, None, None, None, None, FAKE, None,
-                              None) == INVALID  # two segments need the incoming states
+    assert lib.ssd_segment_state(ctypes.byref(p), 3, None, FAKE, FAKE, None, FAKE, FAKE, None) == INVALID
+    assert lib.ssd_segment_passing(ctypes.byref(p), 3, FAKE, FAKE, None, None, None, None) == INVALID
+    assert lib.ssd_fused_scan(ctypes.byref(p), 3, FAKE, FAKE, FAKE, FAKE, None, None, None, None, FAKE, None,
+                              None) == INVALID  # ranges that start inside a row need the incoming states
 
 
 def test_binding_rejects_host_tensors_and_bad_shapes():

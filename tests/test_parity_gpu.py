@@ -64,6 +64,7 @@ SMALL = {
     "bf16_boundary_at_chunk_edge": (1, 768, 2, 64, 128, 1, 256, "bf16", [[256, 256, 256]], "none", True),
     "bf16_short_seqs": (1, 512, 2, 64, 64, 1, 256, "bf16", [[1, 1, 3, 250, 1, 256]], "normal", True),
     "f32_varlen_P32_N48_Q64": (2, 320, 3, 32, 48, 1, 64, "f32", [[1, 63, 64, 100, 92], [320]], "normal", True),
+    "bf16_ragged_tile_Q64": (2, 576, 4, 64, 128, 1, 64, "bf16", [[200, 376], [576]], "normal", True),
     "f32_P16_N16_Q128": (1, 384, 5, 16, 16, 1, 128, "f32", None, "ones", False),
 }
 
@@ -129,54 +130,108 @@ def test_steps(name, path):
 
 
 # --------------------------------------------------------------------------- #
-# The fused path, kernel by kernel, against the oracle's quantities at segment
-# level (a segment is a chunk of the block algorithm)
+# The fused path, kernel by kernel, against the oracle's states at the cuts of
+# the work ranges (a range's piece of a row is a block of the block algorithm)
 # --------------------------------------------------------------------------- #
 
 FUSED_CASES = [
-    # (name, seglen)
-    ("bf16_varlen_N128_Q256", 256),
-    ("bf16_varlen_N128_Q256", 384),   # ragged last segment
-    ("bf16_single_N64_Q128", 128),
-    ("bf16_short_seqs", 256),
-    ("bf16_init_N128_Q128", 1024),    # one segment
-    ("bf16_groups2", 256),
+    # (name, work_tiles)
+    ("bf16_varlen_N128_Q256", 3),     # ranges start and end inside rows and span rows
+    ("bf16_varlen_N128_Q256", 5),
+    ("bf16_varlen_N128_Q256", 8),     # one range per row: no cut inside a row
+    ("bf16_varlen_N128_Q256", 32),    # one range for everything
+    ("bf16_single_N64_Q128", 4),
+    ("bf16_single_N64_Q128", 7),
+    ("bf16_short_seqs", 1),           # one tile per range
+    ("bf16_short_seqs", 3),
+    ("bf16_init_N128_Q128", 5),
+    ("bf16_groups2", 3),
+    ("bf16_boundary_at_chunk_edge", 2),  # cuts on sequence boundaries
+    ("bf16_ragged_tile_Q64", 3),      # a short last tile in every row
 ]
 
 
-@pytest.mark.parametrize("name,seglen", FUSED_CASES)
-def test_fused_steps(name, seglen):
+def _cut_states(d, wt, nseq):
+    """The oracle's (local, decay, incoming) at the cuts of the work ranges,
+    [nwork, 2, N, P] / [nwork, 2] / [nwork, 2, N, P], NaN where not defined:
+    local/decay for ranges whose last piece ends inside its row, incoming for
+    ranges whose first piece starts inside its row. Each is the oracle's
+    per-block quantity on a slice of the row: the slice [s0, s1) as one block
+    for the local state and decay, and [0, s0 + 1) cut at s0 for the incoming state."""
+    X, la, B, init, seq = d["X"], d["log_a"], d["B"], d["init_states"], d["seq_idx"]
+    b, T, H, P = X.shape
+    N = B.shape[3]
+    npairs, nt = H // 2, -(-T // 128)
+    total = b * npairs * nt
+    nwork = -(-total // wt)
+    loc = np.full((nwork, 2, N, P), np.nan)
+    dec = np.full((nwork, 2), np.nan)
+    inc = np.full((nwork, 2, N, P), np.nan)
+    sl_seq = lambda bb, a, e: None if seq is None else seq[bb:bb + 1, a:e]
+    for i in range(nwork):
+        fb, fe = i * wt, min((i + 1) * wt, total)
+        r = (fe - 1) // nt
+        s0, s1 = 128 * max(fb - r * nt, 0), min(128 * (fe - r * nt), T)
+        bb, hp = divmod(r, npairs)
+        hs = slice(2 * hp, 2 * hp + 2)
+        if s1 < T:
+            _, lo = oracle.chunk_states(X[bb:bb + 1, s0:s1], la[bb:bb + 1, s0:s1], B[bb:bb + 1, s0:s1], s1 - s0,
+                                        None, sl_seq(bb, s0, s1), nseq=nseq)
+            loc[i] = lo[0, 0, hs]
+            dec[i] = oracle.segment_decay(la[bb:bb + 1, s0:s1], s1 - s0, sl_seq(bb, s0, s1))[0, 0, hs]
+        r0 = fb // nt
+        s0 = 128 * (fb - r0 * nt)
+        if s0 > 0:
+            bb, hp = divmod(r0, npairs)
+            hs = slice(2 * hp, 2 * hp + 2)
+            ini = None if init is None else init[bb:bb + 1]
+            ic, _ = oracle.chunk_states(X[bb:bb + 1, :s0 + 1], la[bb:bb + 1, :s0 + 1], B[bb:bb + 1, :s0 + 1], s0,
+                                        ini, sl_seq(bb, 0, s0 + 1), nseq=nseq)
+            inc[i] = ic[0, 1, hs]
+    return loc, dec, inc
+
+
+def _close_where(got, ref, tau, what, atol=0.0):
+    m = ~np.isnan(ref)
+    assert m.any(), what
+    assert_close(got[m], ref[m], tau, what, atol)
+
+
+@pytest.mark.parametrize("name,wt", FUSED_CASES)
+def test_fused_steps(name, wt):
     ssd = _ssd()
     b, T, H, P, N, G, Q, dtype, lengths, D, init = SMALL[name]
     nseq = 1 if lengths is None else max(len(r) for r in lengths)
-    d = make_custom(b, T, H, P, N, ngroups=G, dtype=dtype, seed=31 + seglen, has_D=D, has_init=init,
+    d = make_custom(b, T, H, P, N, ngroups=G, dtype=dtype, seed=31 + wt, has_D=D, has_init=init,
                     lengths=lengths, nseq=nseq if lengths else None)
     _skip_unsupported(d, dtype, Q, "fused")
     g = to_device(d, dtype)
     tau = TAU[dtype]
     X, B, C = g["X"], g["B"], g["C"]
-    inc_ref, loc_ref = oracle.chunk_states(d["X"], d["log_a"], d["B"], seglen, d["init_states"], d["seq_idx"],
-                                           nseq=nseq)
-    dec_ref = oracle.segment_decay(d["log_a"], seglen, d["seq_idx"])
     Yr, Fr = run_oracle(d)
-    nseg = -(-T // seglen)
-    if nseg > 1:
-        st, dec = ssd.segment_state(X, g["log_a"], B, seglen, g["seq_idx"], nseq)
-        assert_close(st.cpu().numpy().astype(np.float64), loc_ref, tau, "segment states")
-        assert_close(dec.cpu().numpy().astype(np.float64), dec_ref, 1e-5, "segment decay")
-        inc = ssd.segment_passing(st, dec, X, B, seglen, g["init_states"], g["seq_idx"], nseq)
-        assert_close(inc.cpu().numpy().astype(np.float64), inc_ref, tau, "segment incoming states")
+    nt = -(-T // 128)
+    nwork = -(-(b * (H // 2) * nt) // wt)
+    p = ssd.make_problem(b, T, H, P, N, G, Q, nseq, torch.bfloat16, path="fused")
+    assert ssd.fused_work_count(p, wt) == nwork
+    if nwork > 1 and wt % nt != 0:
+        loc_ref, dec_ref, inc_ref = _cut_states(d, wt, nseq)
+        loc, dec = ssd.segment_state(X, g["log_a"], B, wt, g["seq_idx"], nseq)
+        _close_where(loc.cpu().numpy().astype(np.float64), loc_ref, tau, "range end states")
+        # decays below fp32's normal range come back as 0: an absolute floor far below anything they scale
+        _close_where(dec.cpu().numpy().astype(np.float64), dec_ref, 1e-5, "range decays", atol=1e-30)
+        inc = ssd.segment_passing(loc, dec, X, B, wt, g["init_states"], g["seq_idx"], nseq)
+        _close_where(inc.cpu().numpy().astype(np.float64), inc_ref, tau, "range incoming states")
         # segment_passing alone, fed the oracle's states and decays: fp32 arithmetic
-        st2 = torch.from_numpy(np.ascontiguousarray(loc_ref, dtype=np.float32)).cuda()
+        loc2 = torch.from_numpy(np.ascontiguousarray(loc_ref, dtype=np.float32)).cuda()
         dec2 = torch.from_numpy(np.ascontiguousarray(dec_ref, dtype=np.float32)).cuda()
-        inc2 = ssd.segment_passing(st2, dec2, X, B, seglen, g["init_states"], g["seq_idx"], nseq)
-        assert_close(inc2.cpu().numpy().astype(np.float64), inc_ref, 1e-5, "segment incoming (oracle inputs)")
-        seg_in = torch.from_numpy(np.ascontiguousarray(inc_ref, dtype=np.float32)).cuda()
+        inc2 = ssd.segment_passing(loc2, dec2, X, B, wt, g["init_states"], g["seq_idx"], nseq)
+        _close_where(inc2.cpu().numpy().astype(np.float64), inc_ref, 1e-5, "range incoming (oracle inputs)")
+        work_in = torch.from_numpy(np.ascontiguousarray(inc_ref, dtype=np.float32)).cuda()
     else:
-        seg_in = None
-    # fused_scan fed the oracle's incoming segment states
+        work_in = None
+    # fused_scan fed the oracle's incoming range states
     F = torch.full((b, nseq, H, N, P), float("nan"), dtype=torch.float32, device="cuda")
-    Y = ssd.fused_scan(X, g["log_a"], B, C, seglen, seg_in, D=g["D"], init_states=g["init_states"],
+    Y = ssd.fused_scan(X, g["log_a"], B, C, wt, work_in, D=g["D"], init_states=g["init_states"],
                        seq_idx=g["seq_idx"], nseq=nseq, final_states=F)
     torch.cuda.synchronize()
     assert_close(Y.float().cpu().numpy().astype(np.float64), Yr, tau, "fused_scan Y")
