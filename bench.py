@@ -2,11 +2,12 @@
 """Benchmark of the SSD chunked-scan forward on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                [--workload NAME] [--path auto|simt|tcgen05]
+                [--workload NAME] [--path auto|simt|tcgen05|fused]
 
-One step = one pass of the whole forward path (chunk_cumsum, chunk_state,
-state_passing, chunk_scan) over one batch of the workload, inputs resident in
-HBM. The default workload is the Mamba-2-2.7B-shaped layer (batch 4, T 4096,
+One step = one ssd_fwd call, the whole forward path over one batch of the
+workload with its inputs resident in HBM: on the fused family (the default
+for bf16) segment_state, segment_passing and fused_scan; on the chunked
+families chunk_cumsum, chunk_state, state_passing and chunk_scan. The default workload is the Mamba-2-2.7B-shaped layer (batch 4, T 4096,
 80 heads, P 64, N 128, Q 256, bf16 in / fp32 state). Its inputs (~360 MB) are
 larger than L2, so no flush runs between steps. Prints one JSON line on rank 0.
 
@@ -145,6 +146,26 @@ def kernel_model(w, wt=None):
                                flops=b * ntile * (H * (128 * 129 * P + 4 * 128 * N * P) + G * 128 * 129 * N)),
         })
     return out
+
+
+def profiled_traffic(kernel):
+    """dram bytes read + written per launch of `kernel` from the committed ncu
+    summary of the fused path, or None when that summary was taken on another
+    version of the kernel source (or covers no such kernel)."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "fused_path_mamba2_2p7b_layer.md")
+    src = os.path.join(ROOT, "mamba_ssd_layer_chunked_b200", "csrc", "ssd_fused.cu")
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None
+    text = open(prof).read()
+    m = re.search(r"sha256 prefix `([0-9a-f]+)`", text)
+    with open(src, "rb") as f:
+        if not m or hashlib.sha256(f.read()).hexdigest()[: len(m.group(1))] != m.group(1):
+            return None
+    m = re.search(r"dram_bytes_per_launch (.*)", text)
+    vals = dict(kv.split("=") for kv in m.group(1).split()) if m else {}
+    return int(vals[kernel]) if kernel in vals else None
 
 
 def load_peaks():
@@ -498,7 +519,7 @@ def run_ours(args, w):
         achieved = km["flops"] / per_kernel[dom] / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = profiled_traffic(dom)
     roof["kernel"] = dom
     roof["peak_source"] = peaks["source"]
 
