@@ -380,7 +380,8 @@ static_assert(sizeof(CsBuf) % 16 == 0, "CsBuf must keep 16-byte alignment in an 
 // touches; the four warps of a lane quarter split the columns.
 //
 // Per tile t the compute warps run, in this order,
-//   epilogue(t):  Y = Y_diag + rscale Y_off + D x, staged (bf16) in the buffer
+//   epilogue(t):  Y = Y_diag + rscale Y_off (D x is on the diagonal of L o G, so
+//                 it is part of Y_diag), staged (bf16) in the buffer
 //                 of the carried state, which Y_off(t) has finished reading, for
 //                 the TMA store; X' = w X in place in the tile's X buffer;
 //   L o G(t+1):   the next tile's masked C B^T, written over G in TMEM (while
@@ -413,6 +414,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     __shared__ __align__(16) float colf[kComputeWarps][2][2][32];
     // per-warp factors exp2(c_{r+8} - c_{r+e}), e < 8, of the diagonal blocks [warp][row half][head][e]
     __shared__ __align__(16) float cf8[kComputeWarps][2][2][8];
+    // per-thread row factors of the next tile: rf (head 0, 1), rg (head 0, 1)
+    __shared__ float rowf_s[4][kComputeThreads];
     __shared__ __align__(8) uint64_t bar_c, bar_bx[2], bar_g, bar_yo, bar_yd, bar_s, bar_lg, bar_epi, bar_st,
         bar_free, bar_csfull[kCsBufs], bar_csfree[kCsBufs];
     __shared__ uint32_t tmem_base;
@@ -720,9 +723,23 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // tokens) is zero above rb, exp2(c_k - c_l) masked on the diagonal block, and
         // below it exp2(c_k - c_{16 rb}) * exp2(c_{16 rb} - c_l), both factors <= 1.
         // the per-warp column factor tables of tile t (before the wait for Y(t-1))
+        // and this lane's row factors of tile t (rf: to its row block start, rg: to
+        // the middle of the row block, ck: its cumsum) and the pair's D
+        struct RowF {
+            float rf[2], rg[2], ck[2], dd[2];
+        };
         auto lg_tables = [&](int t) {
             const CsBuf& cs = csb[t & (kCsBufs - 1)];
             const int l = 32 * cq + lane;
+            {
+                const int rb = row_block(q4, lane >> 4);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const float ck = cs.c[hh][k];
+                    rowf_s[hh][tid] = ex2_approx(ck - cs.c[hh][16 * rb]);
+                    rowf_s[2 + hh][tid] = ex2_approx(ck - cs.c[hh][16 * rb + 8]);
+                }
+            }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const float cl = cs.c[hh][l];
@@ -736,13 +753,63 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 cf8[warp][hf][hh][e] = ex2_approx(cs.c[hh][r + 8] - cs.c[hh][r + e]);
             }
         };
+        // The diagonal 16x16 block of row block rb for head hh, this lane's 16
+        // columns as 8 packed words: 8x8 quadrants, row i < 8 has columns [0, 8)
+        // direct (masked); row i >= 8 has [8, 16) direct and [0, 8) as
+        // exp2(c_k - c_{r+8}) exp2(c_{r+8} - c_l) (both factors <= 1); the
+        // diagonal element also carries D_h, so that Y_diag includes D x.
+        // g(j) = (selb ? gb : ga)[j] are the block's 16 G values of this lane.
+        auto diag_block = [&](const CsBuf& cs, const RowF& f, int hh, int rb, const uint32_t* ga, const uint32_t* gb,
+                              bool selb, uint32_t* w) {
+            const int hi = lane >> 4, i = lane & 15;
+            const bool lo = i < 8;
+            const int own = lo ? 0 : 8;
+            const float* cr = &cs.c[hh][16 * rb + own];
+            const float4 ca = *reinterpret_cast<const float4*>(cr);
+            const float4 cb = *reinterpret_cast<const float4*>(cr + 4);
+            const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+            const float4 fa = *reinterpret_cast<const float4*>(&cf8[warp][hi][hh][0]);
+            const float4 fb = *reinterpret_cast<const float4*>(&cf8[warp][hi][hh][4]);
+            const float fv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+            float dv[8], lv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t g0 = selb ? gb[e] : ga[e], g8 = selb ? gb[8 + e] : ga[8 + e];
+                const float v = __uint_as_float(lo ? g0 : g8) * ex2_approx(f.ck[hh] - cv[e]);
+                dv[e] = own + e < i ? v : (own + e == i ? v + f.dd[hh] : 0.f);
+                lv[e] = lo ? dv[e] : __uint_as_float(g0) * f.rg[hh] * fv[e];
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                w[e] = pack_bf16(lv[2 * e], lv[2 * e + 1]);
+                w[4 + e] = lo ? 0u : pack_bf16(dv[2 * e], dv[2 * e + 1]);
+            }
+        };
+        // a full block (all columns below the row block) for head hh: 8 packed words
+        auto full_block = [&](const RowF& f, int hh, int cc, const uint32_t* g, uint32_t* w) {
+            const int hi = lane >> 4;
+            const float rf = f.rf[hh];
+            const float* cf = &colf[warp][hh][hi][0];
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+                const float4 fq = *reinterpret_cast<const float4*>(cf + ((16 * cc + 4 * v4) ^ (4 * hi)));
+                const uint32_t* g4 = g + 4 * v4;
+                w[2 * v4] = pack_bf16(__uint_as_float(g4[0]) * rf * fq.x, __uint_as_float(g4[1]) * rf * fq.y);
+                w[2 * v4 + 1] = pack_bf16(__uint_as_float(g4[2]) * rf * fq.z, __uint_as_float(g4[3]) * rf * fq.w);
+            }
+        };
         auto build_lg = [&](int t) {
             const CsBuf& cs = csb[t & (kCsBufs - 1)];
-            const int hi = lane >> 4, i = lane & 15;
+            const int hi = lane >> 4;
             const int rb = row_block(q4, hi);
-            const float ck0 = cs.c[0][k], ck1 = cs.c[1][k];
-            const float rf0 = ex2_approx(ck0 - cs.c[0][16 * rb]), rf1 = ex2_approx(ck1 - cs.c[1][16 * rb]);
-            const float rg0 = ex2_approx(ck0 - cs.c[0][16 * rb + 8]), rg1 = ex2_approx(ck1 - cs.c[1][16 * rb + 8]);
+            RowF f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                f.ck[hh] = cs.c[hh][k];
+                f.rf[hh] = rowf_s[hh][tid];
+                f.rg[hh] = rowf_s[2 + hh][tid];
+                f.dd[hh] = Dv ? Dv[2 * cs.td.hp + hh] : 0.f;
+            }
             __syncwarp();
             mbar_wait(&bar_g, t & 1);
             tc_fence_after();
@@ -751,57 +818,48 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 tmem_ld32_async(tm_g + lane_off + 32 * cq, gw);
                 tmem_wait_ld();
             }
+            if (!kPermRows && cq == q4) {
+                // the diagonal warp of the natural order: lane half hi's diagonal
+                // block is column block hi; block 0 is full for half 1, block 1
+                // zero for half 0. One pass for both halves, no divergence.
+                // own block's G (block hi) into ob, block 0's G for the full part into fb
+                uint32_t ob[16], o0[16];
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c = 2 * cq + cc;  // columns [16 c, 16 c + 16)
-                const uint32_t* g = gw + 16 * cc;
-                uint32_t o[16];
+                for (int e = 0; e < 16; ++e) ob[e] = hi ? gw[16 + e] : gw[e];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t* w = o + 8 * hh;
-                    if (c < rb) {
-                        const float rf = hh ? rf1 : rf0;
-                        const float* cf = &colf[warp][hh][hi][0];
+                    uint32_t dw[8], fw[8];
+                    diag_block(cs, f, hh, rb, ob, ob, false, dw);
+                    full_block(f, hh, 0, gw, fw);
 #pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4) {
-                            const float4 f = *reinterpret_cast<const float4*>(cf + ((16 * cc + 4 * v4) ^ (4 * hi)));
-                            const uint32_t* g4 = g + 4 * v4;
-                            w[2 * v4] = pack_bf16(__uint_as_float(g4[0]) * rf * f.x, __uint_as_float(g4[1]) * rf * f.y);
-                            w[2 * v4 + 1] = pack_bf16(__uint_as_float(g4[2]) * rf * f.z, __uint_as_float(g4[3]) * rf * f.w);
-                        }
-                    } else if (c == rb) {
-                        // diagonal block as 8x8 quadrants: row i < 8 has columns [0, 8)
-                        // direct (masked); row i >= 8 has [8, 16) direct and [0, 8) as
-                        // exp2(c_k - c_{r+8}) exp2(c_{r+8} - c_l), both factors <= 1
-                        const float ck = hh ? ck1 : ck0, rg = hh ? rg1 : rg0;
-                        const bool lo = i < 8;
-                        const int own = lo ? 0 : 8;
-                        const float* cr = &cs.c[hh][16 * c + own];
-                        const float4 ca = *reinterpret_cast<const float4*>(cr);
-                        const float4 cb = *reinterpret_cast<const float4*>(cr + 4);
-                        const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-                        const float4 fa = *reinterpret_cast<const float4*>(&cf8[warp][hi][hh][0]);
-                        const float4 fb = *reinterpret_cast<const float4*>(&cf8[warp][hi][hh][4]);
-                        const float fv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
-                        float dv[8], lv[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float gd = __uint_as_float(lo ? g[e] : g[8 + e]);
-                            dv[e] = own + e <= i ? gd * ex2_approx(ck - cv[e]) : 0.f;
-                            lv[e] = lo ? dv[e] : __uint_as_float(g[e]) * rg * fv[e];
-                        }
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            w[e] = pack_bf16(lv[2 * e], lv[2 * e + 1]);
-                            w[4 + e] = lo ? 0u : pack_bf16(dv[2 * e], dv[2 * e + 1]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) w[e] = 0u;
+                    for (int e = 0; e < 8; ++e) {
+                        o0[8 * hh + e] = hi ? fw[e] : dw[e];   // block 0: full (half 1), diagonal (half 0)
+                        gw[16 + 8 * hh + e] = hi ? dw[e] : 0u;  // block 1: diagonal (half 1), zero (half 0)
                     }
                 }
 #pragma unroll
-                for (int e = 0; e < 16; ++e) gw[16 * cc + e] = o[e];
+                for (int e = 0; e < 16; ++e) gw[e] = o0[e];
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * cq + cc;  // columns [16 c, 16 c + 16)
+                    const uint32_t* g = gw + 16 * cc;
+                    uint32_t o[16];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t* w = o + 8 * hh;
+                        if (c < rb) {
+                            full_block(f, hh, cc, g, w);
+                        } else if (c == rb) {
+                            diag_block(cs, f, hh, rb, g, g, false, w);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) w[e] = 0u;
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) gw[16 * cc + e] = o[e];
+                }
             }
             tmem_st32(tm_lg + lane_off + 32 * cq, gw);
             tmem_wait_st();
@@ -876,7 +934,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const float* ct = csb[t & (kCsBufs - 1)].c[eh];
             uint8_t* Xst = smem + S::oX + st * S::kX + eh * kBox;
             const int64_t rowt = (int64_t)cur.b * d.seqlen;
-            const float dh = Dv ? Dv[2 * cur.hp + eh] : 0.f;
 
             // the next tile's column factor tables while Y(t) is computed
             TileDesc nx = cur;
@@ -886,14 +943,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 lg_tables(t + 1);
             }
             // ---- epilogue(t): Y staged in Hs (or stored), X' = w X in place ----
+            const float ck_e = ct[k], cend_e = ct[cur.v - 1];
+            const float rs = ex2_approx(ck_e);                               // decay from the tile start
+            const float wx = k < cur.v ? ex2_approx(cend_e - ck_e) : 0.f;  // decay to the tile end
             mbar_wait(&bar_yd, par);
             mbar_wait(&bar_yo, par);
             tc_fence_after();
             {
-                const float ck = ct[k];
-                const float cend = ct[cur.v - 1];
-                const float rs = ex2_approx(ck);                            // decay from the tile start
-                const float wx = k < cur.v ? ex2_approx(cend - ck) : 0.f;  // decay to the tile end
                 const __nv_bfloat162 wx2 = __floats2bfloat162_rn(wx, wx);
                 __nv_bfloat16* yrow = Y + ((rowt + cur.ts + k) * d.nheads + 2 * cur.hp + eh) * (int64_t)kP + p0;
 #pragma unroll
@@ -912,10 +968,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&xu[i]);
-                            const float2 xf = __bfloat1622float2(xb);
-                            const int e0 = 8 * c + 2 * i;  // of this half
-                            out[i] = pack_bf16(fmaf(dh, xf.x, fmaf(rs, __uint_as_float(yo[e0]), __uint_as_float(yd[e0]))),
-                                               fmaf(dh, xf.y, fmaf(rs, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1]))));
+                            const int e0 = 8 * c + 2 * i;  // of this half; D x is in Y_diag (L o G diagonal)
+                            out[i] = pack_bf16(fmaf(rs, __uint_as_float(yo[e0]), __uint_as_float(yd[e0])),
+                                               fmaf(rs, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1])));
                             const __nv_bfloat162 xs = __hmul2(xb, wx2);
                             xu[i] = *reinterpret_cast<const uint32_t*>(&xs);
                         }
