@@ -99,15 +99,13 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     segment_state_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b, Dims d,
                          Work wk, const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
                          float* __restrict__ work_local, float* __restrict__ work_decay) {
-    constexpr uint32_t kXB = 2 * kBox, kBB = (N / 64) * kBox;
+    constexpr uint32_t kXB = 2 * kBox, kBB = (N / 64) * kBox, kStage = kXB + kBB;  // two stages
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* Xs = smem;
-    uint8_t* Bs = smem + kXB;
     __shared__ float wsum[8];
     __shared__ float tail_s[2];
     __shared__ int st_shared;
-    __shared__ __align__(8) uint64_t bar_load, bar_mma;
+    __shared__ __align__(8) uint64_t bar_load[2], bar_mma[2];
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -125,8 +123,10 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     if (tid == 0) {
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_b);
-        mbar_init(&bar_load, 1);
-        mbar_init(&bar_mma, 1);
+        mbar_init(&bar_load[0], 1);
+        mbar_init(&bar_load[1], 1);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 1);
         mbar_fence_init();
         // start of the segment's last sequence piece
         int st = s0;
@@ -151,7 +151,6 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     const uint32_t idesc = idesc_bf16(128, N, true, true);
     float tail = 0.f;  // sum of log a after the current tile, this thread's head
     bool cut = false;
-    int done = 0;
     // log a of this thread's (row, head) in a tile; unconditional (clamped row)
     // so that the prefetch does not stall until the value is used
     auto load_la = [&](int i) -> float {
@@ -159,17 +158,30 @@ __global__ void __launch_bounds__(kSegThreads, 1)
         const int v = min(128, s1 - ts);
         return log_a[(row + ts + min(rr, v - 1)) * d.nheads + h0 + hh];
     };
+    // tile i's X (two heads) and B into stage sg
+    auto issue_load = [&](int i, int sg) {
+        const int ts = st + 128 * i;
+        uint8_t* xs = smem + sg * kStage;
+        uint8_t* bs = xs + kXB;
+        mbar_arrive_expect_tx(&bar_load[sg], kStage);
+        tma_load_4d(xs, &tm_x, &bar_load[sg], 0, h0, ts, b);
+        tma_load_4d(xs + kBox, &tm_x, &bar_load[sg], 0, h0 + 1, ts, b);
+#pragma unroll
+        for (int q = 0; q < N / 64; ++q) tma_load_4d(bs + q * kBox, &tm_b, &bar_load[sg], 64 * q, g, ts, b);
+    };
     float la_cur = load_la(ntiles - 1);
-    for (int i = ntiles - 1; i >= 0; --i) {
+    if (tid == 0) issue_load(ntiles - 1, 0);
+    // tiles from the end backwards, two stages: the load of the tile before
+    // runs while this one is scaled and multiplied
+    int it = 0;
+    for (int i = ntiles - 1; i >= 0; --i, ++it) {
+        const int sg = it & 1;
         const int ts = st + 128 * i;
         const int v = min(128, s1 - ts);
         const float la_nxt = i > 0 ? load_la(i - 1) : 0.f;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_load, kXB + kBB);
-            tma_load_4d(Xs, &tm_x, &bar_load, 0, h0, ts, b);
-            tma_load_4d(Xs + kBox, &tm_x, &bar_load, 0, h0 + 1, ts, b);
-#pragma unroll
-            for (int q = 0; q < N / 64; ++q) tma_load_4d(Bs + q * kBox, &tm_b, &bar_load, 64 * q, g, ts, b);
+        if (tid == 0 && i > 0) {
+            if (it >= 1) mbar_wait(&bar_mma[sg ^ 1], ((it - 1) >> 1) & 1);  // its stage was read by the last MMAs
+            issue_load(i - 1, sg ^ 1);
         }
         // within-tile inclusive cumsum of log a (one row per thread, one head per 4 warps)
         float x = rr < v ? la_cur : 0.f;
@@ -184,16 +196,17 @@ __global__ void __launch_bounds__(kSegThreads, 1)
         float pre = 0.f, tot = 0.f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            const float s = wsum[4 * hh + w];
-            if (w < (warp & 3)) pre += s;
-            tot += s;
+            const float sw = wsum[4 * hh + w];
+            if (w < (warp & 3)) pre += sw;
+            tot += sw;
         }
         const float cs = x + pre;
         // weight of row rr: prod of a over (rr, segment end] = exp(tail + tot - cs)
         const float wgt = rr < v ? ex2_approx((tail + tot - cs) * kLog2e) : 0.f;
-        mbar_wait(&bar_load, done & 1);
+        mbar_wait(&bar_load[sg], (it >> 1) & 1);
         // scale row rr of head hh in place; the chunk order is rotated by row so
         // that the 32 rows of a warp spread over all banks
+        uint8_t* Xs = smem + sg * kStage;
         {
             uint8_t* rowp = Xs + hh * kBox + rr * 128;
 #pragma unroll
@@ -213,15 +226,13 @@ __global__ void __launch_bounds__(kSegThreads, 1)
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t xa = smem_u32(Xs), ba = smem_u32(Bs);
+            const uint32_t xa = smem_u32(Xs), ba = smem_u32(Xs + kXB);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 mma_bf16_ss(tacc, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
-                            idesc, (done > 0 || k > 0) ? 1u : 0u);
-            mma_commit(&bar_mma);
+                            idesc, (it > 0 || k > 0) ? 1u : 0u);
+            mma_commit(&bar_mma[sg]);
         }
-        mbar_wait(&bar_mma, done & 1);
-        ++done;
         tail += tot;
         if (rr == 0) tail_s[hh] = tail;
         __syncthreads();
@@ -231,6 +242,10 @@ __global__ void __launch_bounds__(kSegThreads, 1)
             break;
         }
     }
+    // the last MMAs (iteration lm) and, after a cut, the load issued for the tile before
+    const int lm = cut ? it : it - 1;
+    mbar_wait(&bar_mma[lm & 1], (lm >> 1) & 1);
+    if (cut && tid == 0) mbar_wait(&bar_load[(lm + 1) & 1], ((lm + 1) >> 1) & 1);
     tc_fence_after();
     // epilogue: lane m = (head, p); warps w and w+4 split the N columns
     const int m = 32 * (warp & 3) + lane, half = warp >> 2;
@@ -1126,7 +1141,7 @@ cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* 
     if ((e = bc_map(&mb, d, B, 128)) != cudaSuccess) return e;
     const Work w = make_work(d, work_tiles);
     const dim3 grid(w.nwork);
-    const int smem = 2 * (int)kBox + (d.dstate / 64) * (int)kBox + 1024;
+    const int smem = 2 * (2 * (int)kBox + (d.dstate / 64) * (int)kBox) + 1024;
     if (d.dstate == 64) {
         auto k = segment_state_kernel<64>;
         if ((e = set_smem_attr(k, smem, 30)) != cudaSuccess) return e;
