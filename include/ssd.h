@@ -281,6 +281,25 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
                           const float* init_states, const int32_t* seq_idx, void* Y,
                           float* final_states, void* stream);
 
+/* ---- decoding: one step of the recurrence with an fp32 state cache ----
+ * For every (b, h), with g = h / (nheads / ngroups) and a = exp(log_a[b, h]):
+ *   state[b, h] <- a * state[b, h] + B[b, g] x[b, h]^T      (in place)
+ *   y[b, h]      = C[b, g]^T state[b, h] + D[h] x[b, h]
+ * (wang-x-xia "Mamba and state space models" section 2; wq-win section 2.1):
+ * the same recurrence as ssd_fwd, one token at a time, so that a sequence fed
+ * token by token from init_states gives ssd_fwd's Y and final states.
+ *   x, y      [batch, nheads, headdim]            p->dtype
+ *   log_a     [batch, nheads]                     fp32
+ *   B, C      [batch, ngroups, dstate]            p->dtype
+ *   D         [nheads] fp32 or NULL (=> 0)
+ *   state     [batch, nheads, dstate, headdim]    fp32, read and written
+ * Only batch, nheads, headdim (a multiple of 4, at most 1024), dstate, ngroups
+ * and dtype of p are read. Pointers 16-byte aligned (x, y: 8-byte for bf16).
+ * SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED on bad arguments before any
+ * launch; asynchronous on `stream`. */
+ssd_status ssd_decode_step(const ssd_problem* p, const void* x, const float* log_a, const void* B, const void* C,
+                           const float* D, float* state, void* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

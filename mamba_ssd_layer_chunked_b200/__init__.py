@@ -16,6 +16,7 @@ from .ssd import (  # noqa: F401
     chunk_cumsum,
     chunk_scan,
     chunk_state,
+    decode_step,
     declared_functions,
     fused_scan,
     fused_work_count,

@@ -234,6 +234,28 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
                                               Y, final_states, (cudaStream_t)stream));
 }
 
+ssd_status ssd_decode_step(const ssd_problem* p, const void* x, const float* log_a, const void* B, const void* C,
+                           const float* D, float* state, void* y, void* stream) {
+    if (!p) return SSD_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->nheads < 1 || p->headdim < 1 || p->dstate < 1 || p->ngroups < 1 ||
+        p->nheads % p->ngroups != 0)
+        return SSD_ERR_INVALID_ARG;
+    if (p->dtype != SSD_DTYPE_F32 && p->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (p->headdim % 4 != 0 || p->headdim > 1024) return SSD_ERR_UNSUPPORTED;
+    if (p->batch * p->nheads > INT32_MAX || p->dstate > (1 << 20)) return SSD_ERR_UNSUPPORTED;
+    if (!x || !log_a || !B || !C || !state || !y) return SSD_ERR_INVALID_ARG;
+    const uintptr_t vec = p->dtype == SSD_DTYPE_F32 ? 15u : 7u;  // float4 / 4 x bf16 accesses
+    if ((reinterpret_cast<uintptr_t>(x) & vec) || (reinterpret_cast<uintptr_t>(y) & vec) || !aligned16(state) ||
+        (reinterpret_cast<uintptr_t>(log_a) & 3u) || (reinterpret_cast<uintptr_t>(B) & 1u) ||
+        (reinterpret_cast<uintptr_t>(C) & 1u) || (reinterpret_cast<uintptr_t>(D) & 3u))
+        return SSD_ERR_INVALID_ARG;
+    ssd_status s = check_device();
+    if (s != SSD_OK) return s;
+    return cuda_status(ssd::launch_decode_step((int)p->batch, (int)p->nheads, (int)p->headdim, (int)p->dstate,
+                                               (int)p->ngroups, p->dtype, x, log_a, B, C, D, state, y,
+                                               (cudaStream_t)stream));
+}
+
 ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs, void* stream) {
     ssd_status s = check_dims(p);  // log a only: nseq and seq_idx play no part here
     if (s != SSD_OK) return s;

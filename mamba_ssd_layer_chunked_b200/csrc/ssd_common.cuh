@@ -54,6 +54,10 @@ __host__ __device__ __forceinline__ int64_t seqst_off(const Dims& d, int b, int 
 
 // ---- launchers (host) ------------------------------------------------------
 
+cudaError_t launch_decode_step(int batch, int nheads, int headdim, int dstate, int ngroups, ssd_dtype dt,
+                               const void* x, const float* log_a, const void* B, const void* C, const float* D,
+                               float* state, void* y, cudaStream_t st);
+
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* log_a, float* cs, cudaStream_t st);
 
 cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,

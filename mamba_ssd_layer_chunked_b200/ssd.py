@@ -66,6 +66,7 @@ def _declare(lib):
         "ssd_segment_state": ([P, ctypes.c_int64] + [vp] * 7, ctypes.c_int),
         "ssd_segment_passing": ([P, ctypes.c_int64] + [vp] * 6, ctypes.c_int),
         "ssd_fused_scan": ([P, ctypes.c_int64] + [vp] * 11, ctypes.c_int),
+        "ssd_decode_step": ([P] + [vp] * 8, ctypes.c_int),
     }
     for name, (argtypes, restype) in sig.items():
         f = getattr(lib, name)
@@ -327,3 +328,26 @@ def fused_scan(X, log_a, B, C, work_tiles, work_incoming=None, D=None, init_stat
                                 _ptr(work_incoming), _ptr(init_states), _ptr(seq_idx), _ptr(Y), _ptr(final_states),
                                 _stream(stream)), "ssd_fused_scan")
     return Y
+
+
+def decode_step(x: torch.Tensor, log_a: torch.Tensor, B: torch.Tensor, C: torch.Tensor, state: torch.Tensor,
+                D: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One step of the recurrence for every (b, h): state [b, H, N, P] fp32 is
+    updated in place (state <- a state + B x^T) and y = C^T state + D x
+    [b, H, P] (dtype of x) is returned. x [b, H, P], log_a [b, H] fp32,
+    B and C [b, G, N]."""
+    if x.dim() != 3 or B.dim() != 3 or C.shape != B.shape or log_a.shape != x.shape[:2]:
+        raise ValueError("shapes: x [b,H,P], log_a [b,H], B and C [b,G,N]")
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    if B.shape[0] != b or state.shape != (b, H, N, P) or state.dtype != torch.float32:
+        raise ValueError("state must be float32 [b, H, N, P]")
+    if x.dtype not in (torch.float32, torch.bfloat16) or B.dtype != x.dtype or C.dtype != x.dtype:
+        raise TypeError("x, B and C must share one dtype, float32 or bfloat16")
+    if log_a.dtype != torch.float32 or (D is not None and (D.dtype != torch.float32 or D.shape != (H,))):
+        raise TypeError("log_a and D must be float32 (D [nheads])")
+    p = make_problem(b, 64, H, P, N, G, 64, 1, x.dtype)  # seqlen, chunk, nseq are not read by the step
+    y = torch.empty_like(x) if out is None else out
+    _check(lib().ssd_decode_step(ctypes.byref(p), _ptr(x), _ptr(log_a), _ptr(B), _ptr(C), _ptr(D), _ptr(state),
+                                 _ptr(y), _stream(stream)), "ssd_decode_step")
+    return y
