@@ -553,6 +553,99 @@ def run_ours(args, w):
     return 0
 
 
+def _device_inputs(w, dev):
+    import torch
+    inputs = make_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def dev_t(a, dt=torch.float32):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dt).to(dev)
+
+    g = dict(X=dev_t(inputs["X"], tdt), la=dev_t(inputs["log_a"]), B=dev_t(inputs["B"], tdt),
+             C=dev_t(inputs["C"], tdt), D=dev_t(inputs["D"]), init=dev_t(inputs["init_states"]),
+             seq=None if inputs["seq_idx"] is None else torch.from_numpy(inputs["seq_idx"]).to(dev),
+             nseq=inputs["nseq"])
+    return inputs, g
+
+
+def _time_device(fn, steps, warmup, stream):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / steps
+
+
+def run_sweep(args):
+    """--mode sweep: ssd_fwd on every workload (device time, inputs resident),
+    one JSON line each: tokens*heads/s, TFLOP/s and the fractions of the
+    measured bf16 and HBM peaks. Not the headline line."""
+    import torch
+    import mamba_ssd_layer_chunked_b200 as ssd
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    for name in sorted(WORKLOADS):
+        w = WORKLOADS[name]
+        _, g = _device_inputs(w, dev)
+        seq = g["seq"]
+        p = ssd.problem_from(g["X"], g["B"], w.chunk, g["nseq"], args.path)
+        wsp = torch.empty(ssd.workspace_bytes(p), dtype=torch.uint8, device=dev)
+        Y = torch.empty_like(g["X"])
+        F = torch.empty((w.batch, g["nseq"], w.nheads, w.dstate, w.headdim), dtype=torch.float32, device=dev)
+        fn = lambda: ssd.ssd_fwd(g["X"], g["la"], g["B"], g["C"], w.chunk, D=g["D"], init_states=g["init"],
+                                 seq_idx=seq, nseq=g["nseq"] if seq is not None else None, path=args.path,
+                                 out=Y, final_out=F, workspace=wsp)
+        t = _time_device(fn, args.steps, args.warmup, stream)
+        flops, byts = algorithmic_flops(w), algorithmic_bytes(w)
+        print(json.dumps({"mode": "sweep", "workload": name, "path": family(ssd, p, args.path),
+                          "tokens_heads_per_s": w.tokens_heads / t, "ms_per_step": t * 1e3,
+                          "tflops": flops / t / 1e12, "pct_bf16_peak": flops / t / 1e12 / peaks["bf16_tflops"],
+                          "pct_hbm": byts / t / 1e9 / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                          "steps": args.steps, "warmup": args.warmup}), flush=True)
+        del g, wsp, Y, F
+        torch.cuda.empty_cache()
+    return 0
+
+
+def run_decode(args, w):
+    """--mode decode: ssd_decode_step over --decode-batch sequences with the
+    workload's heads, state and dtype (state cache larger than L2). Bytes per
+    step: the state read and written (2 * b * H * N * P * 4) plus x, y, B, C,
+    log a. One JSON line, not the headline."""
+    import torch
+    import mamba_ssd_layer_chunked_b200 as ssd
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    b, H, P, N, G = args.decode_batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=dev).manual_seed(7)
+    x = torch.randn(b, H, P, device=dev, generator=gen).to(tdt)
+    Bm = (torch.randn(b, G, N, device=dev, generator=gen) / N ** 0.5).to(tdt)
+    Cm = (torch.randn(b, G, N, device=dev, generator=gen) / N ** 0.5).to(tdt)
+    la = -torch.rand(b, H, device=dev, generator=gen) * 0.1
+    state = torch.randn(b, H, N, P, device=dev, generator=gen)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+    t = _time_device(lambda: ssd.decode_step(x, la, Bm, Cm, state, out=y), args.steps, args.warmup, stream)
+    e = 2 if w.dtype == "bf16" else 4
+    byts = 2 * b * H * N * P * 4 + 2 * b * H * P * e + 2 * b * G * N * e + b * H * 4
+    peaks = load_peaks()
+    print(json.dumps({"mode": "decode", "metric": "SSD decode step tokens·heads/s", "workload": w.name,
+                      "decode_batch": b, "value": b * H / t, "unit": "tokens·heads/s", "us_per_step": t * 1e6,
+                      "roofline": {"bound": "hbm", "achieved": byts / t / 1e9, "peak": peaks["hbm_gbs"],
+                                   "unit": "GB/s", "frac": byts / t / 1e9 / peaks["hbm_gbs"]},
+                      "steps": args.steps, "warmup": args.warmup, "dtype": w.dtype}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -564,12 +657,19 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--mode", choices=["scan", "sweep", "decode"], default="scan",
+                    help="scan: the headline line (default); sweep: every workload; decode: the decode step")
+    ap.add_argument("--decode-batch", type=int, default=64)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.mode == "sweep":
+        return run_sweep(args)
+    if args.mode == "decode":
+        return run_decode(args, w)
     return run_ours(args, w)
 
 
