@@ -97,12 +97,72 @@ ssd_path fwd_family(const ssd_problem* p) {
         case SSD_PATH_FUSED: return SSD_PATH_FUSED;
         default: break;
     }
-    if (ssd::fused_supported(p)) return SSD_PATH_FUSED;
+    if (ssd::fused_fwd_supported(p)) return SSD_PATH_FUSED;
     if (ssd::tc_supported(p)) return SSD_PATH_TCGEN05;
     return SSD_PATH_SIMT;
 }
 
 size_t chunked_workspace_bytes(const ssd_problem* p) { return align256(cs_bytes(p)) + align256(states_bytes(p)); }
+
+// The fused family on the dstate it was given directly (64 or 128), or on
+// slices of at most 128 state rows padded to Np (64 when dstate <= 64, else
+// 128): the work-range states of the padded problem, the padded B and C,
+// padded initial and final states, and one more Y for slices after the first.
+struct FusedPlan {
+    bool direct;
+    int pieces, np;
+};
+
+FusedPlan fused_plan(const ssd_problem* p) {
+    FusedPlan f;
+    f.direct = p->dstate == 64 || p->dstate == 128;
+    f.pieces = (int)((p->dstate + 127) / 128);
+    f.np = f.direct ? (int)p->dstate : (p->dstate <= 64 ? 64 : 128);
+    return f;
+}
+
+struct FusedLayout {
+    size_t work, bc, st, y, total;
+};
+
+FusedLayout fused_layout(const ssd_problem* p) {
+    const FusedPlan f = fused_plan(p);
+    ssd::Dims d = make_dims(p);
+    d.dstate = f.np;
+    FusedLayout l;
+    l.work = align256(ssd::fused_workspace_bytes(d, ssd::fused_default_work_tiles(d)));
+    l.bc = l.st = l.y = 0;
+    if (!f.direct) {
+        l.bc = align256((size_t)p->batch * p->seqlen * p->ngroups * f.np * 2);
+        l.st = align256((size_t)p->batch * p->nseq * p->nheads * f.np * p->headdim * sizeof(float));
+        if (f.pieces > 1) l.y = align256((size_t)p->batch * p->seqlen * p->nheads * p->headdim * 2);
+    }
+    l.total = l.work + 2 * l.bc + 2 * l.st + l.y;
+    return l;
+}
+
+// The three fused launches on dims d (dstate 64 or 128), workspace ws.
+cudaError_t run_fused(const ssd::Dims& d, const void* X, const float* log_a, const void* B, const void* C,
+                      const float* D, const float* init_states, const int32_t* seq_idx, void* Y, float* final_states,
+                      void* ws, cudaStream_t st) {
+    const int64_t wt = ssd::fused_default_work_tiles(d);
+    const size_t nwork = (size_t)ssd::fused_work_count(d, wt);
+    const size_t stb = nwork * 2 * d.dstate * d.headdim * sizeof(float);
+    float* work_local = static_cast<float*>(ws);
+    float* work_in = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(stb));
+    float* work_decay = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * align256(stb));
+    const bool cuts = ssd::fused_needs_cut_states(d, wt);
+    cudaError_t e = cudaSuccess;
+    if (cuts) {
+        if ((e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st)) != cudaSuccess)
+            return e;
+        if ((e = ssd::launch_segment_passing(d, wt, work_local, work_decay, init_states, seq_idx, work_in, st)) !=
+            cudaSuccess)
+            return e;
+    }
+    return ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, cuts ? work_in : nullptr, init_states, seq_idx, Y,
+                                  final_states, st);
+}
 
 ssd_status check_common(const ssd_problem* p, const int32_t* seq_idx) {
     ssd_status s = check_dims(p);
@@ -116,7 +176,7 @@ ssd_status check_runnable(const ssd_problem* p) {
     ssd_status s = check_device();
     if (s != SSD_OK) return s;
     if (p->path == SSD_PATH_TCGEN05 && !ssd::tc_supported(p)) return SSD_ERR_UNSUPPORTED;
-    if (p->path == SSD_PATH_FUSED && !ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+    if (p->path == SSD_PATH_FUSED && !ssd::fused_fwd_supported(p)) return SSD_ERR_UNSUPPORTED;
     return SSD_OK;
 }
 
@@ -155,7 +215,7 @@ int ssd_path_supported(const ssd_problem* p, ssd_path path) {
     if (check_dims(p) != SSD_OK || check_device() != SSD_OK) return 0;
     if (path == SSD_PATH_SIMT) return 1;
     if (path == SSD_PATH_TCGEN05) return ssd::tc_supported(p) ? 1 : 0;
-    if (path == SSD_PATH_FUSED) return ssd::fused_supported(p) ? 1 : 0;
+    if (path == SSD_PATH_FUSED) return ssd::fused_fwd_supported(p) ? 1 : 0;
     return 0;
 }
 
@@ -167,9 +227,8 @@ size_t ssd_states_bytes(const ssd_problem* p) {
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
     if (check_dims(p) != SSD_OK) return (size_t)-1;
     size_t need = chunked_workspace_bytes(p);
-    if (ssd::fused_supported(p)) {
-        const ssd::Dims d = make_dims(p);
-        const size_t f = ssd::fused_workspace_bytes(d, ssd::fused_default_work_tiles(d));
+    if (ssd::fused_fwd_supported(p)) {
+        const size_t f = fused_layout(p).total;
         if (f > need) need = f;
     }
     return need;
@@ -321,22 +380,40 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
     cudaStream_t st = (cudaStream_t)stream;
     const ssd_path fam = fwd_family(p);
     if (fam == SSD_PATH_FUSED) {
-        const int64_t wt = ssd::fused_default_work_tiles(d);
-        const size_t nwork = (size_t)ssd::fused_work_count(d, wt);
-        const size_t stb = nwork * 2 * d.dstate * d.headdim * sizeof(float);
-        float* work_local = static_cast<float*>(workspace);
-        float* work_in = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(stb));
-        float* work_decay = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * align256(stb));
-        const bool cuts = ssd::fused_needs_cut_states(d, wt);
+        const FusedPlan f = fused_plan(p);
+        if (f.direct)
+            return cuda_status(run_fused(d, X, log_a, B, C, D, init_states, seq_idx, Y, final_states, workspace, st));
+        // slices of the state rows, each padded to np columns of B and C
+        const FusedLayout l = fused_layout(p);
+        char* w = static_cast<char*>(workspace);
+        void* Bp = w + l.work;
+        void* Cp = w + l.work + l.bc;
+        float* init_p = reinterpret_cast<float*>(w + l.work + 2 * l.bc);
+        float* fin_p = reinterpret_cast<float*>(w + l.work + 2 * l.bc + l.st);
+        void* Yk = w + l.work + 2 * l.bc + 2 * l.st;
+        ssd::Dims dp = d;
+        dp.dstate = f.np;
+        const int64_t rows = (int64_t)d.batch * d.seqlen * d.ngroups;
+        const int64_t S = (int64_t)d.batch * d.nseq * d.nheads;
         cudaError_t e = cudaSuccess;
-        if (cuts) {
-            e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st);
-            if (e != cudaSuccess) return cuda_status(e);
-            e = ssd::launch_segment_passing(d, wt, work_local, work_decay, init_states, seq_idx, work_in, st);
-            if (e != cudaSuccess) return cuda_status(e);
+        for (int k = 0; k < f.pieces && e == cudaSuccess; ++k) {
+            const int n0 = 128 * k, wd = d.dstate - n0 < 128 ? d.dstate - n0 : 128;
+            if ((e = ssd::launch_pad_bc(B, Bp, rows, d.dstate, n0, wd, f.np, st)) != cudaSuccess) break;
+            if ((e = ssd::launch_pad_bc(C, Cp, rows, d.dstate, n0, wd, f.np, st)) != cudaSuccess) break;
+            if (init_states &&
+                (e = ssd::launch_pad_states(init_states, init_p, S, d.dstate, n0, wd, f.np, d.headdim, st)) !=
+                    cudaSuccess)
+                break;
+            void* Yo = k == 0 ? Y : Yk;
+            if ((e = run_fused(dp, X, log_a, Bp, Cp, k == 0 ? D : nullptr, init_states ? init_p : nullptr, seq_idx, Yo,
+                               final_states ? fin_p : nullptr, w, st)) != cudaSuccess)
+                break;
+            if (final_states &&
+                (e = ssd::launch_unpad_states(fin_p, final_states, S, d.dstate, n0, wd, f.np, d.headdim, st)) !=
+                    cudaSuccess)
+                break;
+            if (k > 0) e = ssd::launch_add_bf16(Y, Yk, (int64_t)d.batch * d.seqlen * d.nheads * d.headdim, st);
         }
-        e = ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, cuts ? work_in : nullptr, init_states, seq_idx, Y,
-                                   final_states, st);
         return cuda_status(e);
     }
     float* cs = static_cast<float*>(workspace);

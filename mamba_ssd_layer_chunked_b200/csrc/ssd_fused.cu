@@ -1104,6 +1104,13 @@ bool fused_supported(const ssd_problem* p) {
     return true;
 }
 
+bool fused_fwd_supported(const ssd_problem* p) {
+    if (p->dtype != SSD_DTYPE_BF16 || p->headdim != kP) return false;
+    if (p->dstate % 16 != 0 || p->dstate > 256) return false;
+    if ((p->nheads / p->ngroups) % 2 != 0) return false;
+    return true;
+}
+
 bool fused_work_ok(const Dims& d, int64_t work_tiles) {
     const int64_t total = (int64_t)d.batch * (d.nheads / 2) * ((d.seqlen + 127) / 128);
     if (work_tiles < 1 || work_tiles > total) return false;

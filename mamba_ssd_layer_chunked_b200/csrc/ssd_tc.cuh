@@ -27,7 +27,10 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* X, const void* B, co
 // ---- fused path (ssd_fused.cu) ----
 // The rows (batch row, head pair) x 128-token tiles laid end to end, cut into
 // ranges of work_tiles tiles, one CTA each.
-bool fused_supported(const ssd_problem* p);
+bool fused_supported(const ssd_problem* p);  // the step entry points: dstate 64 or 128
+// ssd_fwd on the fused family: any dstate that is a multiple of 16 up to 256,
+// as slices of at most 128 state rows padded to 64 or 128 (ssd_pad.cu)
+bool fused_fwd_supported(const ssd_problem* p);
 // tiles per range chosen for problem d on the current device
 int fused_default_work_tiles(const Dims& d);
 bool fused_work_ok(const Dims& d, int64_t work_tiles);
@@ -43,5 +46,13 @@ cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const floa
 cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
                               const void* C, const float* D, const float* work_in, const float* init_states,
                               const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st);
+
+// state-dimension slices (ssd_pad.cu)
+cudaError_t launch_pad_bc(const void* src, void* dst, int64_t rows, int N, int n0, int w, int Np, cudaStream_t st);
+cudaError_t launch_pad_states(const float* src, float* dst, int64_t S, int N, int n0, int w, int Np, int P,
+                              cudaStream_t st);
+cudaError_t launch_unpad_states(const float* src, float* dst, int64_t S, int N, int n0, int w, int Np, int P,
+                                cudaStream_t st);
+cudaError_t launch_add_bf16(void* y, const void* yk, int64_t n, cudaStream_t st);
 
 }  // namespace ssd
