@@ -349,9 +349,10 @@ struct FusedSmem {
 };
 
 // One tile of a range, as the decay warp publishes it: batch row, head pair,
-// first token, valid rows, the sequence id of its tokens and flags.
+// first token, valid rows, the sequence id of its tokens, the id of the token
+// before it in the row (-1 at the row start) and flags.
 struct TileDesc {
-    int b, hp, ts, v, sid, flags;
+    int b, hp, ts, v, sid, psid, flags;
 };
 enum : int {
     kTileLast = 1,      // last tile of its sequence piece in this range
@@ -615,10 +616,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int b = r / wk.npairs, hp = r % wk.npairs;
             const int64_t row = (int64_t)b * d.seqlen;
             int v = min(128, s1 - pos);
-            int sid = 0;
+            int sid = 0, psid = pos > 0 ? 0 : -1;
             bool change = false;  // the sequence changes right after the tile
             if (seq_idx) {
                 sid = seq_clamped(seq_idx, row, pos, d.nseq);
+                if (pos > 0) psid = seq_clamped(seq_idx, row, pos - 1, d.nseq);
                 // first offset j in [1, min(128, s1 - pos - 1)] whose id differs
                 const int jmax = min(128, s1 - pos - 1);
                 int jm = 1 << 30;
@@ -651,6 +653,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             td.ts = pos;
             td.v = v;
             td.sid = sid;
+            td.psid = psid;
             td.flags = flags;
             first = false;
             pos = pend;
@@ -923,9 +926,25 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             return init_states ? init_states + seqst_off(d, b, sid, 2 * hp + sh) : nullptr;
         };
 
+        // ids that never occur between the sequence before tile td and its own
+        // keep their initial state (or zero) as final state
+        auto fill_gap = [&](const TileDesc& td) {
+            if (!final_states || !seq_idx) return;
+            for (int sq = td.psid + 1; sq < td.sid; ++sq) {
+                float* f = final_states + seqst_off(d, td.b, sq, 2 * td.hp + sh);
+                const float* src = init_src(td.b, td.hp, sq);
+#pragma unroll
+                for (int i = 0; i < NQ; ++i) {
+                    const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
+                    f[o] = src ? src[o] : 0.f;
+                }
+            }
+        };
+
         // ---- prologue: the first piece's state and tile 0's L o G ----
         wait_cs(0);
         TileDesc cur = csb[0].td;
+        fill_gap(cur);
         {
             const float* src = (cur.flags & kTileFromWork) ? work_in + ((int64_t)i_work * 2 + sh) * N * kP
                                                            : init_src(cur.b, cur.hp, cur.sid);
@@ -1017,7 +1036,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         for (int i = 0; i < NQ; ++i) f[(int64_t)(cq * NQ + i) * kP + sp] = hv[i];
                     }
                     // the next tile starts a new sequence or a new row
-                    if (!fin) load_state(hv, init_src(nx.b, nx.hp, nx.sid));
+                    if (!fin) {
+                        load_state(hv, init_src(nx.b, nx.hp, nx.sid));
+                        fill_gap(nx);
+                    }
                 }
                 // ids after the row's last sequence never occur: they keep their initial state
                 if ((cur.flags & kTileRowEnd) && final_states && seq_idx) {

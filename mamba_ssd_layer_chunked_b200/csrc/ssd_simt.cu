@@ -251,6 +251,16 @@ __global__ void __launch_bounds__(kThreads) state_passing_kernel(Dims d, const f
         float* dst = incoming + st_off(d, b, c, h);
         float4 S = active ? ld4(src + idx) : zero;
         if (active) st4(dst + idx, hin);
+        // ids that never occur (between the previous sequence and this chunk's
+        // first, or between two pieces of this chunk) keep their initial state
+        if (seq_idx && final_states && active) {
+            if (!continues)
+                for (int s = (c > 0 ? s_prev_last : -1) + 1; s < s_first; ++s)
+                    st4(final_states + seqst_off(d, b, s, h) + idx, init_of(s));
+            for (int j = 1; j < np; ++j)
+                for (int s = pseq[j - 1] + 1; s < pseq[j]; ++s)
+                    st4(final_states + seqst_off(d, b, s, h) + idx, init_of(s));
+        }
         if (seq_idx && final_states && active) {
             for (int j = 0; j + 1 < np; ++j) {
                 const int st = pstart[j], e = pstart[j + 1] - 1, s = pseq[j];

@@ -65,6 +65,10 @@ SMALL = {
     "bf16_short_seqs": (1, 512, 2, 64, 64, 1, 256, "bf16", [[1, 1, 3, 250, 1, 256]], "normal", True),
     "f32_varlen_P32_N48_Q64": (2, 320, 3, 32, 48, 1, 64, "f32", [[1, 63, 64, 100, 92], [320]], "normal", True),
     "bf16_ragged_tile_Q64": (2, 576, 4, 64, 128, 1, 64, "bf16", [[200, 376], [576]], "normal", True),
+    # ids that never occur (zero-length sequences): they keep their initial state
+    "bf16_skipped_ids_Q128": (2, 512, 4, 64, 128, 1, 128, "bf16", [[100, 0, 300, 0, 112], [512, 0, 0, 0, 0]],
+                              "normal", True),
+    "f32_skipped_ids_Q64": (2, 256, 3, 32, 48, 1, 64, "f32", [[60, 0, 100, 96], [0, 256, 0, 0]], "normal", True),
     "f32_P16_N16_Q128": (1, 384, 5, 16, 16, 1, 128, "f32", None, "ones", False),
 }
 
