@@ -92,7 +92,8 @@ typedef enum {
 
 typedef struct {
     int64_t batch;     /* b  >= 1 */
-    int64_t seqlen;    /* T  >= 1, a multiple of chunk */
+    int64_t seqlen;    /* T  >= 1; a multiple of chunk on the SIMT and TCGEN05 families and the
+                          chunked step entry points, any length on the FUSED family */
     int64_t nheads;    /* H  >= 1, a multiple of ngroups */
     int64_t headdim;   /* P: multiple of 16, <= 256 */
     int64_t dstate;    /* N: multiple of 16, <= 256 */

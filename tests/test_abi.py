@@ -73,7 +73,7 @@ def test_fused_work_count():
 @pytest.mark.parametrize("field,value,expect", [
     ("batch", 0, INVALID), ("seqlen", 0, INVALID), ("nheads", 0, INVALID), ("headdim", -1, INVALID),
     ("dstate", 0, INVALID), ("ngroups", 3, INVALID), ("nseq", 0, INVALID), ("dtype", 7, INVALID),
-    ("path", 9, INVALID), ("chunk", 100, UNSUPPORTED), ("seqlen", 500, UNSUPPORTED),
+    ("path", 9, INVALID), ("chunk", 100, UNSUPPORTED),
     ("headdim", 24, UNSUPPORTED), ("dstate", 512, UNSUPPORTED)])
 def test_bad_problem_rejected(field, value, expect):
     p = prob(**{field: value})
@@ -81,6 +81,20 @@ def test_bad_problem_rejected(field, value, expect):
     assert lib.ssd_fwd_workspace_bytes(ctypes.byref(p)) == ctypes.c_size_t(-1).value
     assert lib.ssd_check_problem(ctypes.byref(p)) == expect
     assert lib.ssd_fwd(ctypes.byref(p), *([FAKE] * 9), FAKE, 1 << 30, None) == expect
+
+
+def test_ragged_length_needs_the_fused_family():
+    # T % Q != 0: the chunked families refuse it, the fused family (bf16, P 64) takes it
+    lib = ssd.lib()
+    for path in (1, 2):
+        p = prob(seqlen=500, path=path)
+        assert lib.ssd_fwd(ctypes.byref(p), *([FAKE] * 9), FAKE, 1 << 30, None) == UNSUPPORTED
+    p = prob(seqlen=500, dtype=ssd.ssd.SSD_DTYPE_F32)  # AUTO falls to SIMT
+    assert lib.ssd_fwd(ctypes.byref(p), *([FAKE] * 9), FAKE, 1 << 30, None) == UNSUPPORTED
+    assert lib.ssd_states_bytes(ctypes.byref(p)) == ctypes.c_size_t(-1).value
+    assert lib.ssd_chunk_cumsum(ctypes.byref(p), FAKE, FAKE, None) == UNSUPPORTED
+    q = prob(seqlen=500)  # AUTO, bf16: the fused family
+    assert ssd.workspace_bytes(q) > 0
 
 
 def test_null_problem_rejected():

@@ -65,6 +65,8 @@ SMALL = {
     "bf16_short_seqs": (1, 512, 2, 64, 64, 1, 256, "bf16", [[1, 1, 3, 250, 1, 256]], "normal", True),
     "f32_varlen_P32_N48_Q64": (2, 320, 3, 32, 48, 1, 64, "f32", [[1, 63, 64, 100, 92], [320]], "normal", True),
     "bf16_ragged_tile_Q64": (2, 576, 4, 64, 128, 1, 64, "bf16", [[200, 376], [576]], "normal", True),
+    # T not a multiple of Q (or of the 128-token tile): the fused family only
+    "bf16_ragged_T1000_Q256": (2, 1000, 4, 64, 128, 1, 256, "bf16", [[400, 600], [1000]], "normal", True),
     # ids that never occur (zero-length sequences): they keep their initial state
     "bf16_skipped_ids_Q128": (2, 512, 4, 64, 128, 1, 128, "bf16", [[100, 0, 300, 0, 112], [512, 0, 0, 0, 0]],
                               "normal", True),
@@ -152,6 +154,7 @@ FUSED_CASES = [
     ("bf16_groups2", 3),
     ("bf16_boundary_at_chunk_edge", 2),  # cuts on sequence boundaries
     ("bf16_ragged_tile_Q64", 3),      # a short last tile in every row
+    ("bf16_ragged_T1000_Q256", 3),    # T not a multiple of the chunk
 ]
 
 
