@@ -282,6 +282,23 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
                           const float* init_states, const int32_t* seq_idx, void* Y,
                           float* final_states, void* stream);
 
+/* ---- discretisation: the step before the scan in the Mamba block ----
+ * For every (b, t, h), with z = dt[b, t, h] + dt_bias[h]:
+ *   delta = softplus(z) = log(1 + exp(z)),   log_a[b, t, h] = delta * A[h]
+ *   X[b, t, h, :] = s * x[b, t, h, :],  s = delta                    (zoh == 0)
+ *                                       s = (exp(delta A) - 1) / A   (zoh != 0; delta when A == 0)
+ * (ai.tomabc.com "Mamba": delta = softplus(linear + bias), A_bar = exp(delta A);
+ * wang-x-xia "Mamba and state space models" section 2: zero-order hold). X and
+ * log_a are the X and log_a inputs of ssd_fwd: zoh == 0 puts B_bar = delta B on
+ * x, zoh != 0 the zero-order-hold B_bar = (exp(delta A) - 1) / A B.
+ *   dt, log_a   [batch, seqlen, nheads]           fp32
+ *   dt_bias, A  [nheads] fp32 (dt_bias may be NULL => 0; A <= 0 expected)
+ *   x, X        [batch, seqlen, nheads, headdim]  p->dtype (X may alias x)
+ * Only batch, seqlen, nheads, headdim (a multiple of 4) and dtype of p are
+ * read. SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED before any launch. */
+ssd_status ssd_discretize(const ssd_problem* p, const float* dt, const float* dt_bias, const float* A,
+                          const void* x, int zoh, float* log_a, void* X, void* stream);
+
 /* ---- decoding: one step of the recurrence with an fp32 state cache ----
  * For every (b, h), with g = h / (nheads / ngroups) and a = exp(log_a[b, h]):
  *   state[b, h] <- a * state[b, h] + B[b, g] x[b, h]^T      (in place)

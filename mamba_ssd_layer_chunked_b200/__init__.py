@@ -6,7 +6,7 @@
                               seq_idx=seq_idx, nseq=nseq)
 
 Importing the package loads the library and raises ImportError when it has
-not been built (``python -m mamba_ssd_layer_chunked_b200.build``): there is no
+not been built (``python mamba_ssd_layer_chunked_b200/build.py``): there is no
 fallback implementation.
 """
 from .ssd import (  # noqa: F401
@@ -17,6 +17,7 @@ from .ssd import (  # noqa: F401
     chunk_scan,
     chunk_state,
     decode_step,
+    discretize,
     declared_functions,
     fused_scan,
     fused_work_count,

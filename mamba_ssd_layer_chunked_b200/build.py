@@ -1,7 +1,7 @@
 """Build libssd_b200.so (all CUDA sources under csrc/) for sm_100a with nvcc.
 
 The library is built in-tree, next to this file, so it ships with the package.
-Usage: python -m mamba_ssd_layer_chunked_b200.build [--force] [--verbose]
+Usage: python mamba_ssd_layer_chunked_b200/build.py [--force] [--verbose]
 """
 from __future__ import annotations
 

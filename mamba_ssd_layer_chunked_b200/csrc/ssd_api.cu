@@ -297,6 +297,25 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
                                               Y, final_states, (cudaStream_t)stream));
 }
 
+ssd_status ssd_discretize(const ssd_problem* p, const float* dt, const float* dt_bias, const float* A,
+                          const void* x, int zoh, float* log_a, void* X, void* stream) {
+    if (!p) return SSD_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->seqlen < 1 || p->nheads < 1 || p->headdim < 1) return SSD_ERR_INVALID_ARG;
+    if (p->dtype != SSD_DTYPE_F32 && p->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (p->headdim % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (p->batch * p->seqlen * p->nheads * p->headdim / 4 > ((int64_t)1 << 40)) return SSD_ERR_UNSUPPORTED;
+    if (!dt || !A || !x || !log_a || !X) return SSD_ERR_INVALID_ARG;
+    const uintptr_t el = p->dtype == SSD_DTYPE_F32 ? 3u : 1u;
+    if ((reinterpret_cast<uintptr_t>(dt) & 3u) || (reinterpret_cast<uintptr_t>(dt_bias) & 3u) ||
+        (reinterpret_cast<uintptr_t>(A) & 3u) || (reinterpret_cast<uintptr_t>(log_a) & 3u) ||
+        (reinterpret_cast<uintptr_t>(x) & el) || (reinterpret_cast<uintptr_t>(X) & el))
+        return SSD_ERR_INVALID_ARG;
+    ssd_status s = check_device();
+    if (s != SSD_OK) return s;
+    return cuda_status(ssd::launch_discretize(p->batch * p->seqlen * p->nheads, (int)p->nheads, (int)p->headdim,
+                                              p->dtype, dt, dt_bias, A, x, zoh, log_a, X, (cudaStream_t)stream));
+}
+
 ssd_status ssd_decode_step(const ssd_problem* p, const void* x, const float* log_a, const void* B, const void* C,
                            const float* D, float* state, void* y, void* stream) {
     if (!p) return SSD_ERR_INVALID_ARG;

@@ -54,6 +54,10 @@ __host__ __device__ __forceinline__ int64_t seqst_off(const Dims& d, int b, int 
 
 // ---- launchers (host) ------------------------------------------------------
 
+cudaError_t launch_discretize(int64_t rows, int nheads, int headdim, ssd_dtype dt_x, const float* dt,
+                              const float* dt_bias, const float* A, const void* x, int zoh, float* log_a, void* X,
+                              cudaStream_t st);
+
 cudaError_t launch_decode_step(int batch, int nheads, int headdim, int dstate, int ngroups, ssd_dtype dt,
                                const void* x, const float* log_a, const void* B, const void* C, const float* D,
                                float* state, void* y, cudaStream_t st);

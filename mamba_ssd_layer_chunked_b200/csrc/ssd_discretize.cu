@@ -1,0 +1,65 @@
+// ssd_discretize.cu -- the step before the SSD scan in the Mamba block: the
+// input-dependent step size and the discretisation of A and B x.
+//
+//   delta = softplus(dt + dt_bias[h]),   log a = delta * A[h]
+//   X = s * x  with  s = delta                       (Euler for B: B_bar = delta B)
+//                 or s = (exp(delta A) - 1) / A      (zero-order hold for B)
+//
+// Source: the Mamba page (ai.tomabc.com, paper story 21): delta = softplus(
+// linear(x) + bias) in the block pseudocode and A_bar = exp(delta * A); "Mamba
+// and state space models" (wang-x-xia.github.io), section 2: the zero-order-hold
+// discretisation h_t = A_bar h_{t-1} + B_bar x_t. The per-head scalar s is put
+// on x (B is shared by the heads of a group), which the recurrence does not
+// distinguish from putting it on B. Bandwidth-bound: x in, X out.
+
+#include "ssd_common.cuh"
+
+namespace ssd {
+
+namespace {
+
+constexpr int kDiscThreads = 256;
+
+__device__ __forceinline__ float softplus_f(float z) { return z > 20.f ? z : log1pf(expf(z)); }
+
+// one thread per 4 consecutive elements of a row (b, t, h) of P elements
+template <typename T>
+__global__ void __launch_bounds__(kDiscThreads) discretize_kernel(int64_t rows, int nheads, int headdim,
+                                                                  const float* __restrict__ dt,
+                                                                  const float* __restrict__ dt_bias,
+                                                                  const float* __restrict__ A, const T* __restrict__ x,
+                                                                  int zoh, float* __restrict__ log_a, T* __restrict__ X) {
+    const int P4 = headdim / 4;
+    const int64_t i = (int64_t)blockIdx.x * kDiscThreads + threadIdx.x;
+    if (i >= rows * P4) return;
+    const int64_t r = i / P4;
+    const int q = (int)(i % P4);
+    const int h = (int)(r % nheads);
+    const float a = A[h];
+    const float delta = softplus_f(dt[r] + (dt_bias ? dt_bias[h] : 0.f));
+    const float la = delta * a;
+    if (q == 0) log_a[r] = la;
+    const float s = zoh ? (a != 0.f ? expm1f(la) / a : delta) : delta;
+    const T* xr = x + r * headdim + 4 * q;
+    T* Xr = X + r * headdim + 4 * q;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Xr[e] = from_f32<T>(s * to_f32(xr[e]));
+}
+
+}  // namespace
+
+cudaError_t launch_discretize(int64_t rows, int nheads, int headdim, ssd_dtype dt_x, const float* dt,
+                              const float* dt_bias, const float* A, const void* x, int zoh, float* log_a, void* X,
+                              cudaStream_t st) {
+    const int64_t n = rows * (headdim / 4);
+    const unsigned grid = (unsigned)((n + kDiscThreads - 1) / kDiscThreads);
+    if (dt_x == SSD_DTYPE_F32)
+        discretize_kernel<float><<<grid, kDiscThreads, 0, st>>>(rows, nheads, headdim, dt, dt_bias, A,
+                                                                 (const float*)x, zoh, log_a, (float*)X);
+    else
+        discretize_kernel<__nv_bfloat16><<<grid, kDiscThreads, 0, st>>>(
+            rows, nheads, headdim, dt, dt_bias, A, (const __nv_bfloat16*)x, zoh, log_a, (__nv_bfloat16*)X);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

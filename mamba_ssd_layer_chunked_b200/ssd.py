@@ -67,6 +67,7 @@ def _declare(lib):
         "ssd_segment_passing": ([P, ctypes.c_int64] + [vp] * 6, ctypes.c_int),
         "ssd_fused_scan": ([P, ctypes.c_int64] + [vp] * 11, ctypes.c_int),
         "ssd_decode_step": ([P] + [vp] * 8, ctypes.c_int),
+        "ssd_discretize": ([P, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp], ctypes.c_int),
     }
     for name, (argtypes, restype) in sig.items():
         f = getattr(lib, name)
@@ -81,7 +82,7 @@ def lib():
         if _lib is None:
             if not os.path.exists(LIB_PATH):
                 raise ImportError(
-                    f"{LIB_PATH} is missing: build it with `python -m mamba_ssd_layer_chunked_b200.build` "
+                    f"{LIB_PATH} is missing: build it with `python mamba_ssd_layer_chunked_b200/build.py` "
                     "(there is no fallback implementation)")
             l = ctypes.CDLL(LIB_PATH)
             _declare(l)
@@ -351,3 +352,21 @@ def decode_step(x: torch.Tensor, log_a: torch.Tensor, B: torch.Tensor, C: torch.
     _check(lib().ssd_decode_step(ctypes.byref(p), _ptr(x), _ptr(log_a), _ptr(B), _ptr(C), _ptr(D), _ptr(state),
                                  _ptr(y), _stream(stream)), "ssd_decode_step")
     return y
+
+
+def discretize(dt: torch.Tensor, A: torch.Tensor, x: torch.Tensor, dt_bias: Optional[torch.Tensor] = None,
+               zoh: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """log_a = softplus(dt + dt_bias) * A and X = s * x (s = delta, or the
+    zero-order-hold (exp(delta A) - 1) / A when zoh): the log_a and X inputs of
+    ssd_fwd. dt [b, T, H] fp32, A and dt_bias [H] fp32, x [b, T, H, P]."""
+    if x.dim() != 4 or dt.shape != x.shape[:3] or A.shape != (x.shape[2],):
+        raise ValueError("shapes: x [b,T,H,P], dt [b,T,H], A [H]")
+    if dt.dtype != torch.float32 or A.dtype != torch.float32 or (dt_bias is not None and dt_bias.dtype != torch.float32):
+        raise TypeError("dt, A and dt_bias must be float32")
+    b, T, H, P = x.shape
+    p = make_problem(b, T, H, P, 16, 1, 64, 1, x.dtype)  # dstate, ngroups, chunk are not read by this step
+    log_a = torch.empty(dt.shape, dtype=torch.float32, device=dt.device)
+    X = torch.empty_like(x)
+    _check(lib().ssd_discretize(ctypes.byref(p), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(x), int(bool(zoh)),
+                                _ptr(log_a), _ptr(X), _stream(stream)), "ssd_discretize")
+    return log_a, X

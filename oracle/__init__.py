@@ -21,6 +21,8 @@ Contents
                        output), tiny sizes only.
 ``recurrence_numpy``   a NumPy twin of the C recurrence for tiny inputs (used to
                        show that the pins catch planted mistakes).
+``discretize``         the step before the scan: softplus step size, log a = delta A,
+                       and x scaled by delta (or by the zero-order hold factor).
 
 Every function takes and returns NumPy arrays; floating inputs are read as
 float64 (bf16/fp32 input values convert exactly).
@@ -33,6 +35,7 @@ from .ssd_oracle import (  # noqa: F401
     dual_matrix,
     blockwise,
     recurrence_numpy,
+    discretize,
     oracle_library_path,
     build_oracle,
     max_threads,

@@ -326,3 +326,26 @@ def recurrence_numpy(X, log_a, B, C, D=None, init_states=None, seq_idx=None, nse
             if seqlen:
                 final[b, cur, h] = H
     return Y, final
+
+
+def discretize(dt, A, x, dt_bias=None, zoh: bool = False):
+    """The step before the scan in the Mamba block, fp64: (log_a [b,T,H], X [b,T,H,P]).
+
+    delta = softplus(dt + dt_bias) and A_bar = exp(delta A) (the Mamba page,
+    ai.tomabc.com paper story 21: the block pseudocode and the discretisation of
+    A); B_bar x is delta B x (zoh False) or the zero-order hold
+    (exp(delta A) - 1) / A B x ("Mamba and state space models", section 2), the
+    scalar put on x: log_a = delta A, X = s x.
+    """
+    dt = np.asarray(dt, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    z = dt + (0.0 if dt_bias is None else np.asarray(dt_bias, dtype=np.float64))
+    delta = np.logaddexp(0.0, z)  # log(1 + e^z)
+    log_a = delta * A
+    if zoh:
+        nz = A != 0.0
+        s = np.where(nz, np.expm1(log_a) / np.where(nz, A, 1.0), delta)
+    else:
+        s = delta
+    X = s[..., None] * np.asarray(x, dtype=np.float64)
+    return log_a, X
