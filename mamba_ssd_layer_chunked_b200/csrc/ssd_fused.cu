@@ -812,8 +812,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             for (int v4 = 0; v4 < 4; ++v4) {
                 const float4 fq = *reinterpret_cast<const float4*>(cf + ((16 * cc + 4 * v4) ^ (4 * hi)));
                 const uint32_t* g4 = g + 4 * v4;
-                w[2 * v4] = pack_bf16(__uint_as_float(g4[0]) * rf * fq.x, __uint_as_float(g4[1]) * rf * fq.y);
-                w[2 * v4 + 1] = pack_bf16(__uint_as_float(g4[2]) * rf * fq.z, __uint_as_float(g4[3]) * rf * fq.w);
+                const float2 r2 = make_float2(rf, rf);
+                const float2 a = __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g4[0]), __uint_as_float(g4[1])), r2),
+                                            make_float2(fq.x, fq.y));
+                const float2 c = __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g4[2]), __uint_as_float(g4[3])), r2),
+                                            make_float2(fq.z, fq.w));
+                w[2 * v4] = pack_bf16(a.x, a.y);
+                w[2 * v4 + 1] = pack_bf16(c.x, c.y);
             }
         };
         auto build_lg = [&](int t) {
@@ -903,7 +908,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // scales v in place, then stores it
         auto st_state_scaled = [&](float (&v)[NQ], float a) {
 #pragma unroll
-            for (int i = 0; i < NQ; ++i) v[i] *= a;
+            for (int i = 0; i < NQ; i += 2) {
+                const float2 sc = __fmul2_rn(make_float2(v[i], v[i + 1]), make_float2(a, a));
+                v[i] = sc.x;
+                v[i + 1] = sc.y;
+            }
             if constexpr (NQ == 32) tmem_st32(tm_h + lane_off + NQ * cq, reinterpret_cast<const uint32_t(&)[32]>(v));
             else tmem_st16(tm_h + lane_off + NQ * cq, reinterpret_cast<const uint32_t(&)[16]>(v));
         };
@@ -1003,8 +1012,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         for (int i = 0; i < 4; ++i) {
                             const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&xu[i]);
                             const int e0 = 8 * c + 2 * i;  // of this half; D x is in Y_diag (L o G diagonal)
-                            out[i] = pack_bf16(fmaf(rs, __uint_as_float(yo[e0]), __uint_as_float(yd[e0])),
-                                               fmaf(rs, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1])));
+                            const float2 yy = __ffma2_rn(make_float2(rs, rs),
+                                                         make_float2(__uint_as_float(yo[e0]), __uint_as_float(yo[e0 + 1])),
+                                                         make_float2(__uint_as_float(yd[e0]), __uint_as_float(yd[e0 + 1])));
+                            out[i] = pack_bf16(yy.x, yy.y);
                             const __nv_bfloat162 xs = __hmul2(xb, wx2);
                             xu[i] = *reinterpret_cast<const uint32_t*>(&xs);
                         }
