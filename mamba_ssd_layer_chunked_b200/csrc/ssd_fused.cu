@@ -269,22 +269,31 @@ __global__ void __launch_bounds__(kSegThreads, 1)
 }
 
 // ===========================================================================
-// segment_passing: per (batch row, head), over the ranges that cover the row
-// in order, H_end = decay * H_start + local for each piece that ends inside
-// the row, with H_start = H_end of the previous piece when the piece's last
-// sequence continues from it, else that sequence's initial state (or zero);
-// and, for each piece that starts inside the row, the state entering it for
-// the sequence of its first token into work_in.
+// segment_passing: for every range i that starts inside its row r, the state
+// entering it for the sequence of its first token. Over the pieces of row r
+// before that cut (ranges i0 .. i-1 in order), H_end = decay * H_start + local,
+// with H_start = H_end of the previous piece when the piece's last sequence
+// continues from it, else that sequence's initial state (or zero); the entering
+// state is H_end of the last piece when the first token continues the previous
+// token's sequence, else its initial state (or zero). One block per (cut, head,
+// slice of the state): the cuts are independent, each chain is a few pieces.
 // ===========================================================================
+constexpr int kPassMaxLinks = 64;  // pieces before a cut handled per block (longer chains loop)
+
 __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, Work wk, const float* __restrict__ work_local,
                                                               const float* __restrict__ work_decay,
                                                               const float* __restrict__ init_states,
                                                               const int32_t* __restrict__ seq_idx,
                                                               float* __restrict__ work_in) {
-    __shared__ int info[4];  // last id, last piece continues, first id, first token continues
-    const int bh = blockIdx.x;
-    const int h = bh % d.nheads, b = bh / d.nheads;
-    const int r = b * wk.npairs + h / 2, hh = h & 1;
+    // per piece j of the chain: last id, last piece continues, and for the cut itself
+    __shared__ int sl_s[kPassMaxLinks], cl_s[kPassMaxLinks];
+    __shared__ int sf_s, cf_s;
+    const int i = blockIdx.x >> 1, hh = blockIdx.x & 1;
+    const int64_t fb = work_begin(wk, i);
+    const int r = (int)(fb / wk.nt);
+    const int64_t rb = (int64_t)r * wk.nt;
+    if (fb == rb) return;  // the range starts at its row start: no entering state needed
+    const int b = r / wk.npairs, h = 2 * (r % wk.npairs) + hh;
     const int NP = d.dstate * d.headdim;
     const int idx = (blockIdx.y * 256 + threadIdx.x) * 4;
     const bool active = idx < NP;
@@ -294,39 +303,49 @@ __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, Work wk, c
         if (!init_states) return zero;
         return *reinterpret_cast<const float4*>(init_states + seqst_off(d, b, sq, h) + idx);
     };
-    const int64_t rb = (int64_t)r * wk.nt;
-    const int i0 = (int)(rb / wk.wt), i1 = (int)((rb + wk.nt - 1) / wk.wt);
+    const int i0 = (int)(rb / wk.wt);
+    const int s_cut = (int)(128 * (fb - rb));  // first token of range i in row r
     float4 H = zero;
-    for (int i = i0; i <= i1; ++i) {
-        int s0, s1;
-        row_piece(wk, d.seqlen, work_begin(wk, i), work_end(wk, i), r, s0, s1);
+    for (int j0 = i0; j0 < i; j0 += kPassMaxLinks) {
+        const int nl = min(kPassMaxLinks, i - j0);
         __syncthreads();
-        if (threadIdx.x == 0) {
-            int sl = 0, cont_last = (s0 > 0), sf = 0, cont_first = (s0 > 0);
+        // sequence information of the pieces [s0, s1) of ranges j0 .. j0+nl-1 in row r
+        for (int l = threadIdx.x; l < nl; l += blockDim.x) {
+            int s0, s1;
+            row_piece(wk, d.seqlen, work_begin(wk, j0 + l), work_end(wk, j0 + l), r, s0, s1);
+            int sl = 0, cont_last = (s0 > 0);
             if (seq_idx) {
                 sl = seq_clamped(seq_idx, row, s1 - 1, d.nseq);
-                sf = seq_clamped(seq_idx, row, s0, d.nseq);
                 const int st = lower_bound_global(seq_idx, row, s0, s1 - 1, sl, d.nseq);
                 const int prev = s0 > 0 ? seq_clamped(seq_idx, row, s0 - 1, d.nseq) : -1;
                 cont_last = (st == s0) && prev == sl;
-                cont_first = prev == sf;
             }
-            info[0] = sl;
-            info[1] = cont_last;
-            info[2] = sf;
-            info[3] = cont_first;
+            sl_s[l] = sl;
+            cl_s[l] = cont_last;
+        }
+        if (threadIdx.x == 0 && j0 + nl == i) {
+            int sf = 0, cont_first = 1;
+            if (seq_idx) {
+                sf = seq_clamped(seq_idx, row, s_cut, d.nseq);
+                cont_first = seq_clamped(seq_idx, row, s_cut - 1, d.nseq) == sf;
+            }
+            sf_s = sf;
+            cf_s = cont_first;
         }
         __syncthreads();
         if (!active) continue;
-        const int64_t o = ((int64_t)i * 2 + hh) * NP + idx;
-        if (s0 > 0) *reinterpret_cast<float4*>(work_in + o) = info[3] ? H : init_of(info[2]);
-        if (s1 < d.seqlen) {
-            const float dec = work_decay[(int64_t)i * 2 + hh];
+#pragma unroll 4
+        for (int l = 0; l < nl; ++l) {
+            const int j = j0 + l;
+            const int64_t o = ((int64_t)j * 2 + hh) * NP + idx;
+            const float dec = work_decay[(int64_t)j * 2 + hh];
             const float4 sv = *reinterpret_cast<const float4*>(work_local + o);
-            const float4 st = info[1] ? H : init_of(info[0]);
+            const float4 st = cl_s[l] ? H : init_of(sl_s[l]);
             H = make_float4(fmaf(dec, st.x, sv.x), fmaf(dec, st.y, sv.y), fmaf(dec, st.z, sv.z), fmaf(dec, st.w, sv.w));
         }
     }
+    if (active)
+        *reinterpret_cast<float4*>(work_in + ((int64_t)i * 2 + hh) * NP + idx) = cf_s ? H : init_of(sf_s);
 }
 
 // ===========================================================================
@@ -1199,7 +1218,7 @@ cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* 
 cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const float* work_local, const float* work_decay,
                                    const float* init_states, const int32_t* seq_idx, float* work_in, cudaStream_t st) {
     const Work w = make_work(d, work_tiles);
-    const dim3 grid(d.batch * d.nheads, (d.dstate * d.headdim + 1023) / 1024);
+    const dim3 grid(2 * w.nwork, (d.dstate * d.headdim + 1023) / 1024);
     segment_passing_kernel<<<grid, 256, 0, st>>>(d, w, work_local, work_decay, init_states, seq_idx, work_in);
     return cudaGetLastError();
 }
