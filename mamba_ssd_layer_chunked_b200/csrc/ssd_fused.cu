@@ -971,11 +971,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
         // ---- prologue: the first piece's state and tile 0's L o G ----
         wait_cs(0);
-        TileDesc cur = csb[0].td;
-        fill_gap(cur);
+        fill_gap(csb[0].td);
         {
-            const float* src = (cur.flags & kTileFromWork) ? work_in + ((int64_t)i_work * 2 + sh) * N * kP
-                                                           : init_src(cur.b, cur.hp, cur.sid);
+            const TileDesc& td0 = csb[0].td;
+            const float* src = (td0.flags & kTileFromWork) ? work_in + ((int64_t)i_work * 2 + sh) * N * kP
+                                                           : init_src(td0.b, td0.hp, td0.sid);
             float hv[NQ];
             load_state(hv, src);
             write_hs(hv);
@@ -992,16 +992,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int t = 0;; ++t) {
             const uint32_t par = t & 1;
             const int st = t & 1;
+            // the descriptors are read from the decay buffers where they are used:
+            // held in registers across the loop they spill at the register cap
+            const TileDesc& cur = csb[t & (kCsBufs - 1)].td;
             const bool fin = (cur.flags & kTileFinal) != 0;
             const float* ct = csb[t & (kCsBufs - 1)].c[eh];
             uint8_t* Xst = smem + S::oX + st * S::kX + eh * kBox;
             const int64_t rowt = (int64_t)cur.b * d.seqlen;
 
             // the next tile's column factor tables while Y(t) is computed
-            TileDesc nx = cur;
+            const TileDesc& nx = csb[(t + 1) & (kCsBufs - 1)].td;  // read only when !fin
             if (!fin) {
                 wait_cs(t + 1);
-                nx = csb[(t + 1) & (kCsBufs - 1)].td;
                 lg_tables(t + 1);
             }
             // ---- epilogue(t): Y staged in Hs (or stored), X' = w X in place ----
@@ -1094,7 +1096,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             signal(&bar_st);
             signal(&bar_csfree[t & (kCsBufs - 1)]);  // done with tile t's decay data
             if (fin) break;
-            cur = nx;
         }
     }
     tc_fence_before();
