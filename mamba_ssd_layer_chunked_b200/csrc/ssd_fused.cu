@@ -355,7 +355,6 @@ constexpr int kComputeWarps = 16;
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kFusedThreads = kComputeThreads + 64;  // + the MMA/TMA control warp and the decay warp
 constexpr int kCsBufs = 4;                           // decay buffers in flight
-constexpr bool kPermRows = false;                     // balanced row order of C (see row_token)
 
 template <int N>
 struct FusedSmem {
@@ -381,22 +380,10 @@ enum : int {
     kTileFromWork = 16  // first tile of a range that starts inside its row
 };
 
-// Token of the tile held by TMEM lane m in G, L o G and the Y accumulators.
-// With kPermRows, C is loaded as eight 16-row blocks so that lane quarter q
-// holds tokens [16 q, 16 q + 16) and [112 - 16 q, 128 - 16 q): every quarter
-// then gets the same share of the causal triangle (tensor memory lane quarter
-// q can only be reached from SM sub-partition q).
-__device__ __forceinline__ int row_token(int m) {
-    if (!kPermRows) return m;
-    const int q = m >> 5, i = m & 15;
-    return (m & 16) ? 112 - 16 * q + i : 16 * q + i;
-}
-
-// 16-row block of the tokens held by lane half hi (lanes 16 hi .. 16 hi + 15) of quarter q
-__device__ __forceinline__ int row_block(int q, int hi) {
-    if (!kPermRows) return 2 * q + hi;
-    return hi ? 7 - q : q;
-}
+// 16-row block of the tokens held by lane half hi (lanes 16 hi .. 16 hi + 15)
+// of TMEM lane quarter q: TMEM lane m holds token m of the tile in G, L o G
+// and the Y accumulators.
+__device__ __forceinline__ int row_block(int q, int hi) { return 2 * q + hi; }
 
 // Per-tile data, written by the decay warp: c[h][k] = log2(e) * the
 // within-tile inclusive cumsum of log a for head h, the whole-tile decays and
@@ -512,22 +499,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 tma_load_4d(Xsg, &tm_x, &bar_bx[st], 0, h0, td.ts, td.b);
                 tma_load_4d(Xsg + kBox, &tm_x, &bar_bx[st], 0, h0 + 1, td.ts, td.b);
             };
-            // C rows in the order of row_token: with kPermRows smem rows
-            // [16 s, 16 s + 16) hold the tokens of row_block(s / 2, s % 2)
             auto load_c = [&](const TileDesc& td) {
                 const int g = 2 * td.hp / d.heads_per_group;
                 mbar_arrive_expect_tx(&bar_c, S::kC);
 #pragma unroll
-                for (int q = 0; q < N / 64; ++q) {
-                    if (kPermRows) {
-#pragma unroll
-                        for (int sblk = 0; sblk < 8; ++sblk)
-                            tma_load_4d(Cs + q * kBox + sblk * 2048, &tm_c, &bar_c, 64 * q, g,
-                                        td.ts + 16 * row_block(sblk >> 1, sblk & 1), td.b);
-                    } else {
-                        tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, td.ts, td.b);
-                    }
-                }
+                for (int q = 0; q < N / 64; ++q) tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, td.ts, td.b);
             };
             const uint32_t ca = smem_u32(Cs), ha = smem_u32(Hs);
             auto issue_g = [&](int t) {
@@ -744,7 +720,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // =================== compute warps ===================
         const int q4 = warp & 3, cq = warp >> 2;
         const int m = 32 * q4 + lane;           // TMEM lane
-        const int k = row_token(m);             // its token in G, L o G and Y
+        const int k = m;                        // its token in G, L o G and Y
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
         const int sh = m >> 6, sp = m & 63;     // state row (head, p) of lane m
 
@@ -759,12 +735,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // Lane half hi holds the 16-row block rb of tokens; column block c (16
         // tokens) is zero above rb, exp2(c_k - c_l) masked on the diagonal block, and
         // below it exp2(c_k - c_{16 rb}) * exp2(c_{16 rb} - c_l), both factors <= 1.
-        // the per-warp column factor tables of tile t (before the wait for Y(t-1))
-        // and this lane's row factors of tile t (rf: to its row block start, rg: to
-        // the middle of the row block, ck: its cumsum) and the pair's D
-        struct RowF {
-            float rf[2], rg[2], ck[2], dd[2];
+        // this lane's row factors for one head: rf to its row block start, rg
+        // to the middle of the row block, ck its cumsum, dd the head's D
+        struct HeadF {
+            float rf, rg, ck, dd;
         };
+        // the per-warp column factor tables of tile t and this lane's row factors
+        // rf, rg of tile t (before the wait for Y(t-1))
         auto lg_tables = [&](int t) {
             const CsBuf& cs = csb[t & (kCsBufs - 1)];
             const int l = 32 * cq + lane;
@@ -796,7 +773,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // exp2(c_k - c_{r+8}) exp2(c_{r+8} - c_l) (both factors <= 1); the
         // diagonal element also carries D_h, so that Y_diag includes D x.
         // g(j) = (selb ? gb : ga)[j] are the block's 16 G values of this lane.
-        auto diag_block = [&](const CsBuf& cs, const RowF& f, int hh, int rb, const uint32_t* ga, const uint32_t* gb,
+        auto diag_block = [&](const CsBuf& cs, const HeadF& f, int hh, int rb, const uint32_t* ga, const uint32_t* gb,
                               bool selb, uint32_t* w) {
             const int hi = lane >> 4, i = lane & 15;
             const bool lo = i < 8;
@@ -812,9 +789,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const uint32_t g0 = selb ? gb[e] : ga[e], g8 = selb ? gb[8 + e] : ga[8 + e];
-                const float v = __uint_as_float(lo ? g0 : g8) * ex2_approx(f.ck[hh] - cv[e]);
-                dv[e] = own + e < i ? v : (own + e == i ? v + f.dd[hh] : 0.f);
-                lv[e] = lo ? dv[e] : __uint_as_float(g0) * f.rg[hh] * fv[e];
+                const float v = __uint_as_float(lo ? g0 : g8) * ex2_approx(f.ck - cv[e]);
+                dv[e] = own + e < i ? v : (own + e == i ? v + f.dd : 0.f);
+                lv[e] = lo ? dv[e] : __uint_as_float(g0) * f.rg * fv[e];
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -823,15 +800,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             }
         };
         // a full block (all columns below the row block) for head hh: 8 packed words
-        auto full_block = [&](const RowF& f, int hh, int cc, const uint32_t* g, uint32_t* w) {
+        auto full_block = [&](const HeadF& f, int hh, int cc, const uint32_t* g, uint32_t* w) {
             const int hi = lane >> 4;
-            const float rf = f.rf[hh];
             const float* cf = &colf[warp][hh][hi][0];
+            const float2 r2 = make_float2(f.rf, f.rf);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
                 const float4 fq = *reinterpret_cast<const float4*>(cf + ((16 * cc + 4 * v4) ^ (4 * hi)));
                 const uint32_t* g4 = g + 4 * v4;
-                const float2 r2 = make_float2(rf, rf);
                 const float2 a = __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g4[0]), __uint_as_float(g4[1])), r2),
                                             make_float2(fq.x, fq.y));
                 const float2 c = __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g4[2]), __uint_as_float(g4[3])), r2),
@@ -840,70 +816,51 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 w[2 * v4 + 1] = pack_bf16(c.x, c.y);
             }
         };
+        // L o G(t) over G(t) in TMEM. Warp (q4, cq) covers row blocks 2 q4,
+        // 2 q4 + 1 and column blocks 2 cq, 2 cq + 1: all zero for cq > q4, all
+        // full for cq < q4, the diagonal pair for cq == q4. G stays in registers
+        // while each head's two 8-column groups go back to TMEM, so the head
+        // loop needs no staging and is not unrolled (code size).
         auto build_lg = [&](int t) {
             const CsBuf& cs = csb[t & (kCsBufs - 1)];
             const int hi = lane >> 4;
             const int rb = row_block(q4, hi);
-            RowF f;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                f.ck[hh] = cs.c[hh][k];
-                f.rf[hh] = rowf_s[hh][tid];
-                f.rg[hh] = rowf_s[2 + hh][tid];
-                f.dd[hh] = Dv ? Dv[2 * cs.td.hp + hh] : 0.f;
-            }
+            const int hp = cs.td.hp;
+            const uint32_t tcol = tm_lg + lane_off + 32 * cq;  // this warp's 32 columns
             __syncwarp();
             mbar_wait(&bar_g, t & 1);
             tc_fence_after();
-            uint32_t gw[32];  // G columns [32 cq, 32 cq + 32), then L o G over them
-            if (2 * cq <= row_block(q4, 1)) {
-                tmem_ld32_async(tm_g + lane_off + 32 * cq, gw);
-                tmem_wait_ld();
-            }
-            if (!kPermRows && cq == q4) {
-                // the diagonal warp of the natural order: lane half hi's diagonal
-                // block is column block hi; block 0 is full for half 1, block 1
-                // zero for half 0. One pass for both halves, no divergence.
-                // own block's G (block hi) into ob, block 0's G for the full part into fb
-                uint32_t ob[16], o0[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) ob[e] = hi ? gw[16 + e] : gw[e];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t dw[8], fw[8];
-                    diag_block(cs, f, hh, rb, ob, ob, false, dw);
-                    full_block(f, hh, 0, gw, fw);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        o0[8 * hh + e] = hi ? fw[e] : dw[e];   // block 0: full (half 1), diagonal (half 0)
-                        gw[16 + 8 * hh + e] = hi ? dw[e] : 0u;  // block 1: diagonal (half 1), zero (half 0)
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) gw[e] = o0[e];
+            if (cq > q4) {
+                const uint32_t z[32] = {};
+                tmem_st32(tcol, z);
             } else {
+                uint32_t gw[32];  // G columns [32 cq, 32 cq + 32)
+                tmem_ld32_async(tcol, gw);
+                tmem_wait_ld();
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    const HeadF f = {rowf_s[hh][tid], rowf_s[2 + hh][tid], cs.c[hh][k], Dv ? Dv[2 * hp + hh] : 0.f};
+                    uint32_t w0[8], w1[8];
+                    if (cq == q4) {
+                        // lane half hi's diagonal block is column block hi; block 0
+                        // is full for half 1, block 1 zero for half 0: one pass for
+                        // both halves, no divergence
+                        uint32_t dw[8], fw[8];
+                        diag_block(cs, f, hh, rb, gw, gw + 16, hi != 0, dw);
+                        full_block(f, hh, 0, gw, fw);
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * cq + cc;  // columns [16 c, 16 c + 16)
-                    const uint32_t* g = gw + 16 * cc;
-                    uint32_t o[16];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t* w = o + 8 * hh;
-                        if (c < rb) {
-                            full_block(f, hh, cc, g, w);
-                        } else if (c == rb) {
-                            diag_block(cs, f, hh, rb, g, g, false, w);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) w[e] = 0u;
+                        for (int e = 0; e < 8; ++e) {
+                            w0[e] = hi ? fw[e] : dw[e];
+                            w1[e] = hi ? dw[e] : 0u;
                         }
+                    } else {
+                        full_block(f, hh, 0, gw, w0);
+                        full_block(f, hh, 1, gw + 16, w1);
                     }
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) gw[16 * cc + e] = o[e];
+                    tmem_st8(tcol + 8 * hh, w0);       // column block 2 cq, head hh
+                    tmem_st8(tcol + 16 + 8 * hh, w1);  // column block 2 cq + 1, head hh
                 }
             }
-            tmem_st32(tm_lg + lane_off + 32 * cq, gw);
             tmem_wait_st();
             tc_fence_before();
             signal(&bar_lg);
@@ -961,7 +918,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             for (int sq = td.psid + 1; sq < td.sid; ++sq) {
                 float* f = final_states + seqst_off(d, td.b, sq, 2 * td.hp + sh);
                 const float* src = init_src(td.b, td.hp, sq);
-#pragma unroll
+#pragma unroll 1
                 for (int i = 0; i < NQ; ++i) {
                     const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
                     f[o] = src ? src[o] : 0.f;
@@ -1078,7 +1035,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     for (int sq = cur.sid + 1; sq < d.nseq; ++sq) {
                         float* f = final_states + seqst_off(d, cur.b, sq, 2 * cur.hp + sh);
                         const float* src = init_src(cur.b, cur.hp, sq);
-#pragma unroll
+#pragma unroll 1
                         for (int i = 0; i < NQ; ++i) {
                             const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
                             f[o] = src ? src[o] : 0.f;
@@ -1231,7 +1188,7 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
     cudaError_t e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
     if ((e = bc_map(&mb, d, B, 128)) != cudaSuccess) return e;
-    if ((e = bc_map(&mc, d, C, kPermRows ? 16 : 128)) != cudaSuccess) return e;  // C in 16-row blocks
+    if ((e = bc_map(&mc, d, C, 128)) != cudaSuccess) return e;
     if ((e = x_map(&my, d, Y, 128)) != cudaSuccess) return e;
     const Work w = make_work(d, work_tiles);
     const dim3 grid(w.nwork);
