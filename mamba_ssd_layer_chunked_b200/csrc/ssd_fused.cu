@@ -353,7 +353,9 @@ __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, Work wk, c
 // ===========================================================================
 constexpr int kComputeWarps = 16;
 constexpr int kComputeThreads = 32 * kComputeWarps;
-constexpr int kFusedThreads = kComputeThreads + 64;  // + the MMA/TMA control warp and the decay warp
+// + two MMA-issue warps, the decay warp and the TMA warp: 5 warps on two of the
+// four SM sub-partitions, which still fits 96 registers a thread
+constexpr int kFusedThreads = kComputeThreads + 128;
 constexpr int kCsBufs = 4;                           // decay buffers in flight
 
 template <int N>
@@ -411,8 +413,11 @@ static_assert(sizeof(CsBuf) % 16 == 0, "CsBuf must keep 16-byte alignment in an 
 //   state(t):     the carried state H(t) (in TMEM: the tile state MMA adds
 //                 X'^T B onto it) to bf16 for the next C H and to the final
 //                 states, then pre-scaled by the next tile's decay.
-// The decay warp runs ahead, filling the decay buffers; the control warp
-// issues the TMA copies and the MMAs.
+// The decay warp runs ahead, filling the decay buffers. One thread each issues
+// the MMAs of the L o G side (G, Y_diag), those of the state side (Y_off, the
+// Y store, the tile state), and the TMA loads: an MMA issue blocks for about
+// the MMA's run time, so one issuing thread would serialise work whose inputs
+// are ready at different times.
 // Tensor memory: G, then L o G in place [0,128); Y_diag [128,256);
 // Y_off [256,384); the carried state H [384,512) (rows (head, p), N columns).
 template <int N>
@@ -438,8 +443,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     __shared__ __align__(16) float cf8[kComputeWarps][2][2][8];
     // per-thread row factors of the next tile: rf (head 0, 1), rg (head 0, 1)
     __shared__ float rowf_s[4][kComputeThreads];
-    __shared__ __align__(8) uint64_t bar_c, bar_bx[2], bar_g, bar_yo, bar_yd, bar_s, bar_lg, bar_epi, bar_st,
-        bar_free, bar_csfull[kCsBufs], bar_csfree[kCsBufs];
+    __shared__ __align__(8) uint64_t bar_c, bar_bx[2], bar_g, bar_yo, bar_yd, bar_s, bar_sfree[2], bar_lg, bar_epi,
+        bar_st, bar_free, bar_csfull[kCsBufs], bar_csfree[kCsBufs];
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -459,6 +464,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         mbar_init(&bar_yo, 1);
         mbar_init(&bar_yd, 1);
         mbar_init(&bar_s, 1);
+        mbar_init(&bar_sfree[0], 1);
+        mbar_init(&bar_sfree[1], 1);
         mbar_init(&bar_lg, kComputeWarps);
         mbar_init(&bar_epi, kComputeWarps);
         mbar_init(&bar_st, kComputeWarps);
@@ -478,16 +485,100 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const uint32_t tm_g = tmem_base, tm_lg = tmem_base, tm_yd = tmem_base + 128, tm_yo = tmem_base + 256,
                    tm_h = tmem_base + 384;
 
+    const uint32_t ca = smem_u32(Cs), ha = smem_u32(Hs);
+    auto stage_x = [&](int t) { return smem_u32(smem + S::oX + (t & 1) * S::kX); };
+    auto stage_b = [&](int t) { return smem_u32(smem + S::oB + (t & 1) * S::kB); };
+    // tile t's descriptor, once the decay warp has published it
+    auto desc = [&](int t) -> TileDesc {
+        mbar_wait(&bar_csfull[t & (kCsBufs - 1)], (t / kCsBufs) & 1);
+        return csb[t & (kCsBufs - 1)].td;
+    };
+    // Every wait below is for an event that cannot be followed by the barrier's
+    // next phase before the waiting thread acts: the thread itself issues, or
+    // loads an operand of, the work that completes that next phase.
     if (warp == kComputeWarps) {
-        // =================== control warp: TMA and MMA issue ===================
+        // =================== MMA issue, L o G side: G(t), Y_diag(t) ===================
         if (lane == 0) {
-            const uint32_t idesc_nn = idesc_bf16(128, 128, false, false);   // K-major A and B
-            const uint32_t idesc_ts = idesc_bf16(128, 64, false, true);     // TMEM A, MN-major B
-            const uint32_t idesc_st = idesc_bf16(128, N, true, true);       // MN-major A and B
-            auto desc = [&](int t) -> TileDesc {
-                mbar_wait(&bar_csfull[t & (kCsBufs - 1)], (t / kCsBufs) & 1);
-                return csb[t & (kCsBufs - 1)].td;
-            };
+            const uint32_t idesc_nn = idesc_bf16(128, 128, false, false);  // K-major A and B
+            const uint32_t idesc_ts = idesc_bf16(128, 64, false, true);    // TMEM A, MN-major B
+            for (int t = 0;; ++t) {
+                const bool fin = (desc(t).flags & kTileFinal) != 0;
+                // G(t) = C(t) B(t)^T once both are in and Y_diag(t-1) has read
+                // L o G(t-1) from the same tensor memory columns
+                mbar_wait(&bar_c, t & 1);
+                mbar_wait(&bar_bx[t & 1], (t >> 1) & 1);
+                if (t > 0) mbar_wait(&bar_yd, (t - 1) & 1);
+                tc_fence_after();
+                const uint32_t ba = stage_b(t);
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
+                    mma_bf16_ss(tm_g, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ba + off, 16, 1024),
+                                idesc_nn, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&bar_g);
+                // Y_diag(t) = (L o G)(t) X(t), A operand from TMEM, once L o G(t) is
+                // built (the compute warps build it after epilogue(t-1) has read
+                // Y_diag(t-1), and before state(t-1))
+                mbar_wait(&bar_lg, t & 1);
+                tc_fence_after();
+                const uint32_t xa = stage_x(t);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 16 * k + 8 * hh,
+                                    smem_desc_sw128(xa + hh * kBox + k * 2048, kBox, 1024), idesc_ts, k > 0 ? 1u : 0u);
+                mma_commit(&bar_yd);
+                if (fin) break;
+            }
+        }
+        __syncwarp();
+    } else if (warp == kComputeWarps + 2) {
+        // =================== MMA issue, state side: Y_off(t), Y store, tile state ===================
+        if (lane == 0) {
+            const uint32_t idesc_nn = idesc_bf16(128, 128, false, false);  // K-major A and B
+            const uint32_t idesc_st = idesc_bf16(128, N, true, true);      // MN-major A and B
+            for (int t = 0;; ++t) {
+                const uint32_t par = t & 1;
+                // Y_off(t) = C(t) Hs once the state before tile t is in Hs
+                mbar_wait(&bar_c, par);
+                mbar_wait(&bar_st, par);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
+                    mma_bf16_ss(tm_yo, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ha + off, 16, 1024),
+                                idesc_nn, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&bar_yo);
+                // epilogue(t) done: store Y(t) from the staging buffer; H += X'^T B
+                mbar_wait(&bar_epi, par);
+                const TileDesc cur = desc(t);
+                tc_fence_after();
+                const bool full = cur.v == 128;
+                if (full) {
+                    tma_store_4d(&tm_y, Hs, 0, 2 * cur.hp, cur.ts, cur.b);
+                    tma_store_4d(&tm_y, Hs + kBox, 0, 2 * cur.hp + 1, cur.ts, cur.b);
+                    tma_store_commit();
+                }
+                const uint32_t xa = stage_x(t), ba = stage_b(t);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ss(tm_h, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
+                                idesc_st, 1u);
+                mma_commit(&bar_s);
+                mma_commit(&bar_sfree[t & 1]);  // the B/X stage of tile t is free
+                if (full) tma_store_wait_read0();
+                mbar_arrive(&bar_free);
+                if (cur.flags & kTileFinal) break;
+            }
+            tma_store_wait0();
+        }
+        __syncwarp();
+    } else if (warp == kComputeWarps + 3) {
+        // =================== TMA loads: C(t), B(t), X(t) ===================
+        if (lane == 0) {
             auto load_bx = [&](const TileDesc& td, int st) {
                 const int h0 = 2 * td.hp, g = h0 / d.heads_per_group;
                 uint8_t* Bsg = smem + S::oB + st * S::kB;
@@ -505,94 +596,26 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 #pragma unroll
                 for (int q = 0; q < N / 64; ++q) tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, td.ts, td.b);
             };
-            const uint32_t ca = smem_u32(Cs), ha = smem_u32(Hs);
-            auto issue_g = [&](int t) {
-                const uint32_t ba = smem_u32(smem + S::oB + (t & 1) * S::kB);
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                    mma_bf16_ss(tm_g, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ba + off, 16, 1024),
-                                idesc_nn, k > 0 ? 1u : 0u);
-                }
-                mma_commit(&bar_g);
-            };
-            TileDesc cur = desc(0), nx = cur;
-            bool has_nx = !(cur.flags & kTileFinal);
-            load_c(cur);
-            load_bx(cur, 0);
-            if (has_nx) {
+            TileDesc nx = desc(0);
+            load_c(nx);
+            load_bx(nx, 0);
+            bool more = !(nx.flags & kTileFinal);
+            if (more) {
                 nx = desc(1);
                 load_bx(nx, 1);
             }
-            mbar_wait(&bar_c, 0);
-            mbar_wait(&bar_bx[0], 0);
-            tc_fence_after();
-            issue_g(0);
-            for (int t = 0;; ++t) {
-                const int st = t & 1;
-                const uint32_t par = t & 1;
-                const uint32_t xa = smem_u32(smem + S::oX + st * S::kX);
-                const uint32_t ba = smem_u32(smem + S::oB + st * S::kB);
-                // Y_diag = (L o G) X, A operand from TMEM: L o G(t) is built before
-                // state(t-1), so this runs while the state update does
-                mbar_wait(&bar_lg, par);
-                tc_fence_after();
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 16 * k + 8 * hh,
-                                    smem_desc_sw128(xa + hh * kBox + k * 2048, kBox, 1024), idesc_ts, k > 0 ? 1u : 0u);
-                mma_commit(&bar_yd);
-                // Y_off = C Hs once the state before this tile is in Hs
-                mbar_wait(&bar_st, par);
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                    mma_bf16_ss(tm_yo, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ha + off, 16, 1024),
-                                idesc_nn, k > 0 ? 1u : 0u);
-                }
-                mma_commit(&bar_yo);
-                // C is free once G(t) and Y_off(t) have read it; G(t+1) once its
-                // operands are in and Y_diag(t) has read L o G(t) from the same columns
-                if (has_nx) {
-                    mbar_wait(&bar_yo, par);
-                    load_c(nx);
-                    mbar_wait(&bar_c, (t + 1) & 1);
-                    mbar_wait(&bar_bx[st ^ 1], ((t + 1) >> 1) & 1);
-                    mbar_wait(&bar_yd, par);
-                    tc_fence_after();
-                    issue_g(t + 1);
-                }
-                // epilogue done: store Y(t) from the staging buffer; H += X'^T B
-                mbar_wait(&bar_epi, par);
-                tc_fence_after();
-                const bool full = cur.v == 128;
-                if (full) {
-                    tma_store_4d(&tm_y, Hs, 0, 2 * cur.hp, cur.ts, cur.b);
-                    tma_store_4d(&tm_y, Hs + kBox, 0, 2 * cur.hp + 1, cur.ts, cur.b);
-                    tma_store_commit();
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16_ss(tm_h, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
-                                idesc_st, 1u);
-                mma_commit(&bar_s);
-                if (full) tma_store_wait_read0();
-                mbar_arrive(&bar_free);
-                if (!has_nx) break;
-                // this stage is free once the tile state has been added
-                TileDesc nx2 = nx;
-                const bool has_nx2 = !(nx.flags & kTileFinal);
-                if (has_nx2) {
-                    nx2 = desc(t + 2);
-                    mbar_wait(&bar_s, par);
-                    load_bx(nx2, st);
-                }
-                cur = nx;
-                nx = nx2;
-                has_nx = has_nx2;
+            for (int t = 0; more; ++t) {
+                // C(t+1) once G(t) and Y_off(t) have read C(t) (at t = 0 the
+                // initial state can release Y_off(0) before G(0) has run)
+                mbar_wait(&bar_g, t & 1);
+                mbar_wait(&bar_yo, t & 1);
+                load_c(nx);
+                more = !(nx.flags & kTileFinal);
+                if (!more) break;
+                // B, X of tile t+2 into tile t's stage once the tile state MMA has read it
+                nx = desc(t + 2);
+                mbar_wait(&bar_sfree[t & 1], (t >> 1) & 1);
+                load_bx(nx, t & 1);
             }
         }
         __syncwarp();
