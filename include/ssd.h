@@ -282,6 +282,47 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
                           const float* init_states, const int32_t* seq_idx, void* Y,
                           float* final_states, void* stream);
 
+/* ---- sequence parallelism: each batch row's tokens in consecutive segments,
+ * one per rank (rank r holds tokens [t_r, t_{r+1}) of every row; segments may
+ * differ in length; seq_idx ids ascend along a row as everywhere) ----
+ * Over a segment the recurrence is affine in its state: the state after the
+ * segment is E = dec * H_start + loc, with loc the state reached from zero at
+ * the start of the segment's last sequence piece and dec the product of a over
+ * that piece (wq-win section 3: a block's local end state and block decay, for
+ * a block that is a whole segment; the pages' sequence-parallel scheme
+ * exchanges these per-segment states once). Per rank: ssd_sp_summary on its
+ * segment, an all-gather of (loc, dec, ids) over the R ranks (in rank order),
+ * ssd_sp_combine for the initial states of its segment, ssd_fwd with them; for
+ * final states, ssd_sp_own_finals on ssd_fwd's final states and a sum over
+ * the ranks. p is the rank's local problem (seqlen = its segment length).
+ *   loc   [batch, nheads, dstate, headdim] fp32     dec [batch, nheads] fp32
+ *   ids   [batch, 2] int32: the segment's first and last sequence id (0, 0
+ *         without seq_idx)
+ *   g_loc, g_dec, g_ids: the R ranks' loc, dec, ids stacked in rank order
+ *   init_states, init_local, final_states [batch, nseq, nheads, dstate, headdim]
+ * ssd_sp_summary covers the FUSED family's domain (SSD_ERR_UNSUPPORTED
+ * elsewhere); dec is 0 where the product is below fp32 range. */
+ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_a, const void* B,
+                          const int32_t* seq_idx, float* loc, float* dec, int32_t* ids, void* stream);
+
+/* init_local[b, s] = the state entering this rank's first token when that
+ * token continues sequence s from the previous rank, else init_states[b, s]
+ * (or zero when init_states is NULL). The state entering rank r is E_{r-1},
+ * chained over ranks j < r: E_j = dec_j * start_j + loc_j, start_j = E_{j-1}
+ * when segment j is one sequence piece continuing rank j-1's last sequence,
+ * else the initial state of segment j's last sequence. Reads only batch,
+ * nheads, dstate, headdim, nseq of p. */
+ssd_status ssd_sp_combine(const ssd_problem* p, int nranks, int rank, const float* g_loc, const float* g_dec,
+                          const int32_t* g_ids, const float* init_states, float* init_local, void* stream);
+
+/* Zeroes final_states[b, s] (in place) unless this rank owns sequence s of
+ * row b: the last rank whose first id is <= s (rank 0 when none is), which
+ * holds s's last token or, for an id that never occurs, reports its initial
+ * state. Summing the ranks' results gives the final states of the whole
+ * sequence. Reads only batch, nheads, dstate, headdim, nseq of p. */
+ssd_status ssd_sp_own_finals(const ssd_problem* p, int nranks, int rank, const int32_t* g_ids, float* final_states,
+                             void* stream);
+
 /* ---- discretisation: the step before the scan in the Mamba block ----
  * For every (b, t, h), with z = dt[b, t, h] + dt_bias[h]:
  *   delta = softplus(z) = log(1 + exp(z)),   log_a[b, t, h] = delta * A[h]

@@ -24,6 +24,9 @@ from .ssd import (  # noqa: F401
     fused_work_tiles,
     segment_passing,
     segment_state,
+    sp_combine,
+    sp_own_finals,
+    sp_summary,
     lib,
     make_problem,
     path_supported,
@@ -35,5 +38,7 @@ from .ssd import (  # noqa: F401
     status_string,
     workspace_bytes,
 )
+
+from .sp import ssd_fwd_sp, torch_collectives  # noqa: F401,E402
 
 lib()  # fail loudly at import when the CUDA library is missing

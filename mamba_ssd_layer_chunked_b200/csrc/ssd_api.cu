@@ -45,9 +45,13 @@ ssd_status check_dims(const ssd_problem* p) {
 }
 
 // The build targets sm_100a only: the device must be compute capability 10.0.
+// Also binds the calling thread to its current device's primary context: this
+// library carries its own CUDA runtime, so a host thread that has not used it
+// before (a thread per rank, say) would otherwise reach the first launch
+// without a current context.
 ssd_status check_device() {
     int dev = 0, major = 0, minor = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) {
         cudaGetLastError();
         return SSD_ERR_UNSUPPORTED;
     }
@@ -295,6 +299,45 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
     if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
     return cuda_status(ssd::launch_fused_scan(d, work_tiles, X, log_a, B, C, D, work_incoming, init_states, seq_idx,
                                               Y, final_states, (cudaStream_t)stream));
+}
+
+ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_a, const void* B,
+                          const int32_t* seq_idx, float* loc, float* dec, int32_t* ids, void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!X || !log_a || !B || !loc || !dec || !ids) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, log_a, B, seq_idx, loc, dec, ids)) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = make_dims(p);
+    if ((s = check_device()) != SSD_OK) return s;
+    if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+    const int64_t nt = ((int64_t)p->seqlen + 127) / 128;  // one work range per (batch row, head pair)
+    return cuda_status(ssd::launch_segment_state(d, nt, X, log_a, B, seq_idx, loc, dec, (cudaStream_t)stream, ids));
+}
+
+ssd_status ssd_sp_combine(const ssd_problem* p, int nranks, int rank, const float* g_loc, const float* g_dec,
+                          const int32_t* g_ids, const float* init_states, float* init_local, void* stream) {
+    ssd_status s = check_dims(p);
+    if (s != SSD_OK) return s;
+    if (nranks < 1 || rank < 0 || rank >= nranks) return SSD_ERR_INVALID_ARG;
+    if (!g_loc || !g_dec || !g_ids || !init_local) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(g_loc, g_dec, g_ids, init_states, init_local)) return SSD_ERR_INVALID_ARG;
+    if ((p->dstate * p->headdim) % 4 != 0) return SSD_ERR_INVALID_ARG;
+    if ((s = check_device()) != SSD_OK) return s;
+    return cuda_status(ssd::launch_sp_combine(make_dims(p), nranks, rank, g_loc, g_dec, g_ids, init_states,
+                                              init_local, (cudaStream_t)stream));
+}
+
+ssd_status ssd_sp_own_finals(const ssd_problem* p, int nranks, int rank, const int32_t* g_ids, float* final_states,
+                             void* stream) {
+    ssd_status s = check_dims(p);
+    if (s != SSD_OK) return s;
+    if (nranks < 1 || rank < 0 || rank >= nranks) return SSD_ERR_INVALID_ARG;
+    if (!g_ids || !final_states) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(g_ids, final_states)) return SSD_ERR_INVALID_ARG;
+    if ((p->dstate * p->headdim) % 4 != 0) return SSD_ERR_INVALID_ARG;
+    if ((s = check_device()) != SSD_OK) return s;
+    return cuda_status(
+        ssd::launch_sp_own_finals(make_dims(p), nranks, rank, g_ids, final_states, (cudaStream_t)stream));
 }
 
 ssd_status ssd_discretize(const ssd_problem* p, const float* dt, const float* dt_bias, const float* A,

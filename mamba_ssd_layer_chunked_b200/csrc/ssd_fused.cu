@@ -98,7 +98,8 @@ template <int N>
 __global__ void __launch_bounds__(kSegThreads, 1)
     segment_state_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b, Dims d,
                          Work wk, const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
-                         float* __restrict__ work_local, float* __restrict__ work_decay) {
+                         float* __restrict__ work_local, float* __restrict__ work_decay, int whole_rows,
+                         int32_t* __restrict__ row_ids) {
     constexpr uint32_t kXB = 2 * kBox, kBB = (N / 64) * kBox, kStage = kXB + kBB;  // two stages
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -109,16 +110,21 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // the last piece of range i, when it ends inside its row
+    // the last piece of range i, when it ends inside its row (or, with
+    // whole_rows, one range per row: the whole row, its ids into row_ids)
     const int i_work = blockIdx.x;
     const int64_t fe = work_end(wk, i_work);
     const int r = (int)((fe - 1) / wk.nt);
     int s0, s1;
     row_piece(wk, d.seqlen, work_begin(wk, i_work), fe, r, s0, s1);
-    if (s1 >= d.seqlen) return;  // ends at the row end: nothing feeds a next range
+    if (s1 >= d.seqlen && !whole_rows) return;  // ends at the row end: nothing feeds a next range
     const int hp = r % wk.npairs, b = r / wk.npairs;
     const int h0 = 2 * hp, g = h0 / d.heads_per_group;
     const int64_t row = (int64_t)b * d.seqlen;
+    if (whole_rows && hp == 0 && tid == 0) {
+        row_ids[2 * b] = seq_idx ? seq_clamped(seq_idx, row, 0, d.nseq) : 0;
+        row_ids[2 * b + 1] = seq_idx ? seq_clamped(seq_idx, row, d.seqlen - 1, d.nseq) : 0;
+    }
 
     if (tid == 0) {
         prefetch_tmap(&tm_x);
@@ -1174,7 +1180,8 @@ size_t fused_workspace_bytes(const Dims& d, int64_t work_tiles) {
 }
 
 cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
-                                 const int32_t* seq_idx, float* work_local, float* work_decay, cudaStream_t st) {
+                                 const int32_t* seq_idx, float* work_local, float* work_decay, cudaStream_t st,
+                                 int32_t* row_ids) {
     CUtensorMap mx, mb;
     cudaError_t e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
@@ -1185,11 +1192,13 @@ cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* 
     if (d.dstate == 64) {
         auto k = segment_state_kernel<64>;
         if ((e = set_smem_attr(k, smem, 30)) != cudaSuccess) return e;
-        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay);
+        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay, row_ids != nullptr,
+                                           row_ids);
     } else if (d.dstate == 128) {
         auto k = segment_state_kernel<128>;
         if ((e = set_smem_attr(k, smem, 31)) != cudaSuccess) return e;
-        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay);
+        k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay, row_ids != nullptr,
+                                           row_ids);
     } else {
         return cudaErrorNotSupported;
     }

@@ -39,8 +39,17 @@ int64_t fused_work_count(const Dims& d, int64_t work_tiles);
 bool fused_needs_cut_states(const Dims& d, int64_t work_tiles);
 size_t fused_workspace_bytes(const Dims& d, int64_t work_tiles);
 
+// row_ids non-null: one range per row (work_tiles = tiles per row), every
+// row's state over its last sequence piece, and its first and last ids
 cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
-                                 const int32_t* seq_idx, float* work_local, float* work_decay, cudaStream_t st);
+                                 const int32_t* seq_idx, float* work_local, float* work_decay, cudaStream_t st,
+                                 int32_t* row_ids = nullptr);
+
+// sequence parallelism (ssd_sp.cu)
+cudaError_t launch_sp_combine(const Dims& d, int nranks, int rank, const float* g_loc, const float* g_dec,
+                              const int32_t* g_ids, const float* init_states, float* init_local, cudaStream_t st);
+cudaError_t launch_sp_own_finals(const Dims& d, int nranks, int rank, const int32_t* g_ids, float* final_states,
+                                 cudaStream_t st);
 cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const float* work_local, const float* work_decay,
                                    const float* init_states, const int32_t* seq_idx, float* work_in, cudaStream_t st);
 cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,

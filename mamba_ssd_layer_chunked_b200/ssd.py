@@ -68,6 +68,9 @@ def _declare(lib):
         "ssd_fused_scan": ([P, ctypes.c_int64] + [vp] * 11, ctypes.c_int),
         "ssd_decode_step": ([P] + [vp] * 8, ctypes.c_int),
         "ssd_discretize": ([P, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp], ctypes.c_int),
+        "ssd_sp_summary": ([P] + [vp] * 8, ctypes.c_int),
+        "ssd_sp_combine": ([P, ctypes.c_int, ctypes.c_int] + [vp] * 6, ctypes.c_int),
+        "ssd_sp_own_finals": ([P, ctypes.c_int, ctypes.c_int, vp, vp, vp], ctypes.c_int),
     }
     for name, (argtypes, restype) in sig.items():
         f = getattr(lib, name)
@@ -329,6 +332,41 @@ def fused_scan(X, log_a, B, C, work_tiles, work_incoming=None, D=None, init_stat
                                 _ptr(work_incoming), _ptr(init_states), _ptr(seq_idx), _ptr(Y), _ptr(final_states),
                                 _stream(stream)), "ssd_fused_scan")
     return Y
+
+
+def sp_summary(X, log_a, B, seq_idx=None, nseq=1, chunk=64, stream=None):
+    """This rank's segment summary: (loc [b, H, N, P] fp32, dec [b, H] fp32,
+    ids [b, 2] int32), with E = dec * H_start + loc over the segment's last
+    sequence piece and ids its first and last sequence ids."""
+    p = _fused_problem(X, B, nseq, chunk)
+    b, _, H, P = X.shape
+    N = B.shape[3]
+    loc = torch.empty((b, H, N, P), dtype=torch.float32, device=X.device)
+    dec = torch.empty((b, H), dtype=torch.float32, device=X.device)
+    ids = torch.empty((b, 2), dtype=torch.int32, device=X.device)
+    _check(lib().ssd_sp_summary(ctypes.byref(p), _ptr(X), _ptr(log_a), _ptr(B), _ptr(seq_idx), _ptr(loc), _ptr(dec),
+                                _ptr(ids), _stream(stream)), "ssd_sp_summary")
+    return loc, dec, ids
+
+
+def sp_combine(X, B, g_loc, g_dec, g_ids, rank, init_states=None, nseq=1, chunk=64, stream=None):
+    """Initial states [b, nseq, H, N, P] of this rank's segment from the R
+    ranks' stacked summaries (g_loc [R, b, H, N, P], g_dec [R, b, H], g_ids [R, b, 2])."""
+    p = problem_from(X, B, chunk, nseq)
+    b, _, H, P = X.shape
+    N = B.shape[3]
+    init_local = torch.empty((b, nseq, H, N, P), dtype=torch.float32, device=X.device)
+    _check(lib().ssd_sp_combine(ctypes.byref(p), int(g_loc.shape[0]), int(rank), _ptr(g_loc), _ptr(g_dec),
+                                _ptr(g_ids), _ptr(init_states), _ptr(init_local), _stream(stream)), "ssd_sp_combine")
+    return init_local
+
+
+def sp_own_finals(X, B, final_states, g_ids, rank, nseq=1, chunk=64, stream=None):
+    """Zero, in place, the final states of sequences this rank does not own."""
+    p = problem_from(X, B, chunk, nseq)
+    _check(lib().ssd_sp_own_finals(ctypes.byref(p), int(g_ids.shape[0]), int(rank), _ptr(g_ids), _ptr(final_states),
+                                   _stream(stream)), "ssd_sp_own_finals")
+    return final_states
 
 
 def decode_step(x: torch.Tensor, log_a: torch.Tensor, B: torch.Tensor, C: torch.Tensor, state: torch.Tensor,

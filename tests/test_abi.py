@@ -167,3 +167,22 @@ def test_binding_rejects_host_tensors_and_bad_shapes():
         _ssd._check_shapes(X.double(), la, B.double(), B.double(), None, None, None, 1)
     with pytest.raises(ValueError):
         _ssd._ptr(X)  # CPU tensor
+
+
+def test_sequence_parallel_entry_points_validate_on_host():
+    lib = ssd.lib()
+    p = prob()
+    # summary: every pointer is required, 16-byte alignment
+    assert lib.ssd_sp_summary(ctypes.byref(p), None, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == INVALID
+    assert lib.ssd_sp_summary(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None) == INVALID
+    assert lib.ssd_sp_summary(ctypes.byref(p), FAKE + 8, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == INVALID
+    assert lib.ssd_sp_summary(ctypes.byref(prob(nseq=2)), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE,
+                              None) == INVALID  # nseq > 1 needs seq_idx
+    # combine and ownership: rank within [0, nranks), buffers present
+    for nranks, rank in ((0, 0), (2, 2), (2, -1)):
+        assert lib.ssd_sp_combine(ctypes.byref(p), nranks, rank, FAKE, FAKE, FAKE, None, FAKE, None) == INVALID
+        assert lib.ssd_sp_own_finals(ctypes.byref(p), nranks, rank, FAKE, FAKE, None) == INVALID
+    assert lib.ssd_sp_combine(ctypes.byref(p), 2, 1, None, FAKE, FAKE, None, FAKE, None) == INVALID
+    assert lib.ssd_sp_combine(ctypes.byref(p), 2, 1, FAKE, FAKE, FAKE, None, None, None) == INVALID
+    assert lib.ssd_sp_own_finals(ctypes.byref(p), 2, 1, None, FAKE, None) == INVALID
+    assert lib.ssd_sp_own_finals(ctypes.byref(p), 2, 1, FAKE, FAKE + 4, None) == INVALID

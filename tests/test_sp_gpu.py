@@ -1,0 +1,157 @@
+"""Sequence parallelism on one GPU: R ranks emulated as threads of one
+process, each holding consecutive token segments of every batch row and
+exchanging its segment summary through in-process collectives. The assembled
+Y and the final states are compared with the fp64 oracle run on the whole
+sequence, under the parity rule max|got - ref| <= tau * max|ref| (tau = 2e-2
+for bf16 inputs with fp32 state). The segment summaries themselves are
+compared with the oracle's state after the segment's last sequence piece.
+"""
+import threading
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import TAU, assert_close, run_oracle, to_device
+from workloads import make_custom
+
+pytestmark = pytest.mark.gpu
+
+# name: (batch, T, H, N, segment lengths, sequence lengths per row, D, init)
+CASES = {
+    "two_equal_one_sequence": (2, 1024, 4, 128, [512, 512], None, "none", True),
+    "three_ragged_segments": (2, 1000, 4, 128, [256, 384, 360], None, "normal", True),
+    "four_segments_N64_zero_init": (1, 1024, 4, 64, [256, 256, 256, 256], None, "none", False),
+    # a sequence boundary exactly at the first segment boundary, others inside
+    "varlen_boundary_at_segment_edge": (2, 1024, 4, 128, [256, 384, 384], [[100, 156, 400, 368], [1024]],
+                                        "normal", True),
+    # ids that never occur, one sequence over three segments, one starting at a rank
+    "skipped_ids": (2, 768, 4, 128, [256, 256, 256], [[100, 0, 412, 0, 256], [0, 768, 0, 0, 0]], "normal", True),
+    # one short segment holding only the middle of a sequence
+    "short_middle_segment": (1, 640, 2, 128, [300, 40, 300], [[200, 400, 40]], "none", True),
+}
+
+
+def _ssd():
+    import mamba_ssd_layer_chunked_b200 as ssd
+    return ssd
+
+
+class ThreadGroup:
+    """all_gather / all_reduce_sum among R threads of one process."""
+
+    def __init__(self, nranks):
+        self.nranks = nranks
+        self.barrier = threading.Barrier(nranks, timeout=60)
+        self.slots = [None] * nranks
+
+    def _exchange(self, rank, t):
+        self.slots[rank] = t
+        self.barrier.wait()
+        parts = list(self.slots)
+        self.barrier.wait()
+        return parts
+
+    def collectives(self, rank):
+        def all_gather(t):
+            return torch.stack(self._exchange(rank, t))
+
+        def all_reduce_sum(t):
+            return torch.stack(self._exchange(rank, t)).sum(dim=0)
+
+        return all_gather, all_reduce_sum
+
+
+def _segments(g, seg):
+    bounds = np.cumsum([0] + list(seg))
+    out = []
+    for r in range(len(seg)):
+        a, b = int(bounds[r]), int(bounds[r + 1])
+        out.append({k: (None if g[k] is None else g[k][:, a:b].contiguous())
+                    for k in ("X", "log_a", "B", "C", "seq_idx")})
+    return out
+
+
+def _case(name):
+    batch, T, H, N, seg, lengths, D, init = CASES[name]
+    assert sum(seg) == T
+    d = make_custom(batch, T, H, 64, N, 1, "bf16", seed=4000 + len(name), has_D=D, has_init=init,
+                    lengths=lengths)
+    return d, seg
+
+
+def _run_threads(d, seg, chunk=256):
+    from mamba_ssd_layer_chunked_b200.sp import ssd_fwd_sp
+    g = to_device(d, "bf16")
+    parts = _segments(g, seg)
+    group = ThreadGroup(len(seg))
+    out = [None] * len(seg)
+    errors = []
+    nseq = d["nseq"] if d["seq_idx"] is not None else None
+
+    def rank_main(r):
+        try:
+            ag, ar = group.collectives(r)
+            p = parts[r]
+            out[r] = ssd_fwd_sp(p["X"], p["log_a"], p["B"], p["C"], chunk, rank=r, all_gather=ag, all_reduce_sum=ar,
+                                D=g["D"], init_states=g["init_states"], seq_idx=p["seq_idx"], nseq=nseq)
+        except BaseException as e:  # reported below
+            errors.append(e)
+            group.barrier.abort()
+
+    threads = [threading.Thread(target=rank_main, args=(r,)) for r in range(len(seg))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    if errors:
+        raise errors[0]
+    torch.cuda.synchronize()
+    Y = torch.cat([o[0] for o in out], dim=1).float().cpu().numpy().astype(np.float64)
+    finals = [o[1].cpu().numpy().astype(np.float64) for o in out]
+    return Y, finals
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_sp_emulated_ranks_match_the_whole_sequence(name):
+    d, seg = _case(name)
+    Y, finals = _run_threads(d, seg)
+    Yr, Fr = run_oracle(d)
+    assert_close(Y, Yr, TAU["bf16"], "Y")
+    for r, F in enumerate(finals):
+        assert_close(F, Fr, TAU["bf16"], f"final_states on rank {r}")
+        assert np.array_equal(F, finals[0]), "ranks disagree on the final states"
+
+
+def _last_piece_start(seq_row, a, b):
+    if seq_row is None:
+        return a
+    last = seq_row[b - 1]
+    return a + int(np.argmax(seq_row[a:b] == last))
+
+
+@pytest.mark.parametrize("name", ["varlen_boundary_at_segment_edge", "three_ragged_segments", "skipped_ids"])
+def test_sp_summary_is_the_state_after_the_last_piece(name):
+    ssd = _ssd()
+    d, seg = _case(name)
+    g = to_device(d, "bf16")
+    parts = _segments(g, seg)
+    bounds = np.cumsum([0] + list(seg))
+    nseq = d["nseq"] if d["seq_idx"] is not None else 1
+    batch, H = d["X"].shape[0], d["X"].shape[2]
+    for r, p in enumerate(parts):
+        loc, dec, ids = ssd.sp_summary(p["X"], p["log_a"], p["B"], seq_idx=p["seq_idx"], nseq=nseq)
+        torch.cuda.synchronize()
+        a, b = int(bounds[r]), int(bounds[r + 1])
+        for bb in range(batch):
+            row = None if d["seq_idx"] is None else d["seq_idx"][bb]
+            st = _last_piece_start(row, a, b)
+            sl = slice(bb, bb + 1), slice(st, b)
+            _, Fr = oracle.ssd_reference(d["X"][sl], d["log_a"][sl], d["B"][sl], d["C"][sl])
+            assert_close(loc[bb].cpu().numpy().astype(np.float64), Fr[0, 0], TAU["bf16"], f"loc r={r} b={bb}")
+            dref = np.exp(d["log_a"][bb, st:b].astype(np.float64).sum(axis=0))
+            # an fp32 sum of the piece's log a: relative error ~1e-6 of |sum| in the exponent
+            assert_close(dec[bb].cpu().numpy().astype(np.float64), dref, 1e-4, f"dec r={r} b={bb}", atol=1e-30)
+            want = (0, 0) if row is None else (int(row[a]), int(row[b - 1]))
+            assert tuple(ids[bb].tolist()) == want
