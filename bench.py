@@ -582,6 +582,31 @@ def _time_device(fn, steps, warmup, stream):
     return e0.elapsed_time(e1) / 1e3 / steps
 
 
+def _time_graph(fn, steps, warmup, stream):
+    """Device time per call of fn replayed from a CUDA graph (no host launch
+    cost in the timed region); the eager timing when capture is not possible."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            fn()
+    except Exception:  # capture refused: fall back to eager launches
+        return _time_device(fn, steps, warmup, stream), False
+    g.replay()
+    torch.cuda.synchronize()
+    s_ = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_)
+    for _ in range(steps):
+        g.replay()
+    e1.record(s_)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / steps, True
+
+
 def run_sweep(args):
     """--mode sweep: ssd_fwd on every workload (device time, inputs resident),
     one JSON line each: tokens*heads/s, TFLOP/s and the fractions of the
@@ -646,6 +671,92 @@ def run_decode(args, w):
     return 0
 
 
+def run_sp(args, w):
+    """--mode sp: the sequence-parallel forward (every batch row's tokens in R
+    consecutive segments). Under torchrun (WORLD_SIZE > 1) it runs over NCCL,
+    one segment per rank, timed on the device as the max over ranks. On one
+    GPU it emulates R = --sp-ranks ranks one after another: it times each
+    rank's summary, combine and forward on its segment (the exchanged
+    summaries are those of the real segments) and reports the slowest rank's
+    sum next to the whole-sequence forward; the exchange itself (an all-gather
+    of R x (b H N P + b H) fp32 + b x 2 int32 per rank, and the final-state sum)
+    is not timed there. One JSON line, not the headline."""
+    import torch
+    import mamba_ssd_layer_chunked_b200 as ssd
+    from mamba_ssd_layer_chunked_b200.sp import ssd_fwd_sp, torch_collectives
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    _, g = _device_inputs(w, dev)
+    stream = torch.cuda.current_stream(dev)
+    seq, nseq = g["seq"], g["nseq"]
+    nseq_arg = nseq if seq is not None else None
+    T = w.seqlen
+    R = world if world > 1 else args.sp_ranks
+    bounds = [T * r // R for r in range(R + 1)]
+    seg = lambda t, r: None if t is None else t[:, bounds[r]:bounds[r + 1]].contiguous()
+    b, H, N, P = w.batch, w.nheads, w.dstate, w.headdim
+    xbytes = R * (b * H * N * P * 4 + b * H * 4 + b * 2 * 4)
+    if world > 1:
+        r = rank
+        X, la, B, C, sq = (seg(g[k], r) for k in ("X", "la", "B", "C", "seq"))
+        ag, ar = torch_collectives()
+        fn = lambda: ssd_fwd_sp(X, la, B, C, w.chunk, rank=r, all_gather=ag, all_reduce_sum=ar, D=g["D"],
+                                init_states=g["init"], seq_idx=sq, nseq=nseq_arg)
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        t = reduce_max(e0.elapsed_time(e1) / 1e3 / args.steps)
+        if rank == 0:
+            print(json.dumps({"mode": "sp", "workload": w.name, "ranks": R, "emulated": False,
+                              "value": w.tokens_heads / t, "unit": "tokens·heads/s", "ms_per_step": t * 1e3,
+                              "exchange_bytes_per_rank": xbytes, "scaling": "strong",
+                              "steps": args.steps, "warmup": args.warmup}), flush=True)
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+        return 0
+    graphs = True
+    def timed(fn):
+        nonlocal graphs
+        t, ok = _time_graph(fn, args.steps, args.warmup, stream)
+        graphs = graphs and ok
+        return t
+    t_full = timed(lambda: ssd.ssd_fwd(g["X"], g["la"], g["B"], g["C"], w.chunk, D=g["D"], init_states=g["init"],
+                                       seq_idx=seq, nseq=nseq_arg))
+    parts = [{k: seg(g[k], r) for k in ("X", "la", "B", "C", "seq")} for r in range(R)]
+    sums = [ssd.sp_summary(q["X"], q["la"], q["B"], seq_idx=q["seq"], nseq=nseq) for q in parts]
+    g_loc, g_dec, g_ids = (torch.stack([s_[i] for s_ in sums]) for i in range(3))
+    per_rank = []
+    for r, q in enumerate(parts):
+        init_local = ssd.sp_combine(q["X"], q["B"], g_loc, g_dec, g_ids, r, init_states=g["init"], nseq=nseq)
+        t_sum = timed(lambda: ssd.sp_summary(q["X"], q["la"], q["B"], seq_idx=q["seq"], nseq=nseq))
+        t_comb = timed(lambda: ssd.sp_combine(q["X"], q["B"], g_loc, g_dec, g_ids, r, init_states=g["init"],
+                                              nseq=nseq))
+        t_fwd = timed(lambda: ssd.ssd_fwd(q["X"], q["la"], q["B"], q["C"], w.chunk, D=g["D"],
+                                          init_states=init_local, seq_idx=q["seq"], nseq=nseq_arg))
+        per_rank.append((t_sum, t_comb, t_fwd))
+    slow = max(per_rank, key=sum)
+    t_rank = sum(slow)
+    print(json.dumps({"mode": "sp", "workload": w.name, "ranks": R, "emulated": True, "cuda_graphs": graphs,
+                      "ms_full_one_gpu": t_full * 1e3, "ms_slowest_rank": t_rank * 1e3,
+                      "slowest_rank_ms": {"summary": slow[0] * 1e3, "combine": slow[1] * 1e3, "forward": slow[2] * 1e3},
+                      "speedup_without_exchange": t_full / t_rank, "exchange_bytes_per_rank": xbytes,
+                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -657,9 +768,11 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--mode", choices=["scan", "sweep", "decode"], default="scan",
-                    help="scan: the headline line (default); sweep: every workload; decode: the decode step")
+    ap.add_argument("--mode", choices=["scan", "sweep", "decode", "sp"], default="scan",
+                    help="scan: the headline line (default); sweep: every workload; decode: the decode step; "
+                         "sp: the sequence-parallel forward")
     ap.add_argument("--decode-batch", type=int, default=64)
+    ap.add_argument("--sp-ranks", type=int, default=4, help="ranks emulated on one GPU by --mode sp")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -670,6 +783,8 @@ def main(argv=None):
         return run_sweep(args)
     if args.mode == "decode":
         return run_decode(args, w)
+    if args.mode == "sp":
+        return run_sp(args, WORKLOADS["long16k_N128"] if args.workload == DEFAULT_WORKLOAD else w)
     return run_ours(args, w)
 
 
