@@ -92,8 +92,8 @@ typedef enum {
 
 typedef struct {
     int64_t batch;     /* b  >= 1 */
-    int64_t seqlen;    /* T  >= 1; a multiple of chunk on the SIMT and TCGEN05 families and the
-                          chunked step entry points, any length on the FUSED family */
+    int64_t seqlen;    /* T  >= 1, any length: on the chunked families the last chunk
+                          may be partial */
     int64_t nheads;    /* H  >= 1, a multiple of ngroups */
     int64_t headdim;   /* P: multiple of 16, <= 256 */
     int64_t dstate;    /* N: multiple of 16, <= 256 */
@@ -173,8 +173,11 @@ ssd_status ssd_fwd_noalloc(const ssd_problem* p, const void* X, const float* log
                            const int32_t* seq_idx, void* Y, float* final_states, void* stream);
 
 /* ---- the four steps, callable one by one (ssd_fwd runs them in this order) ----
- * nchunks = seqlen / chunk. cs is [batch, nheads, nchunks, chunk] fp32; a "state
- * buffer" is [batch, nchunks, nheads, dstate, headdim] fp32. */
+ * nchunks = ceil(seqlen / chunk). cs is [batch, nheads, nchunks, chunk] fp32; a
+ * "state buffer" is [batch, nchunks, nheads, dstate, headdim] fp32. Positions of
+ * a partial last chunk past the row end count as tokens with log a = 0 and
+ * x = B = C = 0 in the last token's sequence: they change no state, cs stays
+ * constant over them, and no Y is written for them. */
 
 /* Bytes of one state buffer. */
 size_t ssd_states_bytes(const ssd_problem* p);

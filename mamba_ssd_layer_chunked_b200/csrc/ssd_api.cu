@@ -36,7 +36,7 @@ ssd_status check_dims(const ssd_problem* p) {
     if (p->headdim % 16 != 0 || p->headdim > 256 || p->dstate % 16 != 0 || p->dstate > 256)
         return SSD_ERR_UNSUPPORTED;
     // grid and index limits: every flattened grid dimension stays below 2^31
-    const int64_t nchunks = p->seqlen / p->chunk;
+    const int64_t nchunks = (p->seqlen + p->chunk - 1) / p->chunk;
     if (p->batch > (1 << 20) || p->seqlen > (1 << 26) || p->nheads > (1 << 16) || p->nseq > (1 << 24))
         return SSD_ERR_UNSUPPORTED;
     if (p->batch * p->nheads * nchunks * 4 > INT32_MAX) return SSD_ERR_UNSUPPORTED;
@@ -73,22 +73,23 @@ ssd::Dims make_dims(const ssd_problem* p) {
     d.ngroups = (int)p->ngroups;
     d.chunk = (int)p->chunk;
     d.nseq = (int)p->nseq;
-    d.nchunks = (int)(p->seqlen / p->chunk);
+    d.nchunks = (int)((p->seqlen + p->chunk - 1) / p->chunk);  // the last chunk may be partial
     d.heads_per_group = (int)(p->nheads / p->ngroups);
     return d;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t cs_bytes(const ssd_problem* p) { return (size_t)p->batch * p->seqlen * p->nheads * sizeof(float); }
+// chunks per row: the last one is partial when chunk does not divide seqlen
+int64_t chunk_count(const ssd_problem* p) { return (p->seqlen + p->chunk - 1) / p->chunk; }
 
-size_t states_bytes(const ssd_problem* p) {
-    return (size_t)p->batch * (p->seqlen / p->chunk) * p->nheads * p->dstate * p->headdim * sizeof(float);
+size_t cs_bytes(const ssd_problem* p) {
+    return (size_t)p->batch * chunk_count(p) * p->chunk * p->nheads * sizeof(float);
 }
 
-// The chunked families and their step entry points need whole chunks; the
-// fused family takes any sequence length.
-bool chunked_ok(const ssd_problem* p) { return p->seqlen % p->chunk == 0; }
+size_t states_bytes(const ssd_problem* p) {
+    return (size_t)p->batch * chunk_count(p) * p->nheads * p->dstate * p->headdim * sizeof(float);
+}
 
 // kernels of the chunked steps (chunk_state, chunk_scan)
 bool use_tc(const ssd_problem* p) {
@@ -105,7 +106,7 @@ ssd_path fwd_family(const ssd_problem* p) {
         default: break;
     }
     if (ssd::fused_fwd_supported(p)) return SSD_PATH_FUSED;
-    if (ssd::tc_supported(p) && chunked_ok(p)) return SSD_PATH_TCGEN05;
+    if (ssd::tc_supported(p)) return SSD_PATH_TCGEN05;
     return SSD_PATH_SIMT;
 }
 
@@ -184,7 +185,6 @@ ssd_status check_runnable(const ssd_problem* p) {
     if (s != SSD_OK) return s;
     if (p->path == SSD_PATH_TCGEN05 && !ssd::tc_supported(p)) return SSD_ERR_UNSUPPORTED;
     if (p->path == SSD_PATH_FUSED && !ssd::fused_fwd_supported(p)) return SSD_ERR_UNSUPPORTED;
-    if (fwd_family(p) != SSD_PATH_FUSED && !chunked_ok(p)) return SSD_ERR_UNSUPPORTED;
     return SSD_OK;
 }
 
@@ -221,20 +221,20 @@ ssd_status ssd_check_problem(const ssd_problem* p) {
 
 int ssd_path_supported(const ssd_problem* p, ssd_path path) {
     if (check_dims(p) != SSD_OK || check_device() != SSD_OK) return 0;
-    if (path == SSD_PATH_SIMT) return chunked_ok(p) ? 1 : 0;
-    if (path == SSD_PATH_TCGEN05) return ssd::tc_supported(p) && chunked_ok(p) ? 1 : 0;
+    if (path == SSD_PATH_SIMT) return 1;
+    if (path == SSD_PATH_TCGEN05) return ssd::tc_supported(p) ? 1 : 0;
     if (path == SSD_PATH_FUSED) return ssd::fused_fwd_supported(p) ? 1 : 0;
     return 0;
 }
 
 size_t ssd_states_bytes(const ssd_problem* p) {
-    if (check_dims(p) != SSD_OK || !chunked_ok(p)) return (size_t)-1;
+    if (check_dims(p) != SSD_OK) return (size_t)-1;
     return states_bytes(p);
 }
 
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
     if (check_dims(p) != SSD_OK) return (size_t)-1;
-    size_t need = chunked_ok(p) ? chunked_workspace_bytes(p) : 0;
+    size_t need = chunked_workspace_bytes(p);
     if (ssd::fused_fwd_supported(p)) {
         const size_t f = fused_layout(p).total;
         if (f > need) need = f;
@@ -384,7 +384,6 @@ ssd_status ssd_decode_step(const ssd_problem* p, const void* x, const float* log
 ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs, void* stream) {
     ssd_status s = check_dims(p);  // log a only: nseq and seq_idx play no part here
     if (s != SSD_OK) return s;
-    if (!chunked_ok(p)) return SSD_ERR_UNSUPPORTED;
     if (!log_a || !cs) return SSD_ERR_INVALID_ARG;
     if (!all_aligned(log_a, cs)) return SSD_ERR_INVALID_ARG;
     if ((s = check_device()) != SSD_OK) return s;
@@ -395,7 +394,6 @@ ssd_status ssd_chunk_state(const ssd_problem* p, const void* X, const void* B, c
                            const int32_t* seq_idx, float* states, float* final_states, void* stream) {
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
-    if (!chunked_ok(p)) return SSD_ERR_UNSUPPORTED;
     if (!X || !B || !cs || !states) return SSD_ERR_INVALID_ARG;
     if (!all_aligned(X, B, cs, seq_idx, states, final_states)) return SSD_ERR_INVALID_ARG;
     if ((s = check_runnable(p)) != SSD_OK) return s;
@@ -410,7 +408,6 @@ ssd_status ssd_state_passing(const ssd_problem* p, const float* cs, const float*
                              void* stream) {
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
-    if (!chunked_ok(p)) return SSD_ERR_UNSUPPORTED;
     if (!cs || !chunk_states || !incoming) return SSD_ERR_INVALID_ARG;
     if (!all_aligned(cs, chunk_states, incoming, init_states, seq_idx, final_states)) return SSD_ERR_INVALID_ARG;
     if ((s = check_runnable(p)) != SSD_OK) return s;
@@ -423,7 +420,6 @@ ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, co
                           const int32_t* seq_idx, void* Y, void* stream) {
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
-    if (!chunked_ok(p)) return SSD_ERR_UNSUPPORTED;
     if (!X || !B || !C || !cs || !incoming || !Y) return SSD_ERR_INVALID_ARG;
     if (!all_aligned(X, B, C, cs, D, incoming, init_states, seq_idx, Y)) return SSD_ERR_INVALID_ARG;
     if ((s = check_runnable(p)) != SSD_OK) return s;

@@ -33,6 +33,14 @@ __device__ __forceinline__ int seq_at(const int32_t* seq_idx, int64_t row_off, i
     return s < 0 ? 0 : (s >= nseq ? nseq - 1 : s);
 }
 
+// the id of token t of a chunk position that may lie past the row end: the
+// positions after the last token of a partial last chunk take the last token's
+// id, so that they extend its sequence piece (with log a = 0 and x = B = C = 0
+// they change no state and no output)
+__device__ __forceinline__ int seq_at_padded(const int32_t* seq_idx, int64_t row_off, int t, int seqlen, int nseq) {
+    return seq_at(seq_idx, row_off, t < seqlen ? t : seqlen - 1, nseq);
+}
+
 // Flat offsets (int64 so that large problems cannot overflow).
 __host__ __device__ __forceinline__ int64_t x_off(const Dims& d, int b, int t, int h) {
     return (((int64_t)b * d.seqlen + t) * d.nheads + h) * d.headdim;

@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kThreads) chunk_cumsum_kernel(Dims d, const fl
     for (int i = threadIdx.x; i < Q * 32; i += kThreads) {
         const int k = i >> 5, j = i & 31;
         float v = 0.f;
-        if (j < nh) v = log_a[((int64_t)b * d.seqlen + (int64_t)c * Q + k) * d.nheads + h0 + j];
+        if (j < nh && c * Q + k < d.seqlen) v = log_a[((int64_t)b * d.seqlen + (int64_t)c * Q + k) * d.nheads + h0 + j];
         slab[k][j] = v;
     }
     __syncthreads();
@@ -80,7 +80,7 @@ __device__ void load_chunk_meta(const Dims& d, const float* cs, const int32_t* s
     const int64_t row = (int64_t)b * d.seqlen;
     for (int k = threadIdx.x; k < Q; k += blockDim.x) {
         m.cs[k] = cs[cs_off(d, b, h, c) + k];
-        m.seq[k] = seq_at(seq_idx, row, c * Q + k, d.nseq);
+        m.seq[k] = seq_at_padded(seq_idx, row, c * Q + k, d.seqlen, d.nseq);
     }
     __syncthreads();
     // ids are non-decreasing inside a chunk (in contract): the piece start is the
@@ -163,12 +163,13 @@ __global__ void __launch_bounds__(kThreads) chunk_state_simt_kernel(Dims d, cons
             const int nl = min(32, e - l0 + 1);
             for (int i = threadIdx.x; i < 32 * N; i += kThreads) {
                 const int li = i / N, n = i % N;
-                Bs[i] = li < nl ? to_f32(B[bc_off(d, b, t0 + l0 + li, g) + n]) : 0.f;
+                Bs[i] = li < nl && t0 + l0 + li < d.seqlen ? to_f32(B[bc_off(d, b, t0 + l0 + li, g) + n]) : 0.f;
             }
             for (int i = threadIdx.x; i < 32 * P; i += kThreads) {
                 const int li = i / P, p = i % P;
                 float v = 0.f;
-                if (li < nl) v = expf(cs_end - m.cs[l0 + li]) * to_f32(X[x_off(d, b, t0 + l0 + li, h) + p]);
+                if (li < nl && t0 + l0 + li < d.seqlen)
+                    v = expf(cs_end - m.cs[l0 + li]) * to_f32(X[x_off(d, b, t0 + l0 + li, h) + p]);
                 Xs[i] = v;
             }
             __syncthreads();
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kThreads) state_passing_kernel(Dims d, const f
         const float* csr = cs + cs_off(d, b, h, c);
         if (seq_idx) {
             __syncthreads();
-            if (threadIdx.x < Q) seqbuf[threadIdx.x] = seq_at(seq_idx, row, c * Q + threadIdx.x, d.nseq);
+            if (threadIdx.x < Q) seqbuf[threadIdx.x] = seq_at_padded(seq_idx, row, c * Q + threadIdx.x, d.seqlen, d.nseq);
             __syncthreads();
             chunk_pieces(seqbuf, Q, pstart, pseq, &npieces, warp_tot);
         }
@@ -319,8 +320,10 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_simt_kernel(
     float* Hs = Ws + kRows * 33;    // [32][P]
     load_chunk_meta(d, cs, seq_idx, b, h, c, m);
     const int k0 = rt * kRows, t0 = c * Q;
-    for (int i = threadIdx.x; i < kRows * N; i += kThreads)
-        Cs[(i / N) * NS + i % N] = to_f32(C[bc_off(d, b, t0 + k0 + i / N, g) + i % N]);
+    for (int i = threadIdx.x; i < kRows * N; i += kThreads) {
+        const int t = t0 + k0 + i / N;  // positions past the row end: C = 0
+        Cs[(i / N) * NS + i % N] = t < d.seqlen ? to_f32(C[bc_off(d, b, t, g) + i % N]) : 0.f;
+    }
     __syncthreads();
 
     const int nout = kRows * P / kThreads;
@@ -373,9 +376,14 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_simt_kernel(
     // ---- diagonal block: masked (L o C B^T) X over column tiles of 32 ----
     for (int l0 = 0; l0 < k0 + kRows; l0 += 32) {
         __syncthreads();
-        for (int i = threadIdx.x; i < 32 * N; i += kThreads)
-            Bs[(i / N) * NS + i % N] = to_f32(B[bc_off(d, b, t0 + l0 + i / N, g) + i % N]);
-        for (int i = threadIdx.x; i < 32 * P; i += kThreads) Xs[i] = to_f32(X[x_off(d, b, t0 + l0 + i / P, h) + i % P]);
+        for (int i = threadIdx.x; i < 32 * N; i += kThreads) {
+            const int t = t0 + l0 + i / N;
+            Bs[(i / N) * NS + i % N] = t < d.seqlen ? to_f32(B[bc_off(d, b, t, g) + i % N]) : 0.f;
+        }
+        for (int i = threadIdx.x; i < 32 * P; i += kThreads) {
+            const int t = t0 + l0 + i / P;
+            Xs[i] = t < d.seqlen ? to_f32(X[x_off(d, b, t, h) + i % P]) : 0.f;
+        }
         __syncthreads();
         for (int i = threadIdx.x; i < kRows * 32; i += kThreads) {
             const int rr = i / 32, li = i % 32;
@@ -409,6 +417,7 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_simt_kernel(
         if (j < nout) {
             const int o = j * kThreads + threadIdx.x;
             const int rr = o / P, p = o % P;
+            if (t0 + k0 + rr >= d.seqlen) continue;  // past the row end of a partial last chunk
             const int64_t off = x_off(d, b, t0 + k0 + rr, h) + p;
             float y = acc[j];
             if (D) y = fmaf(dh, to_f32(X[off]), y);

@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     const int64_t row = (int64_t)b * d.seqlen;
     for (int i = tid; i < 2 * Q; i += kTcThreads) cs_s[i / Q][i % Q] = cs[cs_off(d, b, h0 + i / Q, c) + i % Q];
-    for (int k = tid; k < Q; k += kTcThreads) seq_s[k] = seq_at(seq_idx, row, c * Q + k, d.nseq);
+    for (int k = tid; k < Q; k += kTcThreads) seq_s[k] = seq_at_padded(seq_idx, row, c * Q + k, d.seqlen, d.nseq);
     __syncthreads();
     for (int k = tid; k < Q; k += kTcThreads) {
         const int v = seq_s[k];
@@ -236,6 +236,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int h0 = 2 * hp, g = h0 / d.heads_per_group;
     const int t0 = c * Q;  // first token of the chunk
     const int k0 = 128 * rb;  // first row of this block inside the chunk
+    // a row block wholly past the end of a partial last chunk has no output:
+    // leave before any setup, so that no TMA copy starts past the row end
+    if (t0 + k0 >= d.seqlen) return;
 
     if (tid == 0) {
         prefetch_tmap(&tm_x);
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     const int64_t row = (int64_t)b * d.seqlen;
     for (int i = tid; i < 2 * Q; i += kTcThreads) cs_s[i / Q][i % Q] = cs[cs_off(d, b, h0 + i / Q, c) + i % Q];
-    for (int k = tid; k < Q; k += kTcThreads) seq_s[k] = seq_at(seq_idx, row, t0 + k, d.nseq);
+    for (int k = tid; k < Q; k += kTcThreads) seq_s[k] = seq_at_padded(seq_idx, row, t0 + k, d.seqlen, d.nseq);
     if (tid == 0) multi_piece = 0;
     __syncthreads();
     for (int k = tid; k < Q; k += kTcThreads) {

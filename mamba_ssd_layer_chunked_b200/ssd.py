@@ -240,7 +240,7 @@ def chunk_cumsum(log_a: torch.Tensor, chunk: int, stream=None) -> torch.Tensor:
     """cs [b, H, nchunks, chunk] fp32: the within-chunk inclusive cumsum of log a."""
     b, T, H = log_a.shape
     p = make_problem(b, T, H, 16, 16, 1, chunk, 1, torch.float32)
-    cs = torch.empty((b, H, T // chunk, chunk), dtype=torch.float32, device=log_a.device)
+    cs = torch.empty((b, H, -(-T // chunk), chunk), dtype=torch.float32, device=log_a.device)
     _check(lib().ssd_chunk_cumsum(ctypes.byref(p), _ptr(log_a), _ptr(cs), _stream(stream)), "ssd_chunk_cumsum")
     return cs
 
@@ -252,7 +252,7 @@ def chunk_state(X, B, cs, chunk, seq_idx=None, nseq=1, final_partials: Optional[
     p = problem_from(X, B, chunk, nseq, path)
     b, T, H, P = X.shape
     N = B.shape[3]
-    states = torch.empty((b, T // chunk, H, N, P), dtype=torch.float32, device=X.device)
+    states = torch.empty((b, -(-T // chunk), H, N, P), dtype=torch.float32, device=X.device)
     _check(lib().ssd_chunk_state(ctypes.byref(p), _ptr(X), _ptr(B), _ptr(cs), _ptr(seq_idx), _ptr(states),
                                  _ptr(final_partials), _stream(stream)), "ssd_chunk_state")
     return states

@@ -83,18 +83,16 @@ def test_bad_problem_rejected(field, value, expect):
     assert lib.ssd_fwd(ctypes.byref(p), *([FAKE] * 9), FAKE, 1 << 30, None) == expect
 
 
-def test_ragged_length_needs_the_fused_family():
-    # T % Q != 0: the chunked families refuse it, the fused family (bf16, P 64) takes it
+def test_ragged_length_is_supported_by_every_family():
+    # T % Q != 0: the last chunk is partial (host-side sizes only; the GPU
+    # parity tests run ragged lengths on every family). No call reaches a launch.
     lib = ssd.lib()
-    for path in (1, 2):
-        p = prob(seqlen=500, path=path)
-        assert lib.ssd_fwd(ctypes.byref(p), *([FAKE] * 9), FAKE, 1 << 30, None) == UNSUPPORTED
-    p = prob(seqlen=500, dtype=ssd.ssd.SSD_DTYPE_F32)  # AUTO falls to SIMT
-    assert lib.ssd_fwd(ctypes.byref(p), *([FAKE] * 9), FAKE, 1 << 30, None) == UNSUPPORTED
-    assert lib.ssd_states_bytes(ctypes.byref(p)) == ctypes.c_size_t(-1).value
-    assert lib.ssd_chunk_cumsum(ctypes.byref(p), FAKE, FAKE, None) == UNSUPPORTED
-    q = prob(seqlen=500)  # AUTO, bf16: the fused family
-    assert ssd.workspace_bytes(q) > 0
+    p = prob(seqlen=500)  # bf16, P 64, N 128
+    f = prob(seqlen=500, dtype=ssd.ssd.SSD_DTYPE_F32)  # fp32: the SIMT family
+    assert lib.ssd_check_problem(ctypes.byref(f)) in (OK, UNSUPPORTED)  # UNSUPPORTED only without a B200
+    nchunks = -(-500 // 256)
+    assert lib.ssd_states_bytes(ctypes.byref(f)) == 2 * nchunks * 4 * 128 * 64 * 4
+    assert ssd.workspace_bytes(p) > 0 and ssd.workspace_bytes(f) > 0
 
 
 def test_null_problem_rejected():

@@ -72,6 +72,10 @@ SMALL = {
                               "normal", True),
     "f32_skipped_ids_Q64": (2, 256, 3, 32, 48, 1, 64, "f32", [[60, 0, 100, 96], [0, 256, 0, 0]], "normal", True),
     "f32_P16_N16_Q128": (1, 384, 5, 16, 16, 1, 128, "f32", None, "ones", False),
+    # partial last chunks on the chunked families too
+    "f32_ragged_T300_Q64": (2, 300, 3, 32, 48, 1, 64, "f32", [[100, 200], [300]], "normal", True),
+    "f32_ragged_T70_Q128": (1, 70, 2, 16, 16, 1, 128, "f32", None, "ones", True),
+    "bf16_ragged_boundary_in_last_chunk": (1, 700, 4, 64, 128, 1, 256, "bf16", [[600, 100]], "normal", True),
 }
 
 
