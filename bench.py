@@ -6,7 +6,7 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = one ssd_fwd call, the whole forward path over one batch of the
 workload with its inputs resident in HBM: on the fused family (the default
-for bf16) segment_state, segment_passing and fused_scan; on the chunked
+for bf16) segment_state and fused_scan (which chains the cuts); on the chunked
 families chunk_cumsum, chunk_state, state_passing and chunk_scan. The default workload is the Mamba-2-2.7B-shaped layer (batch 4, T 4096,
 80 heads, P 64, N 128, Q 256, bf16 in / fp32 state). Its inputs (~360 MB) are
 larger than L2, so no flush runs between steps. Prints one JSON line on rank 0.
@@ -110,9 +110,11 @@ def kernel_model(w, wt=None):
       segment_state   reads X, B, log a of the last piece of every range that
                       ends inside a row; writes one fp32 state and one decay per
                       such range and head; 2 N P flops per token and head walked.
-      segment_passing reads those states and decays, writes one incoming state
+      segment_passing (the step entry point; ssd_fwd folds it into fused_scan)
+                      reads those states and decays, writes one incoming state
                       per range start inside a row and head; 2 N P flops each.
-      fused_scan      reads X, B, C, log a, D, the incoming states at the cuts and
+      fused_scan      reads X, B, C, log a, D, the states and decays of the pieces
+                      before its cut (one piece per cut at the bench shapes) and
                       the initial states; writes Y and the final states; per
                       (b, tile, h) 128*129 P + 4*128 N P flops, per (b, tile, g) 128*129 N.
     """
@@ -434,18 +436,17 @@ def run_ours(args, w):
         stb = nwork * 2 * N * P * 4
         al = lambda x: (x + 255) // 256 * 256
         wloc = wsp[:stb].view(torch.float32)
-        win = wsp[al(stb): al(stb) + stb].view(torch.float32)
         wdec = wsp[2 * al(stb): 2 * al(stb) + nwork * 2 * 4].view(torch.float32)
         cuts = nwork > 1 and wt % -(-T // 128) != 0
         names, launches = [], []
-        if cuts:
-            names += ["segment_state", "segment_passing"]
-            launches += [
-                lambda: lib.ssd_segment_state(pr, wt, vp(X), vp(la), vp(B), vp(seq), vp(wloc), vp(wdec), sp),
-                lambda: lib.ssd_segment_passing(pr, wt, vp(wloc), vp(wdec), vp(init), vp(seq), vp(win), sp)]
+        if cuts:  # the launches of ssd_fwd: segment_state, then the scan chaining the cuts itself
+            names.append("segment_state")
+            launches.append(
+                lambda: lib.ssd_segment_state(pr, wt, vp(X), vp(la), vp(B), vp(seq), vp(wloc), vp(wdec), sp))
         names.append("fused_scan")
-        launches.append(lambda: lib.ssd_fused_scan(pr, wt, vp(X), vp(la), vp(B), vp(C), vp(D),
-                                                   vp(win) if cuts else None, vp(init), vp(seq), vp(Y), vp(F), sp))
+        launches.append(lambda: lib.ssd_fused_scan_chained(pr, wt, vp(X), vp(la), vp(B), vp(C), vp(D),
+                                                           vp(wloc) if cuts else None, vp(wdec) if cuts else None,
+                                                           vp(init), vp(seq), vp(Y), vp(F), sp))
     else:
         pk = ssd.problem_from(X, B, w.chunk, inputs["nseq"], "tcgen05" if fam == "tcgen05" else "simt")
         pr = ctypes.byref(pk)

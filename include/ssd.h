@@ -326,6 +326,17 @@ ssd_status ssd_sp_combine(const ssd_problem* p, int nranks, int rank, const floa
 ssd_status ssd_sp_own_finals(const ssd_problem* p, int nranks, int rank, const int32_t* g_ids, float* final_states,
                              void* stream);
 
+/* ssd_fused_scan with the centre factors folded in: each range that starts
+ * inside a row chains the pieces of that row before its cut itself, from
+ * work_local / work_decay (the output of ssd_segment_state), by the rule of
+ * ssd_segment_passing; ssd_fwd runs the fused family as ssd_segment_state
+ * then this. work_local and work_decay may be NULL when no range starts
+ * inside a row. */
+ssd_status ssd_fused_scan_chained(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a,
+                                  const void* B, const void* C, const float* D, const float* work_local,
+                                  const float* work_decay, const float* init_states, const int32_t* seq_idx,
+                                  void* Y, float* final_states, void* stream);
+
 /* ---- discretisation: the step before the scan in the Mamba block ----
  * For every (b, t, h), with z = dt[b, t, h] + dt_bias[h]:
  *   delta = softplus(z) = log(1 + exp(z)),   log_a[b, t, h] = delta * A[h]

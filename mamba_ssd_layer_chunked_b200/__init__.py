@@ -20,6 +20,7 @@ from .ssd import (  # noqa: F401
     discretize,
     declared_functions,
     fused_scan,
+    fused_scan_chained,
     fused_work_count,
     fused_work_tiles,
     segment_passing,

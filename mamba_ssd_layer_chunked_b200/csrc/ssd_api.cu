@@ -161,15 +161,11 @@ cudaError_t run_fused(const ssd::Dims& d, const void* X, const float* log_a, con
     float* work_decay = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * align256(stb));
     const bool cuts = ssd::fused_needs_cut_states(d, wt);
     cudaError_t e = cudaSuccess;
-    if (cuts) {
-        if ((e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st)) != cudaSuccess)
-            return e;
-        if ((e = ssd::launch_segment_passing(d, wt, work_local, work_decay, init_states, seq_idx, work_in, st)) !=
-            cudaSuccess)
-            return e;
-    }
-    return ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, cuts ? work_in : nullptr, init_states, seq_idx, Y,
-                                  final_states, st);
+    (void)work_in;  // the fused scan chains the pieces before each cut itself
+    if (cuts && (e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st)) != cudaSuccess)
+        return e;
+    return ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, nullptr, init_states, seq_idx, Y, final_states, st,
+                                  cuts ? work_local : nullptr, cuts ? work_decay : nullptr);
 }
 
 ssd_status check_common(const ssd_problem* p, const int32_t* seq_idx) {
@@ -299,6 +295,24 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
     if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
     return cuda_status(ssd::launch_fused_scan(d, work_tiles, X, log_a, B, C, D, work_incoming, init_states, seq_idx,
                                               Y, final_states, (cudaStream_t)stream));
+}
+
+ssd_status ssd_fused_scan_chained(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a,
+                                  const void* B, const void* C, const float* D, const float* work_local,
+                                  const float* work_decay, const float* init_states, const int32_t* seq_idx,
+                                  void* Y, float* final_states, void* stream) {
+    ssd_status s = check_common(p, seq_idx);
+    if (s != SSD_OK) return s;
+    if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, log_a, B, C, D, work_local, work_decay, init_states, seq_idx, Y, final_states))
+        return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = make_dims(p);
+    if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
+    if (ssd::fused_needs_cut_states(d, work_tiles) && (!work_local || !work_decay)) return SSD_ERR_INVALID_ARG;
+    if ((s = check_device()) != SSD_OK) return s;
+    if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+    return cuda_status(ssd::launch_fused_scan(d, work_tiles, X, log_a, B, C, D, nullptr, init_states, seq_idx, Y,
+                                              final_states, (cudaStream_t)stream, work_local, work_decay));
 }
 
 ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_a, const void* B,

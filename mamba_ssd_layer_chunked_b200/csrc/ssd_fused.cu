@@ -433,7 +433,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                       Work wk, const float* __restrict__ log_a, const float* __restrict__ Dv,
                       const float* __restrict__ work_in, const float* __restrict__ init_states,
                       const int32_t* __restrict__ seq_idx, __nv_bfloat16* __restrict__ Y,
-                      float* __restrict__ final_states) {
+                      float* __restrict__ final_states, const float* __restrict__ work_local,
+                      const float* __restrict__ work_decay) {
     using S = FusedSmem<N>;
     constexpr int NQ = N / 4;  // state columns per thread
     extern __shared__ uint8_t smem_raw[];
@@ -960,10 +961,52 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         fill_gap(csb[0].td);
         {
             const TileDesc& td0 = csb[0].td;
-            const float* src = (td0.flags & kTileFromWork) ? work_in + ((int64_t)i_work * 2 + sh) * N * kP
-                                                           : init_src(td0.b, td0.hp, td0.sid);
             float hv[NQ];
-            load_state(hv, src);
+            if (!(td0.flags & kTileFromWork)) {
+                load_state(hv, init_src(td0.b, td0.hp, td0.sid));
+            } else if (work_in) {
+                load_state(hv, work_in + ((int64_t)i_work * 2 + sh) * N * kP);
+            } else {
+                // The range starts inside its row: the state entering its first
+                // token from the pieces of the row before the cut (ranges i0 ..
+                // i_work - 1, each E = dec * start + loc from segment_state), with
+                // start = the previous piece's E when the piece's last sequence
+                // continues from it, else that sequence's initial state (or zero);
+                // the entering state is the last E when the first token
+                // continues the previous token's sequence, else its initial state.
+                const int64_t fb = work_begin(wk, i_work);
+                const int r = (int)(fb / wk.nt);
+                const int64_t rb = (int64_t)r * wk.nt;
+                const int b = r / wk.npairs, hp = r % wk.npairs;
+                const int64_t row = (int64_t)b * d.seqlen;
+                const int s_cut = (int)(128 * (fb - rb));
+#pragma unroll
+                for (int i = 0; i < NQ; ++i) hv[i] = 0.f;
+                for (int j = (int)(rb / wk.wt); j < i_work; ++j) {
+                    int s0, s1;
+                    row_piece(wk, d.seqlen, work_begin(wk, j), work_end(wk, j), r, s0, s1);
+                    int sl = 0;
+                    bool cont = s0 > 0;
+                    if (seq_idx) {
+                        sl = seq_clamped(seq_idx, row, s1 - 1, d.nseq);
+                        const int st = lower_bound_global(seq_idx, row, s0, s1 - 1, sl, d.nseq);
+                        cont = st == s0 && s0 > 0 && seq_clamped(seq_idx, row, s0 - 1, d.nseq) == sl;
+                    }
+                    const float a = work_decay[(int64_t)j * 2 + sh];
+                    const float* loc = work_local + ((int64_t)j * 2 + sh) * N * kP;
+                    const float* is = cont ? nullptr : init_src(b, hp, sl);
+#pragma unroll
+                    for (int i = 0; i < NQ; ++i) {
+                        const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
+                        const float start = cont ? hv[i] : (is ? is[o] : 0.f);
+                        hv[i] = fmaf(a, start, loc[o]);
+                    }
+                }
+                if (seq_idx) {
+                    const int sf = seq_clamped(seq_idx, row, s_cut, d.nseq);
+                    if (seq_clamped(seq_idx, row, s_cut - 1, d.nseq) != sf) load_state(hv, init_src(b, hp, sf));
+                }
+            }
             write_hs(hv);
             st_state_scaled(hv, csb[0].dec[sh]);
             tmem_wait_st();
@@ -1215,7 +1258,8 @@ cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const floa
 
 cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
                               const void* C, const float* D, const float* work_in, const float* init_states,
-                              const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st) {
+                              const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st,
+                              const float* work_local, const float* work_decay) {
     CUtensorMap mx, mb, mc, my;
     cudaError_t e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
@@ -1229,13 +1273,13 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
         const int smem = fused_smem_bytes<64>();
         if ((e = set_smem_attr(k, smem, 32)) != cudaSuccess) return e;
         k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx,
-                                             (__nv_bfloat16*)Y, final_states);
+                                             (__nv_bfloat16*)Y, final_states, work_local, work_decay);
     } else if (d.dstate == 128) {
         auto k = fused_scan_kernel<128>;
         const int smem = fused_smem_bytes<128>();
         if ((e = set_smem_attr(k, smem, 33)) != cudaSuccess) return e;
         k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx,
-                                             (__nv_bfloat16*)Y, final_states);
+                                             (__nv_bfloat16*)Y, final_states, work_local, work_decay);
     } else {
         return cudaErrorNotSupported;
     }

@@ -52,9 +52,13 @@ cudaError_t launch_sp_own_finals(const Dims& d, int nranks, int rank, const int3
                                  cudaStream_t st);
 cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const float* work_local, const float* work_decay,
                                    const float* init_states, const int32_t* seq_idx, float* work_in, cudaStream_t st);
+// work_in (the output of segment_passing) or, when it is null, work_local and
+// work_decay (the output of segment_state): the kernel then chains the pieces
+// before each range's cut itself
 cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
                               const void* C, const float* D, const float* work_in, const float* init_states,
-                              const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st);
+                              const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st,
+                              const float* work_local = nullptr, const float* work_decay = nullptr);
 
 // state-dimension slices (ssd_pad.cu)
 cudaError_t launch_pad_bc(const void* src, void* dst, int64_t rows, int N, int n0, int w, int Np, cudaStream_t st);

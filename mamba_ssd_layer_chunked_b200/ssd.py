@@ -66,6 +66,7 @@ def _declare(lib):
         "ssd_segment_state": ([P, ctypes.c_int64] + [vp] * 7, ctypes.c_int),
         "ssd_segment_passing": ([P, ctypes.c_int64] + [vp] * 6, ctypes.c_int),
         "ssd_fused_scan": ([P, ctypes.c_int64] + [vp] * 11, ctypes.c_int),
+        "ssd_fused_scan_chained": ([P, ctypes.c_int64] + [vp] * 12, ctypes.c_int),
         "ssd_decode_step": ([P] + [vp] * 8, ctypes.c_int),
         "ssd_discretize": ([P, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp], ctypes.c_int),
         "ssd_sp_summary": ([P] + [vp] * 8, ctypes.c_int),
@@ -367,6 +368,19 @@ def sp_own_finals(X, B, final_states, g_ids, rank, nseq=1, chunk=64, stream=None
     _check(lib().ssd_sp_own_finals(ctypes.byref(p), int(g_ids.shape[0]), int(rank), _ptr(g_ids), _ptr(final_states),
                                    _stream(stream)), "ssd_sp_own_finals")
     return final_states
+
+
+def fused_scan_chained(X, log_a, B, C, work_tiles, work_local=None, work_decay=None, D=None, init_states=None,
+                       seq_idx=None, nseq=1, final_states: Optional[torch.Tensor] = None, chunk=64,
+                       stream=None) -> torch.Tensor:
+    """Y from segment_state's range states, the cuts chained inside the scan."""
+    p = _fused_problem(X, B, nseq, chunk)
+    Y = torch.empty_like(X)
+    _check(lib().ssd_fused_scan_chained(ctypes.byref(p), int(work_tiles), _ptr(X), _ptr(log_a), _ptr(B), _ptr(C),
+                                        _ptr(D), _ptr(work_local), _ptr(work_decay), _ptr(init_states),
+                                        _ptr(seq_idx), _ptr(Y), _ptr(final_states), _stream(stream)),
+           "ssd_fused_scan_chained")
+    return Y
 
 
 def decode_step(x: torch.Tensor, log_a: torch.Tensor, B: torch.Tensor, C: torch.Tensor, state: torch.Tensor,

@@ -65,7 +65,7 @@ SMALL = {
     "bf16_short_seqs": (1, 512, 2, 64, 64, 1, 256, "bf16", [[1, 1, 3, 250, 1, 256]], "normal", True),
     "f32_varlen_P32_N48_Q64": (2, 320, 3, 32, 48, 1, 64, "f32", [[1, 63, 64, 100, 92], [320]], "normal", True),
     "bf16_ragged_tile_Q64": (2, 576, 4, 64, 128, 1, 64, "bf16", [[200, 376], [576]], "normal", True),
-    # T not a multiple of Q (or of the 128-token tile): the fused family only
+    # T not a multiple of Q (or of the 128-token tile)
     "bf16_ragged_T1000_Q256": (2, 1000, 4, 64, 128, 1, 256, "bf16", [[400, 600], [1000]], "normal", True),
     # ids that never occur (zero-length sequences): they keep their initial state
     "bf16_skipped_ids_Q128": (2, 512, 4, 64, 128, 1, 128, "bf16", [[100, 0, 300, 0, 112], [512, 0, 0, 0, 0]],
@@ -239,6 +239,7 @@ def test_fused_steps(name, wt):
         _close_where(inc2.cpu().numpy().astype(np.float64), inc_ref, 1e-5, "range incoming (oracle inputs)")
         work_in = torch.from_numpy(np.ascontiguousarray(inc_ref, dtype=np.float32)).cuda()
     else:
+        loc = dec = inc = None
         work_in = None
     # fused_scan fed the oracle's incoming range states
     F = torch.full((b, nseq, H, N, P), float("nan"), dtype=torch.float32, device="cuda")
@@ -247,6 +248,18 @@ def test_fused_steps(name, wt):
     torch.cuda.synchronize()
     assert_close(Y.float().cpu().numpy().astype(np.float64), Yr, tau, "fused_scan Y")
     assert_close(F.cpu().numpy().astype(np.float64), Fr, tau, "fused_scan final states")
+    # the chained scan (the cuts chained inside it, as ssd_fwd runs it) gives what
+    # segment_passing + fused_scan give: the same fp32 chain in the same order
+    F1 = torch.full_like(F, float("nan"))
+    Y1 = ssd.fused_scan(X, g["log_a"], B, C, wt, inc, D=g["D"], init_states=g["init_states"],
+                        seq_idx=g["seq_idx"], nseq=nseq, final_states=F1)
+    F2 = torch.full_like(F, float("nan"))
+    Y2 = ssd.fused_scan_chained(X, g["log_a"], B, C, wt, loc, dec, D=g["D"], init_states=g["init_states"],
+                                seq_idx=g["seq_idx"], nseq=nseq, final_states=F2)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2), "chained scan Y differs from segment_passing + fused_scan"
+    assert torch.equal(F1.nan_to_num(7.0), F2.nan_to_num(7.0)), "chained scan final states differ"
+    assert_close(Y2.float().cpu().numpy().astype(np.float64), Yr, tau, "fused_scan_chained Y")
 
 
 # --------------------------------------------------------------------------- #
