@@ -92,7 +92,8 @@ __device__ __forceinline__ void row_piece(const Work& w, int seqlen, int64_t fb,
 // ===========================================================================
 // segment_state
 // ===========================================================================
-constexpr int kSegThreads = 256;
+constexpr int kSegScale = 256;                 // the warps that scale X and own the accumulator lanes
+constexpr int kSegThreads = kSegScale + 32;    // + one warp that issues the MMAs
 
 template <int N>
 __global__ void __launch_bounds__(kSegThreads, 1)
@@ -100,13 +101,17 @@ __global__ void __launch_bounds__(kSegThreads, 1)
                          Work wk, const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
                          float* __restrict__ work_local, float* __restrict__ work_decay, int whole_rows,
                          int32_t* __restrict__ row_ids) {
-    constexpr uint32_t kXB = 2 * kBox, kBB = (N / 64) * kBox, kStage = kXB + kBB;  // two stages
+    constexpr uint32_t kXB = 2 * kBox, kBB = (N / 64) * kBox, kStage = kXB + kBB;
+    // three stages: tile it scaled, tile it - 1 multiplied, tile it + 1 loading
+    constexpr int kStages = 3;
+    constexpr uint32_t kScaleBar = 1;  // named barrier of the scaling warps
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     __shared__ float wsum[8];
     __shared__ float tail_s[2];
     __shared__ int st_shared;
-    __shared__ __align__(8) uint64_t bar_load[2], bar_mma[2];
+    __shared__ int n_iter;  // iterations scaled (set when the scaling warps stop)
+    __shared__ __align__(8) uint64_t bar_load[kStages], bar_mma[kStages], bar_scaled[kStages];
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -129,10 +134,11 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     if (tid == 0) {
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_b);
-        mbar_init(&bar_load[0], 1);
-        mbar_init(&bar_load[1], 1);
-        mbar_init(&bar_mma[0], 1);
-        mbar_init(&bar_mma[1], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bar_load[s], 1);
+            mbar_init(&bar_mma[s], 1);
+            mbar_init(&bar_scaled[s], 1);
+        }
         mbar_fence_init();
         // start of the segment's last sequence piece
         int st = s0;
@@ -141,6 +147,7 @@ __global__ void __launch_bounds__(kSegThreads, 1)
             st = lower_bound_global(seq_idx, row, s0, s1 - 1, sl, d.nseq);
         }
         st_shared = st;
+        n_iter = 1 << 30;
         tail_s[0] = tail_s[1] = 0.f;
     }
     if (warp == 0) {
@@ -153,121 +160,143 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     const uint32_t tacc = tmem_base;
     const int st = st_shared;
     const int ntiles = (s1 - st + 127) / 128;
-    const int rr = tid & 127, hh = tid >> 7;  // this thread's row and head in the transform
-    const uint32_t idesc = idesc_bf16(128, N, true, true);
-    float tail = 0.f;  // sum of log a after the current tile, this thread's head
     bool cut = false;
-    // log a of this thread's (row, head) in a tile; unconditional (clamped row)
-    // so that the prefetch does not stall until the value is used
-    auto load_la = [&](int i) -> float {
-        const int ts = st + 128 * i;
-        const int v = min(128, s1 - ts);
-        return log_a[(row + ts + min(rr, v - 1)) * d.nheads + h0 + hh];
-    };
-    // tile i's X (two heads) and B into stage sg
-    auto issue_load = [&](int i, int sg) {
-        const int ts = st + 128 * i;
-        uint8_t* xs = smem + sg * kStage;
-        uint8_t* bs = xs + kXB;
-        mbar_arrive_expect_tx(&bar_load[sg], kStage);
-        tma_load_4d(xs, &tm_x, &bar_load[sg], 0, h0, ts, b);
-        tma_load_4d(xs + kBox, &tm_x, &bar_load[sg], 0, h0 + 1, ts, b);
+    int lm = 0;  // the last iteration scaled (and multiplied)
+    if (warp == kSegScale / 32) {
+        // ---- MMA issue: S += (weighted X)^T B for every scaled tile, in order ----
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, N, true, true);
+            for (int it = 0;; ++it) {
+                const int sg = it % kStages;
+                mbar_wait(&bar_scaled[sg], (it / kStages) & 1);
+                if (it >= *reinterpret_cast<volatile int*>(&n_iter)) break;  // the scaling warps stopped
+                tc_fence_after();
+                const uint32_t xa = smem_u32(smem + sg * kStage), ba = xa + kXB;
 #pragma unroll
-        for (int q = 0; q < N / 64; ++q) tma_load_4d(bs + q * kBox, &tm_b, &bar_load[sg], 64 * q, g, ts, b);
-    };
-    float la_cur = load_la(ntiles - 1);
-    if (tid == 0) issue_load(ntiles - 1, 0);
-    // tiles from the end backwards, two stages: the load of the tile before
-    // runs while this one is scaled and multiplied
-    int it = 0;
-    for (int i = ntiles - 1; i >= 0; --i, ++it) {
-        const int sg = it & 1;
-        const int ts = st + 128 * i;
-        const int v = min(128, s1 - ts);
-        const float la_nxt = i > 0 ? load_la(i - 1) : 0.f;
-        if (tid == 0 && i > 0) {
-            if (it >= 1) mbar_wait(&bar_mma[sg ^ 1], ((it - 1) >> 1) & 1);  // its stage was read by the last MMAs
-            issue_load(i - 1, sg ^ 1);
-        }
-        // within-tile inclusive cumsum of log a (one row per thread, one head per 4 warps)
-        float x = rr < v ? la_cur : 0.f;
-        la_cur = la_nxt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane == 31) wsum[warp] = x;
-        __syncthreads();
-        float pre = 0.f, tot = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const float sw = wsum[4 * hh + w];
-            if (w < (warp & 3)) pre += sw;
-            tot += sw;
-        }
-        const float cs = x + pre;
-        // weight of row rr: prod of a over (rr, segment end] = exp(tail + tot - cs)
-        const float wgt = rr < v ? ex2_approx((tail + tot - cs) * kLog2e) : 0.f;
-        mbar_wait(&bar_load[sg], (it >> 1) & 1);
-        // scale row rr of head hh in place; the chunk order is rotated by row so
-        // that the 32 rows of a warp spread over all banks
-        uint8_t* Xs = smem + sg * kStage;
-        {
-            uint8_t* rowp = Xs + hh * kBox + rr * 128;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                const int c = (cc + rr) & 7;
-                uint4 vv = *reinterpret_cast<uint4*>(rowp + 16 * c);
-                uint32_t* u = reinterpret_cast<uint32_t*>(&vv);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u[k]));
-                    u[k] = pack_bf16(f.x * wgt, f.y * wgt);
-                }
-                *reinterpret_cast<uint4*>(rowp + 16 * c) = vv;
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ss(tacc, smem_desc_sw128(xa + k * 2048, kBox, 1024),
+                                smem_desc_sw128(ba + k * 2048, kBox, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&bar_mma[sg]);
             }
         }
-        fence_async_shared();
-        __syncthreads();
+        __syncwarp();
+    } else {
+        const int rr = tid & 127, hh = tid >> 7;  // this thread's row and head in the transform
+        float tail = 0.f;  // sum of log a after the current tile, this thread's head
+        // log a of this thread's (row, head) in a tile; unconditional (clamped row)
+        // so that the prefetch does not stall until the value is used
+        auto load_la = [&](int i) -> float {
+            const int ts = st + 128 * i;
+            const int v = min(128, s1 - ts);
+            return log_a[(row + ts + min(rr, v - 1)) * d.nheads + h0 + hh];
+        };
+        // tile i's X (two heads) and B into stage sg
+        auto issue_load = [&](int i, int sg) {
+            const int ts = st + 128 * i;
+            uint8_t* xs = smem + sg * kStage;
+            uint8_t* bs = xs + kXB;
+            mbar_arrive_expect_tx(&bar_load[sg], kStage);
+            tma_load_4d(xs, &tm_x, &bar_load[sg], 0, h0, ts, b);
+            tma_load_4d(xs + kBox, &tm_x, &bar_load[sg], 0, h0 + 1, ts, b);
+#pragma unroll
+            for (int q = 0; q < N / 64; ++q) tma_load_4d(bs + q * kBox, &tm_b, &bar_load[sg], 64 * q, g, ts, b);
+        };
+        float la_cur = load_la(ntiles - 1);
+        if (tid == 0) issue_load(ntiles - 1, 0);
+        // tiles from the end backwards; iteration it holds tile ntiles - 1 - it in
+        // stage it % 3 (its use it / 3): while it is scaled, the MMAs of it - 1
+        // run and tile it + 1 loads into the stage of it - 2
+        int it = 0;
+        for (int i = ntiles - 1; i >= 0; --i, ++it) {
+            const int sg = it % kStages;
+            const int ts = st + 128 * i;
+            const int v = min(128, s1 - ts);
+            const float la_nxt = i > 0 ? load_la(i - 1) : 0.f;
+            if (tid == 0 && i > 0) {
+                const int sn = (it + 1) % kStages;
+                if (it >= 2) mbar_wait(&bar_mma[sn], ((it - 2) / kStages) & 1);  // read by the MMAs of it - 2
+                issue_load(i - 1, sn);
+            }
+            // within-tile inclusive cumsum of log a (one row per thread, one head per 4 warps)
+            float x = rr < v ? la_cur : 0.f;
+            la_cur = la_nxt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) wsum[warp] = x;
+            named_bar_sync(kScaleBar, kSegScale);
+            float pre = 0.f, tot = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float sw = wsum[4 * hh + w];
+                if (w < (warp & 3)) pre += sw;
+                tot += sw;
+            }
+            const float cs = x + pre;
+            // weight of row rr: prod of a over (rr, segment end] = exp(tail + tot - cs)
+            const float wgt = rr < v ? ex2_approx((tail + tot - cs) * kLog2e) : 0.f;
+            mbar_wait(&bar_load[sg], (it / kStages) & 1);
+            // scale row rr of head hh in place; the chunk order is rotated by row so
+            // that the 32 rows of a warp spread over all banks
+            uint8_t* Xs = smem + sg * kStage;
+            {
+                uint8_t* rowp = Xs + hh * kBox + rr * 128;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int c = (cc + rr) & 7;
+                    uint4 vv = *reinterpret_cast<uint4*>(rowp + 16 * c);
+                    uint32_t* u = reinterpret_cast<uint32_t*>(&vv);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u[k]));
+                        u[k] = pack_bf16(f.x * wgt, f.y * wgt);
+                    }
+                    *reinterpret_cast<uint4*>(rowp + 16 * c) = vv;
+                }
+            }
+            fence_async_shared();
+            tail += tot;
+            if (rr == 0) tail_s[hh] = tail;
+            named_bar_sync(kScaleBar, kSegScale);
+            if (tid == 0) mbar_arrive(&bar_scaled[sg]);  // the MMA warp may multiply tile it
+            // everything further back decays below fp32 range for both heads
+            if (tail_s[0] < -104.f && tail_s[1] < -104.f && i > 0) {
+                cut = true;
+                break;
+            }
+        }
+        lm = cut ? it : it - 1;
         if (tid == 0) {
-            tc_fence_after();
-            const uint32_t xa = smem_u32(Xs), ba = smem_u32(Xs + kXB);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16_ss(tacc, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
-                            idesc, (it > 0 || k > 0) ? 1u : 0u);
-            mma_commit(&bar_mma[sg]);
+            // stop the MMA warp at iteration lm + 1
+            n_iter = lm + 1;
+            mbar_arrive(&bar_scaled[(lm + 1) % kStages]);
+            // after a cut at tile i >= 1: the load issued for tile i - 1
+            if (cut) mbar_wait(&bar_load[(lm + 1) % kStages], ((lm + 1) / kStages) & 1);
         }
-        tail += tot;
-        if (rr == 0) tail_s[hh] = tail;
-        __syncthreads();
-        // everything further back decays below fp32 range for both heads
-        if (tail_s[0] < -104.f && tail_s[1] < -104.f && i > 0) {
-            cut = true;
-            break;
-        }
+        // the last MMAs (in order, so all of them)
+        mbar_wait(&bar_mma[lm % kStages], (lm / kStages) & 1);
     }
-    // the last MMAs (iteration lm) and, after a cut, the load issued for the tile before
-    const int lm = cut ? it : it - 1;
-    mbar_wait(&bar_mma[lm & 1], (lm >> 1) & 1);
-    if (cut && tid == 0) mbar_wait(&bar_load[(lm + 1) & 1], ((lm + 1) >> 1) & 1);
+    __syncthreads();
     tc_fence_after();
-    // epilogue: lane m = (head, p); warps w and w+4 split the N columns
-    const int m = 32 * (warp & 3) + lane, half = warp >> 2;
-    const int eh = m >> 6, p = m & 63;
-    float* dst = work_local + ((int64_t)i_work * 2 + eh) * N * kP;
-    const uint32_t lane_addr = tacc + ((uint32_t)(32 * (warp & 3)) << 16);
+    if (warp < kSegScale / 32) {
+        // epilogue: lane m = (head, p); warps w and w+4 split the N columns
+        const int m = 32 * (warp & 3) + lane, half = warp >> 2;
+        const int eh = m >> 6, p = m & 63;
+        float* dst = work_local + ((int64_t)i_work * 2 + eh) * N * kP;
+        const uint32_t lane_addr = tacc + ((uint32_t)(32 * (warp & 3)) << 16);
 #pragma unroll
-    for (int n0 = 0; n0 < N / 2; n0 += 32) {
-        float vv[32];
-        tmem_ld32(lane_addr + half * (N / 2) + n0, vv);
+        for (int n0 = 0; n0 < N / 2; n0 += 32) {
+            float vv[32];
+            tmem_ld32(lane_addr + half * (N / 2) + n0, vv);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) dst[(int64_t)(half * (N / 2) + n0 + k) * kP + p] = vv[k];
-    }
-    if (tid < 2) {
-        const float t = tail_s[tid];
-        work_decay[(int64_t)i_work * 2 + tid] = cut ? 0.f : ex2_approx(t * kLog2e);
+            for (int k = 0; k < 32; ++k) dst[(int64_t)(half * (N / 2) + n0 + k) * kP + p] = vv[k];
+        }
+        if (tid < 2) {
+            const float t = tail_s[tid];
+            work_decay[(int64_t)i_work * 2 + tid] = cut ? 0.f : ex2_approx(t * kLog2e);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1231,7 +1260,7 @@ cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* 
     if ((e = bc_map(&mb, d, B, 128)) != cudaSuccess) return e;
     const Work w = make_work(d, work_tiles);
     const dim3 grid(w.nwork);
-    const int smem = 2 * (2 * (int)kBox + (d.dstate / 64) * (int)kBox) + 1024;
+    const int smem = 3 * (2 * (int)kBox + (d.dstate / 64) * (int)kBox) + 1024;
     if (d.dstate == 64) {
         auto k = segment_state_kernel<64>;
         if ((e = set_smem_attr(k, smem, 30)) != cudaSuccess) return e;
