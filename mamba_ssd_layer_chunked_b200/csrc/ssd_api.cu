@@ -165,7 +165,7 @@ cudaError_t run_fused(const ssd::Dims& d, const void* X, const float* log_a, con
     if (cuts && (e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st)) != cudaSuccess)
         return e;
     return ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, nullptr, init_states, seq_idx, Y, final_states, st,
-                                  cuts ? work_local : nullptr, cuts ? work_decay : nullptr);
+                                  cuts ? work_local : nullptr, cuts ? work_decay : nullptr, cuts);
 }
 
 ssd_status check_common(const ssd_problem* p, const int32_t* seq_idx) {

@@ -115,6 +115,9 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the scan that follows may start its setup and first tile now: it waits
+    // for this grid before it reads the range states
+    griddep_launch_dependents();
     // the last piece of range i, when it ends inside its row (or, with
     // whole_rows, one range per row: the whole row, its ids into row_ids)
     const int i_work = blockIdx.x;
@@ -985,9 +988,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             }
         };
 
-        // ---- prologue: the first piece's state and tile 0's L o G ----
+        // ---- prologue: tile 0's L o G and the first piece's state ----
         wait_cs(0);
         fill_gap(csb[0].td);
+        lg_tables(0);
+        build_lg(0);
         {
             const TileDesc& td0 = csb[0].td;
             float hv[NQ];
@@ -1009,6 +1014,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const int b = r / wk.npairs, hp = r % wk.npairs;
                 const int64_t row = (int64_t)b * d.seqlen;
                 const int s_cut = (int)(128 * (fb - rb));
+                griddep_wait();  // the range states come from the kernel before this one
 #pragma unroll
                 for (int i = 0; i < NQ; ++i) hv[i] = 0.f;
                 for (int j = (int)(rb / wk.wt); j < i_work; ++j) {
@@ -1043,8 +1049,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         fence_async_shared();
         tc_fence_before();
         signal(&bar_st);
-        lg_tables(0);
-        build_lg(0);
 
         const int eh = cq >> 1, p0 = 32 * (cq & 1);  // epilogue: head and first p of this thread
         for (int t = 0;; ++t) {
@@ -1288,7 +1292,7 @@ cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const floa
 cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
                               const void* C, const float* D, const float* work_in, const float* init_states,
                               const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st,
-                              const float* work_local, const float* work_decay) {
+                              const float* work_local, const float* work_decay, bool after_segment_state) {
     CUtensorMap mx, mb, mc, my;
     cudaError_t e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
@@ -1296,22 +1300,36 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
     if ((e = bc_map(&mc, d, C, 128)) != cudaSuccess) return e;
     if ((e = x_map(&my, d, Y, 128)) != cudaSuccess) return e;
     const Work w = make_work(d, work_tiles);
-    const dim3 grid(w.nwork);
+    // Right after segment_state in the same stream, the scan is launched as its
+    // programmatic dependent: its CTAs start as segment_state's leave the SMs and
+    // wait for that grid only before reading the range states. Everything the
+    // scan reads before that wait was complete before segment_state started.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(w.nwork);
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_segment_state ? 1 : 0;
+    __nv_bfloat16* Yb = (__nv_bfloat16*)Y;
     if (d.dstate == 64) {
         auto k = fused_scan_kernel<64>;
-        const int smem = fused_smem_bytes<64>();
-        if ((e = set_smem_attr(k, smem, 32)) != cudaSuccess) return e;
-        k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx,
-                                             (__nv_bfloat16*)Y, final_states, work_local, work_decay);
+        cfg.dynamicSmemBytes = fused_smem_bytes<64>();
+        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 32)) != cudaSuccess) return e;
+        e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
+                               final_states, work_local, work_decay);
     } else if (d.dstate == 128) {
         auto k = fused_scan_kernel<128>;
-        const int smem = fused_smem_bytes<128>();
-        if ((e = set_smem_attr(k, smem, 33)) != cudaSuccess) return e;
-        k<<<grid, kFusedThreads, smem, st>>>(mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx,
-                                             (__nv_bfloat16*)Y, final_states, work_local, work_decay);
+        cfg.dynamicSmemBytes = fused_smem_bytes<128>();
+        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 33)) != cudaSuccess) return e;
+        e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
+                               final_states, work_local, work_decay);
     } else {
         return cudaErrorNotSupported;
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -58,7 +58,8 @@ cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const floa
 cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
                               const void* C, const float* D, const float* work_in, const float* init_states,
                               const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st,
-                              const float* work_local = nullptr, const float* work_decay = nullptr);
+                              const float* work_local = nullptr, const float* work_decay = nullptr,
+                              bool after_segment_state = false);
 
 // state-dimension slices (ssd_pad.cu)
 cudaError_t launch_pad_bc(const void* src, void* dst, int64_t rows, int N, int n0, int w, int Np, cudaStream_t st);

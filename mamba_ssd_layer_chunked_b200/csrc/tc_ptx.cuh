@@ -109,6 +109,15 @@ __device__ __forceinline__ void tma_store_wait_read0() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// programmatic dependent launch: let the next kernel of the stream start
+// (its CTAs run up to their griddep_wait), and wait for the previous kernel of
+// the stream to complete with its memory visible (a no-op when the kernel was
+// not launched as a dependent)
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // all bulk stores of this thread complete (their global writes performed)
 __device__ __forceinline__ void tma_store_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
