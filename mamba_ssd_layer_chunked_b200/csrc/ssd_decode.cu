@@ -13,7 +13,9 @@
 // One CTA per (batch row, head). Thread (r, q) owns the 4 consecutive columns
 // p = 4q .. 4q+3 of state rows n = r, r + R, r + 2R, ... (R row groups), so a
 // warp reads and writes contiguous float4s; the read-out C^T H is reduced over
-// the row groups in shared memory.
+// the row groups in shared memory. A thread's rows are loaded together before
+// they are updated (more bytes in flight), with streaming cache hints: each
+// state row is read and written once per step.
 
 #include "ssd_common.cuh"
 
@@ -71,19 +73,31 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(int nheads, in
     float* H = state + (int64_t)bh * dstate * headdim + 4 * q;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < R) {
-#pragma unroll 4
-        for (int n = r; n < dstate; n += R) {
-            const float bn = to_f32(Bb[n]), cn = to_f32(Cb[n]);
-            float4 hv = *reinterpret_cast<const float4*>(H + (int64_t)n * headdim);
-            hv.x = fmaf(a, hv.x, bn * xv.x);
-            hv.y = fmaf(a, hv.y, bn * xv.y);
-            hv.z = fmaf(a, hv.z, bn * xv.z);
-            hv.w = fmaf(a, hv.w, bn * xv.w);
-            *reinterpret_cast<float4*>(H + (int64_t)n * headdim) = hv;
-            acc.x = fmaf(cn, hv.x, acc.x);
-            acc.y = fmaf(cn, hv.y, acc.y);
-            acc.z = fmaf(cn, hv.z, acc.z);
-            acc.w = fmaf(cn, hv.w, acc.w);
+        constexpr int kBatch = 8;  // state rows of this thread in flight at once
+        for (int n0 = r; n0 < dstate; n0 += kBatch * R) {
+            float4 hv[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int n = n0 + j * R;
+                if (n < dstate) hv[j] = __ldcs(reinterpret_cast<const float4*>(H + (int64_t)n * headdim));
+            }
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int n = n0 + j * R;
+                if (n < dstate) {
+                    const float bn = to_f32(Bb[n]), cn = to_f32(Cb[n]);
+                    float4 h = hv[j];
+                    h.x = fmaf(a, h.x, bn * xv.x);
+                    h.y = fmaf(a, h.y, bn * xv.y);
+                    h.z = fmaf(a, h.z, bn * xv.z);
+                    h.w = fmaf(a, h.w, bn * xv.w);
+                    __stcs(reinterpret_cast<float4*>(H + (int64_t)n * headdim), h);
+                    acc.x = fmaf(cn, h.x, acc.x);
+                    acc.y = fmaf(cn, h.y, acc.y);
+                    acc.z = fmaf(cn, h.z, acc.z);
+                    acc.w = fmaf(cn, h.w, acc.w);
+                }
+            }
         }
         red[r * P4 + q] = acc;
     }
