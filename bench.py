@@ -696,6 +696,46 @@ def run_decode(args, w):
     return 0
 
 
+def run_discretize(args, w):
+    """--mode discretize: ssd_discretize over the workload's (b, T, H, P) (the step
+    before the scan: softplus step size, log a = delta A, X = delta x). Bytes per
+    step: x read and X written (P e each per token x head), dt read and log a
+    written (4 each). One JSON line, not the headline."""
+    import torch
+    import mamba_ssd_layer_chunked_b200 as ssd
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    b, T, H, P = w.batch, w.seqlen, w.nheads, w.headdim
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=dev).manual_seed(11)
+    dt = torch.randn(b, T, H, device=dev, generator=gen) - 3
+    A = -torch.rand(H, device=dev, generator=gen) * 16
+    bias = torch.randn(H, device=dev, generator=gen) * 0.1
+    x = torch.randn(b, T, H, P, device=dev, generator=gen).to(tdt)
+    X = torch.empty_like(x)
+    la = torch.empty(b, T, H, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        flush.zero_()  # inputs of one step fit in L2: flush between steps, timed separately below
+        ssd.discretize(dt, A, x, dt_bias=bias, out=(la, X))
+
+    t_all = _time_device(step, args.steps, args.warmup, stream)
+    t_flush = _time_device(lambda: flush.zero_(), args.steps, args.warmup, stream)
+    t = max(t_all - t_flush, 1e-9)
+    e = 2 if w.dtype == "bf16" else 4
+    byts = b * T * H * (2 * P * e + 8)
+    peaks = load_peaks()
+    print(json.dumps({"mode": "discretize", "metric": "discretisation tokens·heads/s", "workload": w.name,
+                      "value": b * T * H / t, "unit": "tokens·heads/s", "us_per_step": t * 1e6,
+                      "roofline": {"bound": "hbm", "achieved": byts / t / 1e9, "peak": peaks["hbm_gbs"],
+                                   "unit": "GB/s", "frac": byts / t / 1e9 / peaks["hbm_gbs"]},
+                      "l2": "flushed between steps (flush time subtracted)", "steps": args.steps,
+                      "warmup": args.warmup, "dtype": w.dtype}), flush=True)
+    return 0
+
+
 def run_sp(args, w):
     """--mode sp: the sequence-parallel forward (every batch row's tokens in R
     consecutive segments). Under torchrun (WORLD_SIZE > 1) it runs over NCCL,
@@ -793,9 +833,9 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--mode", choices=["scan", "sweep", "decode", "sp"], default="scan",
+    ap.add_argument("--mode", choices=["scan", "sweep", "decode", "sp", "discretize"], default="scan",
                     help="scan: the headline line (default); sweep: every workload; decode: the decode step; "
-                         "sp: the sequence-parallel forward")
+                         "sp: the sequence-parallel forward; discretize: the discretisation step")
     ap.add_argument("--decode-batch", type=int, default=64)
     ap.add_argument("--sp-ranks", type=int, default=4, help="ranks emulated on one GPU by --mode sp")
     args = ap.parse_args(argv)
@@ -808,6 +848,8 @@ def main(argv=None):
         return run_sweep(args)
     if args.mode == "decode":
         return run_decode(args, w)
+    if args.mode == "discretize":
+        return run_discretize(args, w)
     if args.mode == "sp":
         return run_sp(args, WORKLOADS["long16k_N128"] if args.workload == DEFAULT_WORKLOAD else w)
     return run_ours(args, w)

@@ -349,8 +349,9 @@ ssd_status ssd_fused_scan_chained(const ssd_problem* p, int64_t work_tiles, cons
  *   dt, log_a   [batch, seqlen, nheads]           fp32
  *   dt_bias, A  [nheads] fp32 (dt_bias may be NULL => 0; A <= 0 expected)
  *   x, X        [batch, seqlen, nheads, headdim]  p->dtype (X may alias x)
- * Only batch, seqlen, nheads, headdim (a multiple of 4) and dtype of p are
- * read. SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED before any launch. */
+ * Only batch, seqlen, nheads, headdim (a multiple of 8 for bf16, of 4 for
+ * fp32: 16-byte rows) and dtype of p are read; x and X 16-byte aligned.
+ * SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED before any launch. */
 ssd_status ssd_discretize(const ssd_problem* p, const float* dt, const float* dt_bias, const float* A,
                           const void* x, int zoh, float* log_a, void* X, void* stream);
 

@@ -359,13 +359,13 @@ ssd_status ssd_discretize(const ssd_problem* p, const float* dt, const float* dt
     if (!p) return SSD_ERR_INVALID_ARG;
     if (p->batch < 1 || p->seqlen < 1 || p->nheads < 1 || p->headdim < 1) return SSD_ERR_INVALID_ARG;
     if (p->dtype != SSD_DTYPE_F32 && p->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
-    if (p->headdim % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    // 16-byte rows: 8 bf16 or 4 fp32 elements per thread
+    if (p->headdim % (p->dtype == SSD_DTYPE_F32 ? 4 : 8) != 0) return SSD_ERR_UNSUPPORTED;
     if (p->batch * p->seqlen * p->nheads * p->headdim / 4 > ((int64_t)1 << 40)) return SSD_ERR_UNSUPPORTED;
     if (!dt || !A || !x || !log_a || !X) return SSD_ERR_INVALID_ARG;
-    const uintptr_t el = p->dtype == SSD_DTYPE_F32 ? 3u : 1u;
     if ((reinterpret_cast<uintptr_t>(dt) & 3u) || (reinterpret_cast<uintptr_t>(dt_bias) & 3u) ||
-        (reinterpret_cast<uintptr_t>(A) & 3u) || (reinterpret_cast<uintptr_t>(log_a) & 3u) ||
-        (reinterpret_cast<uintptr_t>(x) & el) || (reinterpret_cast<uintptr_t>(X) & el))
+        (reinterpret_cast<uintptr_t>(A) & 3u) || (reinterpret_cast<uintptr_t>(log_a) & 3u) || !aligned16(x) ||
+        !aligned16(X))
         return SSD_ERR_INVALID_ARG;
     ssd_status s = check_device();
     if (s != SSD_OK) return s;

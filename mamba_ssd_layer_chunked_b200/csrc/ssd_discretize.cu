@@ -22,28 +22,55 @@ constexpr int kDiscThreads = 256;
 
 __device__ __forceinline__ float softplus_f(float z) { return z > 20.f ? z : log1pf(expf(z)); }
 
-// one thread per 4 consecutive elements of a row (b, t, h) of P elements
+template <typename T>
+struct Vec16;  // 16 bytes of T: 8 bf16 or 4 fp32
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int kN = 8;
+};
+template <>
+struct Vec16<float> {
+    static constexpr int kN = 4;
+};
+
+// one thread per 16 bytes (8 bf16 or 4 fp32 elements) of a row (b, t, h) of P
+// elements; the row's delta is recomputed by each of its threads (cheaper than
+// sharing it: the kernel is bound by the bytes of x and X)
 template <typename T>
 __global__ void __launch_bounds__(kDiscThreads) discretize_kernel(int64_t rows, int nheads, int headdim,
                                                                   const float* __restrict__ dt,
                                                                   const float* __restrict__ dt_bias,
                                                                   const float* __restrict__ A, const T* __restrict__ x,
                                                                   int zoh, float* __restrict__ log_a, T* __restrict__ X) {
-    const int P4 = headdim / 4;
+    constexpr int V = Vec16<T>::kN;
+    const int PV = headdim / V;
     const int64_t i = (int64_t)blockIdx.x * kDiscThreads + threadIdx.x;
-    if (i >= rows * P4) return;
-    const int64_t r = i / P4;
-    const int q = (int)(i % P4);
+    if (i >= rows * PV) return;
+    const int64_t r = i / PV;
+    const int q = (int)(i % PV);
     const int h = (int)(r % nheads);
     const float a = A[h];
     const float delta = softplus_f(dt[r] + (dt_bias ? dt_bias[h] : 0.f));
     const float la = delta * a;
     if (q == 0) log_a[r] = la;
     const float s = zoh ? (a != 0.f ? expm1f(la) / a : delta) : delta;
-    const T* xr = x + r * headdim + 4 * q;
-    T* Xr = X + r * headdim + 4 * q;
+    const uint4 in = __ldcs(reinterpret_cast<const uint4*>(x + r * headdim) + q);
+    uint4 out;
+    if constexpr (V == 8) {
+        const __nv_bfloat162* xi = reinterpret_cast<const __nv_bfloat162*>(&in);
+        __nv_bfloat162* xo = reinterpret_cast<__nv_bfloat162*>(&out);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) Xr[e] = from_f32<T>(s * to_f32(xr[e]));
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(xi[e]);
+            xo[e] = __floats2bfloat162_rn(s * f.x, s * f.y);
+        }
+    } else {
+        const float* xi = reinterpret_cast<const float*>(&in);
+        float* xo = reinterpret_cast<float*>(&out);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) xo[e] = s * xi[e];
+    }
+    __stcs(reinterpret_cast<uint4*>(X + r * headdim) + q, out);
 }
 
 }  // namespace
@@ -51,7 +78,7 @@ __global__ void __launch_bounds__(kDiscThreads) discretize_kernel(int64_t rows, 
 cudaError_t launch_discretize(int64_t rows, int nheads, int headdim, ssd_dtype dt_x, const float* dt,
                               const float* dt_bias, const float* A, const void* x, int zoh, float* log_a, void* X,
                               cudaStream_t st) {
-    const int64_t n = rows * (headdim / 4);
+    const int64_t n = rows * (headdim / (dt_x == SSD_DTYPE_F32 ? 4 : 8));
     const unsigned grid = (unsigned)((n + kDiscThreads - 1) / kDiscThreads);
     if (dt_x == SSD_DTYPE_F32)
         discretize_kernel<float><<<grid, kDiscThreads, 0, st>>>(rows, nheads, headdim, dt, dt_bias, A,

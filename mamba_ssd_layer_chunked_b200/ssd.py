@@ -407,18 +407,22 @@ def decode_step(x: torch.Tensor, log_a: torch.Tensor, B: torch.Tensor, C: torch.
 
 
 def discretize(dt: torch.Tensor, A: torch.Tensor, x: torch.Tensor, dt_bias: Optional[torch.Tensor] = None,
-               zoh: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+               zoh: bool = False, stream=None, out=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """log_a = softplus(dt + dt_bias) * A and X = s * x (s = delta, or the
     zero-order-hold (exp(delta A) - 1) / A when zoh): the log_a and X inputs of
-    ssd_fwd. dt [b, T, H] fp32, A and dt_bias [H] fp32, x [b, T, H, P]."""
+    ssd_fwd. dt [b, T, H] fp32, A and dt_bias [H] fp32, x [b, T, H, P];
+    out = (log_a, X) to write into preallocated tensors."""
     if x.dim() != 4 or dt.shape != x.shape[:3] or A.shape != (x.shape[2],):
         raise ValueError("shapes: x [b,T,H,P], dt [b,T,H], A [H]")
     if dt.dtype != torch.float32 or A.dtype != torch.float32 or (dt_bias is not None and dt_bias.dtype != torch.float32):
         raise TypeError("dt, A and dt_bias must be float32")
     b, T, H, P = x.shape
     p = make_problem(b, T, H, P, 16, 1, 64, 1, x.dtype)  # dstate, ngroups, chunk are not read by this step
-    log_a = torch.empty(dt.shape, dtype=torch.float32, device=dt.device)
-    X = torch.empty_like(x)
+    if out is None:
+        log_a = torch.empty(dt.shape, dtype=torch.float32, device=dt.device)
+        X = torch.empty_like(x)
+    else:
+        log_a, X = out
     _check(lib().ssd_discretize(ctypes.byref(p), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(x), int(bool(zoh)),
                                 _ptr(log_a), _ptr(X), _stream(stream)), "ssd_discretize")
     return log_a, X

@@ -78,6 +78,9 @@ def test_host_checks():
     assert call(p, dt=FAKE + 2) == 1 and call(p, x=FAKE + 1) == 1
     q = ssd.Problem(1, 64, 2, 18, 16, 1, 64, 1, ssd.ssd.SSD_DTYPE_BF16, 0)
     assert call(q) == 2  # headdim not a multiple of 4
+    q = ssd.Problem(1, 64, 2, 20, 16, 1, 64, 1, ssd.ssd.SSD_DTYPE_BF16, 0)
+    assert call(q) == 2  # bf16 rows of 40 bytes: not whole 16-byte groups
+    assert call(p, x=FAKE + 8) == 1 and call(p, X=FAKE + 8) == 1  # x, X 16-byte aligned
     assert lib.ssd_discretize(None, FAKE, None, FAKE, FAKE, 0, FAKE, FAKE, None) == 1
 
 
