@@ -253,7 +253,10 @@ int64_t ssd_fused_work_count(const ssd_problem* p, int64_t work_tiles);
  *   work_local[i, j]  = sum_{l in [st, s1)} (prod_{k=l+1..s1-1} a_k) B_l x_l^T
  *   work_decay[i, j]  = prod_{k in [st, s1)} a_k        (head 2 hp + j)
  * (wq-win section 3, "local_end_state" and "block_decay", for a block that is
- * a range's piece). Entries of ranges that end at a row end are not written. */
+ * a range's piece). Terms that reach s1 through a product of a below e^-40 for
+ * both heads of the pair are left out (below the fp32 rounding of the rest),
+ * and work_decay is then 0. Entries of ranges that end at a row end are not
+ * written. */
 ssd_status ssd_segment_state(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a,
                              const void* B, const int32_t* seq_idx, float* work_local, float* work_decay,
                              void* stream);

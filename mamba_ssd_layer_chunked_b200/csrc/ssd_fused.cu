@@ -92,6 +92,7 @@ __device__ __forceinline__ void row_piece(const Work& w, int seqlen, int64_t fb,
 // ===========================================================================
 // segment_state
 // ===========================================================================
+constexpr float kSegCutLog = -40.f;           // walk cut: natural log of the decay product
 constexpr int kSegScale = 256;                 // the warps that scale X and own the accumulator lanes
 constexpr int kSegThreads = kSegScale + 32;    // + one warp that issues the MMAs
 
@@ -264,8 +265,10 @@ __global__ void __launch_bounds__(kSegThreads, 1)
             if (rr == 0) tail_s[hh] = tail;
             named_bar_sync(kScaleBar, kSegScale);
             if (tid == 0) mbar_arrive(&bar_scaled[sg]);  // the MMA warp may multiply tile it
-            // everything further back decays below fp32 range for both heads
-            if (tail_s[0] < -104.f && tail_s[1] < -104.f && i > 0) {
+            // the rest of the piece reaches the cut through a decay product below
+            // e^kSegCutLog for both heads: its terms are below 1e-17 of the partial
+            // state they come from, under the fp32 rounding of the kept sum
+            if (tail_s[0] < kSegCutLog && tail_s[1] < kSegCutLog && i > 0) {
                 cut = true;
                 break;
             }
