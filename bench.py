@@ -450,9 +450,9 @@ def run_ours(args, w):
     else:
         pk = ssd.problem_from(X, B, w.chunk, inputs["nseq"], "tcgen05" if fam == "tcgen05" else "simt")
         pr = ctypes.byref(pk)
-        nc = T // w.chunk
-        cs = wsp[: b * T * H * 4].view(torch.float32)
-        off = (b * T * H * 4 + 255) // 256 * 256
+        nc = -(-T // w.chunk)
+        cs = wsp[: b * nc * w.chunk * H * 4].view(torch.float32)
+        off = (b * nc * w.chunk * H * 4 + 255) // 256 * 256
         states = wsp[off: off + b * nc * H * N * P * 4].view(torch.float32)
         names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
         launches = [

@@ -118,11 +118,13 @@ ssd_status ssd_check_problem(const ssd_problem* p);
 /* 1 if `path` (SIMT, TCGEN05 or FUSED) can run problem p on the current device. */
 int ssd_path_supported(const ssd_problem* p, ssd_path path);
 
-/* Bytes of workspace ssd_fwd needs, or (size_t)-1 if p is invalid: the larger
- * of the chunked paths' need (the chunk cumulative sums, batch*seqlen*nheads
- * fp32, and one state per chunk, batch*nchunks*nheads*dstate*headdim fp32) and
- * the fused path's need (two states and two decays per work range, see
- * ssd_fused_work_tiles), each part 256-byte aligned. */
+/* Bytes of workspace ssd_fwd needs for p, or (size_t)-1 if p is invalid: for
+ * the family ssd_fwd runs (p->path, or for AUTO the fused family where it
+ * applies, else the chunked ones), the chunked paths' need (the chunk
+ * cumulative sums, batch*nchunks*chunk*nheads fp32, and one state per chunk,
+ * batch*nchunks*nheads*dstate*headdim fp32) or the fused path's (two states and
+ * two decays per work range, see ssd_fused_work_tiles, plus the padded slices
+ * when dstate is not 64 or 128), each part 256-byte aligned. */
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p);
 
 /*

@@ -230,12 +230,8 @@ size_t ssd_states_bytes(const ssd_problem* p) {
 
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
     if (check_dims(p) != SSD_OK) return (size_t)-1;
-    size_t need = chunked_workspace_bytes(p);
-    if (ssd::fused_fwd_supported(p)) {
-        const size_t f = fused_layout(p).total;
-        if (f > need) need = f;
-    }
-    return need;
+    // the family ssd_fwd runs for p (the same host-side decision)
+    return fwd_family(p) == SSD_PATH_FUSED ? fused_layout(p).total : chunked_workspace_bytes(p);
 }
 
 int64_t ssd_fused_work_tiles(const ssd_problem* p) {

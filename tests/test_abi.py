@@ -54,7 +54,8 @@ def test_workspace_bytes_formula():
     nwork = -(-total // wt)
     assert ssd.fused_work_count(p, wt) == nwork
     fused = 2 * align(nwork * 2 * 128 * 64 * 4) + align(nwork * 2 * 4)
-    assert ssd.workspace_bytes(p) == max(align(cs) + align(st), fused)
+    assert ssd.workspace_bytes(p) == fused  # AUTO runs the fused family for this problem
+    assert ssd.workspace_bytes(prob(path=1)) == align(cs) + align(st)  # the SIMT family: the chunked need
     assert ssd.states_bytes(p) == st
     # outside the fused domain (fp32) only the chunked need counts
     q = prob(dtype=ssd.ssd.SSD_DTYPE_F32)

@@ -29,8 +29,9 @@ def _noalloc():
 
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch():
     ssd, f = _noalloc()
-    # the 2.7B-shaped layer needs ~173 MB of scratch, more than the 64 MiB array
-    p = ssd.make_problem(4, 4096, 80, 64, 128, 1, 256, 1, torch.bfloat16)
+    # the 2.7B-shaped layer in fp32 (the SIMT family) needs ~173 MB of scratch
+    # (one state per chunk), more than the 64 MiB array: rejected before any launch
+    p = ssd.make_problem(4, 4096, 80, 64, 128, 1, 256, 1, torch.float32)
     assert ssd.workspace_bytes(p) > 64 << 20
     assert f(ctypes.byref(p), *([FAKE] * 4), None, None, None, FAKE, None, None) == SSD_ERR_WORKSPACE
 
