@@ -277,6 +277,19 @@ def test_single_chunk(path):
 
 
 @pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("T, dtype, P, N, Q", [(1, "bf16", 64, 128, 256), (7, "f32", 32, 48, 64),
+                                              (127, "bf16", 64, 64, 128), (129, "bf16", 64, 128, 128)])
+def test_single_token_and_short_rows(path, T, dtype, P, N, Q):
+    # one token, and rows shorter than (or one token past) a chunk and a 128-token tile
+    d = make_custom(2, T, 4, P, N, dtype=dtype, seed=14 + T, has_D="normal", has_init=True)
+    _skip_unsupported(d, dtype, Q, path)
+    Y, F = run_gpu(d, dtype, Q, path)
+    Yr, Fr = run_oracle(d)
+    assert_close(Y, Yr, TAU[dtype], "Y")
+    assert_close(F, Fr, TAU[dtype], "final")
+
+
+@pytest.mark.parametrize("path", PATHS)
 def test_absent_sequence_ids_keep_initial_state(path):
     d = make_custom(2, 512, 2, 64, 64, dtype="bf16", seed=12, has_init=True, lengths=[[300, 212], [512]], nseq=4)
     _skip_unsupported(d, "bf16", 128, path)
