@@ -143,16 +143,16 @@ FusedLayout fused_layout(const ssd_problem* p) {
     if (!f.direct) {
         l.bc = align256((size_t)p->batch * p->seqlen * p->ngroups * f.np * 2);
         l.st = align256((size_t)p->batch * p->nseq * p->nheads * f.np * p->headdim * sizeof(float));
-        if (f.pieces > 1) l.y = align256((size_t)p->batch * p->seqlen * p->nheads * p->headdim * 2);
     }
     l.total = l.work + 2 * l.bc + 2 * l.st + l.y;
     return l;
 }
 
 // The three fused launches on dims d (dstate 64 or 128), workspace ws.
+// Yacc: Y of the state slices before this one, added in the scan's epilogue.
 cudaError_t run_fused(const ssd::Dims& d, const void* X, const float* log_a, const void* B, const void* C,
                       const float* D, const float* init_states, const int32_t* seq_idx, void* Y, float* final_states,
-                      void* ws, cudaStream_t st) {
+                      void* ws, cudaStream_t st, const void* Yacc = nullptr) {
     const int64_t wt = ssd::fused_default_work_tiles(d);
     const size_t nwork = (size_t)ssd::fused_work_count(d, wt);
     const size_t stb = nwork * 2 * d.dstate * d.headdim * sizeof(float);
@@ -165,7 +165,7 @@ cudaError_t run_fused(const ssd::Dims& d, const void* X, const float* log_a, con
     if (cuts && (e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st)) != cudaSuccess)
         return e;
     return ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, nullptr, init_states, seq_idx, Y, final_states, st,
-                                  cuts ? work_local : nullptr, cuts ? work_decay : nullptr, cuts);
+                                  cuts ? work_local : nullptr, cuts ? work_decay : nullptr, cuts, Yacc);
 }
 
 ssd_status check_common(const ssd_problem* p, const int32_t* seq_idx) {
@@ -466,7 +466,6 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
         void* Cp = w + l.work + l.bc;
         float* init_p = reinterpret_cast<float*>(w + l.work + 2 * l.bc);
         float* fin_p = reinterpret_cast<float*>(w + l.work + 2 * l.bc + l.st);
-        void* Yk = w + l.work + 2 * l.bc + 2 * l.st;
         ssd::Dims dp = d;
         dp.dstate = f.np;
         const int64_t rows = (int64_t)d.batch * d.seqlen * d.ngroups;
@@ -480,15 +479,14 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
                 (e = ssd::launch_pad_states(init_states, init_p, S, d.dstate, n0, wd, f.np, d.headdim, st)) !=
                     cudaSuccess)
                 break;
-            void* Yo = k == 0 ? Y : Yk;
-            if ((e = run_fused(dp, X, log_a, Bp, Cp, k == 0 ? D : nullptr, init_states ? init_p : nullptr, seq_idx, Yo,
-                               final_states ? fin_p : nullptr, w, st)) != cudaSuccess)
+            // slices after the first add their Y to the one in place (read in the epilogue)
+            if ((e = run_fused(dp, X, log_a, Bp, Cp, k == 0 ? D : nullptr, init_states ? init_p : nullptr, seq_idx, Y,
+                               final_states ? fin_p : nullptr, w, st, k > 0 ? Y : nullptr)) != cudaSuccess)
                 break;
             if (final_states &&
                 (e = ssd::launch_unpad_states(fin_p, final_states, S, d.dstate, n0, wd, f.np, d.headdim, st)) !=
                     cudaSuccess)
                 break;
-            if (k > 0) e = ssd::launch_add_bf16(Y, Yk, (int64_t)d.batch * d.seqlen * d.nheads * d.headdim, st);
         }
         return cuda_status(e);
     }

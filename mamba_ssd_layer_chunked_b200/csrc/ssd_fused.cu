@@ -461,7 +461,10 @@ static_assert(sizeof(CsBuf) % 16 == 0, "CsBuf must keep 16-byte alignment in an 
 // are ready at different times.
 // Tensor memory: G, then L o G in place [0,128); Y_diag [128,256);
 // Y_off [256,384); the carried state H [384,512) (rows (head, p), N columns).
-template <int N>
+// kAcc: a later state slice, whose epilogue adds its Y to the Y already there
+// (each thread reads the elements it then writes); a separate instantiation so
+// that the common case keeps its epilogue unchanged.
+template <int N, bool kAcc>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, Dims d,
@@ -1080,9 +1083,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             tc_fence_after();
             {
                 const __nv_bfloat162 wx2 = __floats2bfloat162_rn(wx, wx);
-                __nv_bfloat16* yrow = Y + ((rowt + cur.ts + k) * d.nheads + 2 * cur.hp + eh) * (int64_t)kP + p0;
+                const int64_t yoff = ((rowt + cur.ts + k) * d.nheads + 2 * cur.hp + eh) * (int64_t)kP + p0;
+                __nv_bfloat16* yrow = Y + yoff;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
+                    // a later state slice: the Y this thread's outputs add to
+                    uint4 ya[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+                    if (kAcc && k < cur.v) {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) ya[c] = *reinterpret_cast<const uint4*>(Y + yoff + 8 * (2 * hf + c));
+                    }
                     uint32_t yd[16], yo[16];
                     tmem_ld16_async(tm_yd + lane_off + 32 * cq + 16 * hf, yd);
                     tmem_ld16_async(tm_yo + lane_off + 32 * cq + 16 * hf, yo);
@@ -1098,9 +1108,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         for (int i = 0; i < 4; ++i) {
                             const __nv_bfloat162 xb = *reinterpret_cast<const __nv_bfloat162*>(&xu[i]);
                             const int e0 = 8 * c + 2 * i;  // of this half; D x is in Y_diag (L o G diagonal)
-                            const float2 yy = __ffma2_rn(make_float2(rs, rs),
-                                                         make_float2(__uint_as_float(yo[e0]), __uint_as_float(yo[e0 + 1])),
-                                                         make_float2(__uint_as_float(yd[e0]), __uint_as_float(yd[e0 + 1])));
+                            float2 yy = __ffma2_rn(make_float2(rs, rs),
+                                                   make_float2(__uint_as_float(yo[e0]), __uint_as_float(yo[e0 + 1])),
+                                                   make_float2(__uint_as_float(yd[e0]), __uint_as_float(yd[e0 + 1])));
+                            if (kAcc) {
+                                const float2 pv = __bfloat1622float2(
+                                    *reinterpret_cast<const __nv_bfloat162*>(reinterpret_cast<const uint32_t*>(&ya[c]) + i));
+                                yy.x += pv.x;
+                                yy.y += pv.y;
+                            }
                             out[i] = pack_bf16(yy.x, yy.y);
                             const __nv_bfloat162 xs = __hmul2(xb, wx2);
                             xu[i] = *reinterpret_cast<const uint32_t*>(&xs);
@@ -1295,7 +1311,9 @@ cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const floa
 cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, const float* log_a, const void* B,
                               const void* C, const float* D, const float* work_in, const float* init_states,
                               const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st,
-                              const float* work_local, const float* work_decay, bool after_segment_state) {
+                              const float* work_local, const float* work_decay, bool after_segment_state,
+                              const void* Yacc) {
+    if (Yacc && Yacc != Y) return cudaErrorInvalidValue;  // the slices accumulate in place
     CUtensorMap mx, mb, mc, my;
     cudaError_t e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
@@ -1318,15 +1336,15 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
     cfg.numAttrs = after_segment_state ? 1 : 0;
     __nv_bfloat16* Yb = (__nv_bfloat16*)Y;
     if (d.dstate == 64) {
-        auto k = fused_scan_kernel<64>;
+        auto k = Yacc ? fused_scan_kernel<64, true> : fused_scan_kernel<64, false>;
         cfg.dynamicSmemBytes = fused_smem_bytes<64>();
-        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 32)) != cudaSuccess) return e;
+        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, Yacc ? 34 : 32)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
                                final_states, work_local, work_decay);
     } else if (d.dstate == 128) {
-        auto k = fused_scan_kernel<128>;
+        auto k = Yacc ? fused_scan_kernel<128, true> : fused_scan_kernel<128, false>;
         cfg.dynamicSmemBytes = fused_smem_bytes<128>();
-        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 33)) != cudaSuccess) return e;
+        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, Yacc ? 35 : 33)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
                                final_states, work_local, work_decay);
     } else {

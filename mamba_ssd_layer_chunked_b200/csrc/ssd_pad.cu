@@ -6,8 +6,8 @@
 // 2.1, read row by row). So a problem with dstate N is the sum over slices of n
 // of problems on those slices (D counted once), and a slice padded with zero
 // columns of B and C has zero extra state rows and unchanged outputs. These
-// kernels copy a slice of B / C / states into a padded buffer, copy states
-// back, and add a slice's Y into the output.
+// kernels copy a slice of B / C / states into a padded buffer and copy states
+// back; the scan of a later slice adds its Y to the output in its epilogue.
 
 #include "ssd_common.cuh"
 
@@ -52,16 +52,6 @@ __global__ void unpad_states_kernel(const float* __restrict__ src, float* __rest
     dst[(s * N + n0 + j) * P + p] = src[(s * Np + j) * P + p];
 }
 
-// Y += Yk, bf16 pairs, in fp32 then rounded to nearest even
-__global__ void add_bf16_kernel(__nv_bfloat16* __restrict__ y, const __nv_bfloat16* __restrict__ yk, int64_t n2) {
-    const int64_t i = (int64_t)blockIdx.x * kPadThreads + threadIdx.x;
-    if (i >= n2) return;
-    __nv_bfloat162* a = reinterpret_cast<__nv_bfloat162*>(y) + i;
-    const float2 u = __bfloat1622float2(*a);
-    const float2 v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(yk)[i]);
-    *a = __floats2bfloat162_rn(u.x + v.x, u.y + v.y);
-}
-
 unsigned blocks_for(int64_t n) { return (unsigned)((n + kPadThreads - 1) / kPadThreads); }
 
 }  // namespace
@@ -81,11 +71,6 @@ cudaError_t launch_pad_states(const float* src, float* dst, int64_t S, int N, in
 cudaError_t launch_unpad_states(const float* src, float* dst, int64_t S, int N, int n0, int w, int Np, int P,
                                 cudaStream_t st) {
     unpad_states_kernel<<<blocks_for(S * (int64_t)w * P), kPadThreads, 0, st>>>(src, dst, S, N, n0, w, Np, P);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_add_bf16(void* y, const void* yk, int64_t n, cudaStream_t st) {
-    add_bf16_kernel<<<blocks_for(n / 2), kPadThreads, 0, st>>>((__nv_bfloat16*)y, (const __nv_bfloat16*)yk, n / 2);
     return cudaGetLastError();
 }
 

@@ -59,7 +59,7 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
                               const void* C, const float* D, const float* work_in, const float* init_states,
                               const int32_t* seq_idx, void* Y, float* final_states, cudaStream_t st,
                               const float* work_local = nullptr, const float* work_decay = nullptr,
-                              bool after_segment_state = false);
+                              bool after_segment_state = false, const void* Yacc = nullptr);
 
 // state-dimension slices (ssd_pad.cu)
 cudaError_t launch_pad_bc(const void* src, void* dst, int64_t rows, int N, int n0, int w, int Np, cudaStream_t st);
@@ -67,6 +67,5 @@ cudaError_t launch_pad_states(const float* src, float* dst, int64_t S, int N, in
                               cudaStream_t st);
 cudaError_t launch_unpad_states(const float* src, float* dst, int64_t S, int N, int n0, int w, int Np, int P,
                                 cudaStream_t st);
-cudaError_t launch_add_bf16(void* y, const void* yk, int64_t n, cudaStream_t st);
 
 }  // namespace ssd
