@@ -308,10 +308,20 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
  *         without seq_idx)
  *   g_loc, g_dec, g_ids: the R ranks' loc, dec, ids stacked in rank order
  *   init_states, init_local, final_states [batch, nseq, nheads, dstate, headdim]
- * ssd_sp_summary covers the FUSED family's domain (SSD_ERR_UNSUPPORTED
- * elsewhere); dec is 0 where the product is below fp32 range. */
+ * ssd_sp_summary runs segment_state (whole-row ranges) where those kernels
+ * cover p (bf16, headdim 64, dstate 64 or 128, an even number of heads per
+ * group; path AUTO or FUSED): no workspace, and dec is 0 where the product is
+ * below e^-40 (the start state's share of E is then below the rounding of
+ * loc). Elsewhere it runs the chunked steps (chunk length p->chunk) from zero
+ * initial states: loc is the last sequence's final state, dec the exp of the
+ * fp32 sum of log a over its piece; that needs a device workspace of
+ * ssd_sp_summary_workspace_bytes(p) bytes (16-byte aligned, contents
+ * overwritten; SSD_ERR_WORKSPACE when missing or smaller). The caller owns
+ * every buffer; nothing is allocated. */
+size_t ssd_sp_summary_workspace_bytes(const ssd_problem* p);  /* (size_t)-1 on invalid p */
 ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_a, const void* B,
-                          const int32_t* seq_idx, float* loc, float* dec, int32_t* ids, void* stream);
+                          const int32_t* seq_idx, float* loc, float* dec, int32_t* ids, void* workspace,
+                          size_t workspace_bytes, void* stream);
 
 /* init_local[b, s] = the state entering this rank's first token when that
  * token continues sequence s from the previous rank, else init_states[b, s]

@@ -112,6 +112,19 @@ ssd_path fwd_family(const ssd_problem* p) {
 
 size_t chunked_workspace_bytes(const ssd_problem* p) { return align256(cs_bytes(p)) + align256(states_bytes(p)); }
 
+// The sequence-parallel summary runs segment_state where the fused family's
+// kernels cover p (and the path allows it), else the chunked steps, which need
+// a workspace: their cumsum and chunk states, and final states from zero.
+bool sp_fused(const ssd_problem* p) {
+    return (p->path == SSD_PATH_AUTO || p->path == SSD_PATH_FUSED) && ssd::fused_supported(p);
+}
+
+size_t sp_workspace_bytes(const ssd_problem* p) {
+    if (sp_fused(p)) return 0;
+    return chunked_workspace_bytes(p) +
+           align256((size_t)p->batch * p->nseq * p->nheads * p->dstate * p->headdim * sizeof(float));
+}
+
 // The fused family on the dstate it was given directly (64 or 128), or on
 // slices of at most 128 state rows padded to Np (64 when dstate <= 64, else
 // 128): the work-range states of the padded problem, the padded B and C,
@@ -311,17 +324,39 @@ ssd_status ssd_fused_scan_chained(const ssd_problem* p, int64_t work_tiles, cons
                                               final_states, (cudaStream_t)stream, work_local, work_decay));
 }
 
+size_t ssd_sp_summary_workspace_bytes(const ssd_problem* p) {
+    if (check_dims(p) != SSD_OK) return (size_t)-1;
+    return sp_workspace_bytes(p);
+}
+
 ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_a, const void* B,
-                          const int32_t* seq_idx, float* loc, float* dec, int32_t* ids, void* stream) {
+                          const int32_t* seq_idx, float* loc, float* dec, int32_t* ids, void* workspace,
+                          size_t workspace_bytes, void* stream) {
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !loc || !dec || !ids) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, seq_idx, loc, dec, ids)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, log_a, B, seq_idx, loc, dec, ids, workspace)) return SSD_ERR_INVALID_ARG;
+    const size_t need = sp_workspace_bytes(p);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
+    if ((s = check_runnable(p)) != SSD_OK) return s;
     const ssd::Dims d = make_dims(p);
-    if ((s = check_device()) != SSD_OK) return s;
-    if (!ssd::fused_supported(p)) return SSD_ERR_UNSUPPORTED;
-    const int64_t nt = ((int64_t)p->seqlen + 127) / 128;  // one work range per (batch row, head pair)
-    return cuda_status(ssd::launch_segment_state(d, nt, X, log_a, B, seq_idx, loc, dec, (cudaStream_t)stream, ids));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (sp_fused(p)) {
+        const int64_t nt = ((int64_t)p->seqlen + 127) / 128;  // one work range per (batch row, head pair)
+        return cuda_status(ssd::launch_segment_state(d, nt, X, log_a, B, seq_idx, loc, dec, st, ids));
+    }
+    char* w = static_cast<char*>(workspace);
+    float* cs = reinterpret_cast<float*>(w);
+    float* states = reinterpret_cast<float*>(w + align256(cs_bytes(p)));
+    float* finals = reinterpret_cast<float*>(w + chunked_workspace_bytes(p));
+    cudaError_t e = ssd::launch_chunk_cumsum(d, log_a, cs, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = use_tc(p) ? ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, finals, st)
+                  : ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, finals, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    if ((e = ssd::launch_state_passing(d, cs, states, states, nullptr, seq_idx, finals, st)) != cudaSuccess)
+        return cuda_status(e);
+    return cuda_status(ssd::launch_sp_finish(d, log_a, seq_idx, finals, loc, dec, ids, st));
 }
 
 ssd_status ssd_sp_combine(const ssd_problem* p, int nranks, int rank, const float* g_loc, const float* g_dec,

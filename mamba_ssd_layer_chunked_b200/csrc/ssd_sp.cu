@@ -9,7 +9,9 @@
 // local end state and block decay, here for a whole segment; the pages'
 // sequence-parallel variant exchanges exactly these per-segment states). Each
 // rank computes (loc, dec) and its first and last sequence ids (segment_state
-// in whole-row mode), the ranks all-gather them, and each rank chains the
+// in whole-row mode where the fused family's kernels cover the problem, else
+// the chunked steps from zero initial states and sp_finish), the ranks
+// all-gather them, and each rank chains the
 // segments before its own (sp_combine) to get the state entering its first
 // token, which then runs the ordinary forward pass as that sequence's initial
 // state. Final states: the rank holding a sequence's last token owns it
@@ -89,6 +91,48 @@ __global__ void __launch_bounds__(kSpThreads) sp_own_finals_kernel(Dims d, int n
     if (owner != rank) final_states[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// The summary from the chunked steps' final states (zero initial states), one
+// block per (b, h): loc = the final state of the segment's last sequence (its
+// piece here started from zero), dec = exp of the sum of log a over that
+// piece, ids = the first and last sequence ids of the row (ids ascend along a
+// row, so the piece starts at the first token carrying the last id).
+__global__ void __launch_bounds__(kSpThreads) sp_finish_kernel(Dims d, const float* __restrict__ log_a,
+                                                               const int32_t* __restrict__ seq_idx,
+                                                               const float* __restrict__ finals,
+                                                               float* __restrict__ loc, float* __restrict__ dec,
+                                                               int32_t* __restrict__ ids) {
+    __shared__ float part[kSpThreads / 32];
+    const int64_t bh = blockIdx.x;
+    const int b = (int)(bh / d.nheads), h = (int)(bh % d.nheads);
+    const int64_t row = (int64_t)b * d.seqlen;
+    const int first = seq_at(seq_idx, row, 0, d.nseq), last = seq_at(seq_idx, row, d.seqlen - 1, d.nseq);
+    int lo = 0, hi = d.seqlen - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (seq_at(seq_idx, row, mid, d.nseq) < last) lo = mid + 1;
+        else hi = mid;
+    }
+    float acc = 0.f;
+    for (int t = lo + (int)threadIdx.x; t < d.seqlen; t += kSpThreads) acc += log_a[(row + t) * d.nheads + h];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int w = 0; w < kSpThreads / 32; ++w) s += part[w];
+        dec[bh] = expf(s);
+        if (h == 0) {
+            ids[2 * b] = first;
+            ids[2 * b + 1] = last;
+        }
+    }
+    const int NP = d.dstate * d.headdim;
+    const float* src = finals + seqst_off(d, b, last, h);
+    float* dst = loc + bh * NP;
+    for (int i = (int)threadIdx.x; i < NP; i += kSpThreads) dst[i] = src[i];
+}
+
 unsigned blocks_for(int64_t n) { return (unsigned)((n + kSpThreads - 1) / kSpThreads); }
 
 }  // namespace
@@ -99,6 +143,14 @@ cudaError_t launch_sp_combine(const Dims& d, int nranks, int rank, const float* 
     if (n == 0) return cudaSuccess;
     sp_combine_kernel<<<blocks_for(n), kSpThreads, 0, st>>>(d, nranks, rank, (const float4*)g_loc, g_dec, g_ids,
                                                            (const float4*)init_states, (float4*)init_local);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sp_finish(const Dims& d, const float* log_a, const int32_t* seq_idx, const float* finals,
+                             float* loc, float* dec, int32_t* ids, cudaStream_t st) {
+    const int64_t n = (int64_t)d.batch * d.nheads;
+    if (n == 0) return cudaSuccess;
+    sp_finish_kernel<<<(unsigned)n, kSpThreads, 0, st>>>(d, log_a, seq_idx, finals, loc, dec, ids);
     return cudaGetLastError();
 }
 

@@ -50,6 +50,10 @@ cudaError_t launch_sp_combine(const Dims& d, int nranks, int rank, const float* 
                               const int32_t* g_ids, const float* init_states, float* init_local, cudaStream_t st);
 cudaError_t launch_sp_own_finals(const Dims& d, int nranks, int rank, const int32_t* g_ids, float* final_states,
                                  cudaStream_t st);
+// loc, dec, ids of a segment from the final states of its sequences from zero
+// initial states (the chunked steps' output)
+cudaError_t launch_sp_finish(const Dims& d, const float* log_a, const int32_t* seq_idx, const float* finals,
+                             float* loc, float* dec, int32_t* ids, cudaStream_t st);
 cudaError_t launch_segment_passing(const Dims& d, int64_t work_tiles, const float* work_local, const float* work_decay,
                                    const float* init_states, const int32_t* seq_idx, float* work_in, cudaStream_t st);
 // work_in (the output of segment_passing) or, when it is null, work_local and

@@ -69,7 +69,8 @@ def _declare(lib):
         "ssd_fused_scan_chained": ([P, ctypes.c_int64] + [vp] * 12, ctypes.c_int),
         "ssd_decode_step": ([P] + [vp] * 8, ctypes.c_int),
         "ssd_discretize": ([P, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp], ctypes.c_int),
-        "ssd_sp_summary": ([P] + [vp] * 8, ctypes.c_int),
+        "ssd_sp_summary": ([P] + [vp] * 8 + [ctypes.c_size_t, vp], ctypes.c_int),
+        "ssd_sp_summary_workspace_bytes": ([P], ctypes.c_size_t),
         "ssd_sp_combine": ([P, ctypes.c_int, ctypes.c_int] + [vp] * 6, ctypes.c_int),
         "ssd_sp_own_finals": ([P, ctypes.c_int, ctypes.c_int, vp, vp, vp], ctypes.c_int),
     }
@@ -335,18 +336,29 @@ def fused_scan(X, log_a, B, C, work_tiles, work_incoming=None, D=None, init_stat
     return Y
 
 
-def sp_summary(X, log_a, B, seq_idx=None, nseq=1, chunk=64, stream=None):
+def sp_summary_workspace_bytes(p: Problem) -> int:
+    n = lib().ssd_sp_summary_workspace_bytes(ctypes.byref(p))
+    if n == ctypes.c_size_t(-1).value:
+        _check(lib().ssd_check_problem(ctypes.byref(p)) or SSD_ERR_INVALID_ARG, "ssd_sp_summary_workspace_bytes")
+    return int(n)
+
+
+def sp_summary(X, log_a, B, seq_idx=None, nseq=1, chunk=64, path="auto", stream=None):
     """This rank's segment summary: (loc [b, H, N, P] fp32, dec [b, H] fp32,
     ids [b, 2] int32), with E = dec * H_start + loc over the segment's last
-    sequence piece and ids its first and last sequence ids."""
-    p = _fused_problem(X, B, nseq, chunk)
+    sequence piece and ids its first and last sequence ids. The chunk length
+    is used only where the summary runs the chunked steps (outside the fused
+    family's domain)."""
+    p = problem_from(X, B, chunk, nseq, path)
     b, _, H, P = X.shape
     N = B.shape[3]
     loc = torch.empty((b, H, N, P), dtype=torch.float32, device=X.device)
     dec = torch.empty((b, H), dtype=torch.float32, device=X.device)
     ids = torch.empty((b, 2), dtype=torch.int32, device=X.device)
+    need = sp_summary_workspace_bytes(p)
+    ws = torch.empty(need, dtype=torch.uint8, device=X.device) if need else None
     _check(lib().ssd_sp_summary(ctypes.byref(p), _ptr(X), _ptr(log_a), _ptr(B), _ptr(seq_idx), _ptr(loc), _ptr(dec),
-                                _ptr(ids), _stream(stream)), "ssd_sp_summary")
+                                _ptr(ids), _ptr(ws), need, _stream(stream)), "ssd_sp_summary")
     return loc, dec, ids
 
 

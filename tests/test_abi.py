@@ -125,6 +125,23 @@ def test_nseq_needs_seq_idx():
     assert _fwd(prob(nseq=3)) == INVALID
 
 
+def test_sp_summary_workspace_formula():
+    lib = ssd.lib()
+    align = lambda x: (x + 255) // 256 * 256
+    size = lambda q: lib.ssd_sp_summary_workspace_bytes(ctypes.byref(q))
+    # segment_state covers bf16, P 64, N 64 or 128: no workspace
+    assert size(prob()) == 0 and size(prob(dstate=64)) == 0
+    # the chunked steps: cumsum, chunk states, final states from zero
+    for q, (b, T, H, P, N, Q, S) in ((prob(dtype=ssd.ssd.SSD_DTYPE_F32, headdim=16, dstate=16, chunk=64),
+                                      (2, 512, 4, 16, 16, 64, 1)),
+                                     (prob(dstate=256), (2, 512, 4, 64, 256, 256, 1)),
+                                     (prob(seqlen=500, nseq=3, path=1), (2, 500, 4, 64, 128, 256, 3))):
+        nc = -(-T // Q)
+        want = align(b * nc * Q * H * 4) + align(b * nc * H * N * P * 4) + align(b * S * H * N * P * 4)
+        assert size(q) == want
+    assert size(prob(batch=0)) == ctypes.c_size_t(-1).value
+
+
 def test_workspace_checks():
     p = prob()
     need = ssd.workspace_bytes(p)
@@ -172,11 +189,17 @@ def test_sequence_parallel_entry_points_validate_on_host():
     lib = ssd.lib()
     p = prob()
     # summary: every pointer is required, 16-byte alignment
-    assert lib.ssd_sp_summary(ctypes.byref(p), None, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == INVALID
-    assert lib.ssd_sp_summary(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None) == INVALID
-    assert lib.ssd_sp_summary(ctypes.byref(p), FAKE + 8, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == INVALID
-    assert lib.ssd_sp_summary(ctypes.byref(prob(nseq=2)), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE,
-                              None) == INVALID  # nseq > 1 needs seq_idx
+    summ = lambda q, *a: lib.ssd_sp_summary(ctypes.byref(q), *a)
+    assert summ(p, None, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, 0, None) == INVALID
+    assert summ(p, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None, 0, None) == INVALID
+    assert summ(p, FAKE + 8, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, 0, None) == INVALID
+    assert summ(prob(nseq=2), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, 0, None) == INVALID  # needs seq_idx
+    # outside the fused kernels' domain the chunked steps need a workspace
+    q = prob(dtype=ssd.ssd.SSD_DTYPE_F32, headdim=16, dstate=16, chunk=64)
+    need = lib.ssd_sp_summary_workspace_bytes(ctypes.byref(q))
+    assert summ(q, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, 0, None) == WORKSPACE
+    assert summ(q, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, need - 1, None) == WORKSPACE
+    assert summ(q, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE + 8, need, None) == INVALID
     # combine and ownership: rank within [0, nranks), buffers present
     for nranks, rank in ((0, 0), (2, 2), (2, -1)):
         assert lib.ssd_sp_combine(ctypes.byref(p), nranks, rank, FAKE, FAKE, FAKE, None, FAKE, None) == INVALID

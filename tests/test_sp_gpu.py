@@ -31,6 +31,14 @@ CASES = {
     # one short segment holding only the middle of a sequence
     "short_middle_segment": (1, 640, 2, 128, [300, 40, 300], [[200, 400, 40]], "none", True),
 }
+# outside segment_state's domain the summary runs the chunked steps:
+# name: (batch, T, H, P, N, segments, lengths, D, init, dtype, chunk)
+GENERAL = {
+    "f32_tiny_shape_reset": (1, 256, 2, 16, 16, [100, 156], [[128, 128]], "normal", True, "f32", 64),
+    "bf16_N16": (1, 1024, 4, 64, 16, [512, 512], None, "normal", True, "bf16", 256),
+    "bf16_N256_varlen": (1, 1024, 4, 64, 256, [300, 724], [[600, 424]], "normal", True, "bf16", 256),
+    "bf16_P32_three_ranks": (2, 768, 4, 32, 128, [200, 300, 268], None, "none", True, "bf16", 128),
+}
 
 
 def _ssd():
@@ -74,16 +82,20 @@ def _segments(g, seg):
 
 
 def _case(name):
-    batch, T, H, N, seg, lengths, D, init = CASES[name]
+    """(inputs, segments, dtype, chunk) of a named case."""
+    if name in GENERAL:
+        batch, T, H, P, N, seg, lengths, D, init, dtype, chunk = GENERAL[name]
+    else:
+        (batch, T, H, N, seg, lengths, D, init), P, dtype, chunk = CASES[name], 64, "bf16", 256
     assert sum(seg) == T
-    d = make_custom(batch, T, H, 64, N, 1, "bf16", seed=4000 + len(name), has_D=D, has_init=init,
+    d = make_custom(batch, T, H, P, N, 1, dtype, seed=4000 + len(name), has_D=D, has_init=init,
                     lengths=lengths)
-    return d, seg
+    return d, seg, dtype, chunk
 
 
-def _run_threads(d, seg, chunk=256):
+def _run_threads(d, seg, dtype="bf16", chunk=256):
     from mamba_ssd_layer_chunked_b200.sp import ssd_fwd_sp
-    g = to_device(d, "bf16")
+    g = to_device(d, dtype)
     parts = _segments(g, seg)
     group = ThreadGroup(len(seg))
     out = [None] * len(seg)
@@ -113,14 +125,14 @@ def _run_threads(d, seg, chunk=256):
     return Y, finals
 
 
-@pytest.mark.parametrize("name", sorted(CASES))
+@pytest.mark.parametrize("name", sorted(CASES) + sorted(GENERAL))
 def test_sp_emulated_ranks_match_the_whole_sequence(name):
-    d, seg = _case(name)
-    Y, finals = _run_threads(d, seg)
+    d, seg, dtype, chunk = _case(name)
+    Y, finals = _run_threads(d, seg, dtype, chunk)
     Yr, Fr = run_oracle(d)
-    assert_close(Y, Yr, TAU["bf16"], "Y")
+    assert_close(Y, Yr, TAU[dtype], "Y")
     for r, F in enumerate(finals):
-        assert_close(F, Fr, TAU["bf16"], f"final_states on rank {r}")
+        assert_close(F, Fr, TAU[dtype], f"final_states on rank {r}")
         assert np.array_equal(F, finals[0]), "ranks disagree on the final states"
 
 
@@ -131,17 +143,18 @@ def _last_piece_start(seq_row, a, b):
     return a + int(np.argmax(seq_row[a:b] == last))
 
 
-@pytest.mark.parametrize("name", ["varlen_boundary_at_segment_edge", "three_ragged_segments", "skipped_ids"])
+@pytest.mark.parametrize("name", ["varlen_boundary_at_segment_edge", "three_ragged_segments", "skipped_ids",
+                                  "f32_tiny_shape_reset", "bf16_N256_varlen", "bf16_P32_three_ranks"])
 def test_sp_summary_is_the_state_after_the_last_piece(name):
     ssd = _ssd()
-    d, seg = _case(name)
-    g = to_device(d, "bf16")
+    d, seg, dtype, chunk = _case(name)
+    g = to_device(d, dtype)
     parts = _segments(g, seg)
     bounds = np.cumsum([0] + list(seg))
     nseq = d["nseq"] if d["seq_idx"] is not None else 1
     batch, H = d["X"].shape[0], d["X"].shape[2]
     for r, p in enumerate(parts):
-        loc, dec, ids = ssd.sp_summary(p["X"], p["log_a"], p["B"], seq_idx=p["seq_idx"], nseq=nseq)
+        loc, dec, ids = ssd.sp_summary(p["X"], p["log_a"], p["B"], seq_idx=p["seq_idx"], nseq=nseq, chunk=chunk)
         torch.cuda.synchronize()
         a, b = int(bounds[r]), int(bounds[r + 1])
         for bb in range(batch):
@@ -149,7 +162,7 @@ def test_sp_summary_is_the_state_after_the_last_piece(name):
             st = _last_piece_start(row, a, b)
             sl = slice(bb, bb + 1), slice(st, b)
             _, Fr = oracle.ssd_reference(d["X"][sl], d["log_a"][sl], d["B"][sl], d["C"][sl])
-            assert_close(loc[bb].cpu().numpy().astype(np.float64), Fr[0, 0], TAU["bf16"], f"loc r={r} b={bb}")
+            assert_close(loc[bb].cpu().numpy().astype(np.float64), Fr[0, 0], TAU[dtype], f"loc r={r} b={bb}")
             dref = np.exp(d["log_a"][bb, st:b].astype(np.float64).sum(axis=0))
             # an fp32 sum of the piece's log a: relative error ~1e-6 of |sum| in the exponent
             assert_close(dec[bb].cpu().numpy().astype(np.float64), dref, 1e-4, f"dec r={r} b={bb}", atol=1e-30)
