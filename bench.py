@@ -275,12 +275,26 @@ def aggregate(units_per_rank: float, seconds_per_rank: float, device=None):
 # CPU oracle leg
 # --------------------------------------------------------------------------- #
 
-def oracle_sample(w, inputs, budget_s: float = 12.0):
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def oracle_sample(w, inputs, budget_s: float = 12.0, threads: int = 0):
     """Time the oracle on whole (batch row, head) pairs of the workload, one
-    batch row and `cores` heads per call, until about budget_s seconds of CPU
-    work or the whole workload; return (token·heads/s, cores, sample, seconds)."""
+    batch row and `cores` heads per call (cores = threads, or every host core
+    when threads is 0), until about budget_s seconds of CPU work or the whole
+    workload; return (token·heads/s, cores, sample, seconds)."""
     import oracle
-    cores = max(1, oracle.max_threads())
+    cores = threads if threads > 0 else max(1, oracle.max_threads())
     done, t_total = 0, 0.0
     for b in range(w.batch):
         for h0 in range(0, w.nheads, cores):
@@ -568,8 +582,10 @@ def run_ours(args, w):
     }
     if rank == 0 and not args.no_cpu_baseline:
         v, cores, sample, secs = oracle_sample(w, inputs, budget_s=args.cpu_budget)
+        v1, _, sample1, secs1 = oracle_sample(w, inputs, budget_s=max(1.0, args.cpu_budget / 4), threads=1)
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
-                                  "seconds": secs}
+                                  "seconds": secs, "cpu_model": cpu_model(),
+                                  "one_core": {"value": v1, "sample": sample1, "seconds": secs1}}
     if rank == 0:
         print(json.dumps(result), flush=True)
     if ws > 1:
