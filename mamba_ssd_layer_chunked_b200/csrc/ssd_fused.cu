@@ -37,6 +37,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "ssd_tc.cuh"
 #include "tc_ptx.cuh"
@@ -1201,22 +1202,23 @@ int fused_smem_bytes() {
     return (int)FusedSmem<N>::oTail + 1024;
 }
 
+// SM count of the current device, cached per device (host threads may call
+// concurrently: the cache is atomic, and a race only repeats the query)
 int num_sms() {
-    static int n[16] = {0};
+    static std::atomic<int> n[16];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) {
         cudaGetLastError();
         return 148;
     }
-    if (!n[dev]) {
-        int v = 0;
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
-            cudaGetLastError();
-            v = 148;
-        }
-        n[dev] = v;
+    int v = n[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+        cudaGetLastError();
+        v = 148;
     }
-    return n[dev];
+    n[dev].store(v, std::memory_order_relaxed);
+    return v;
 }
 
 Work make_work(const Dims& d, int64_t work_tiles) {
