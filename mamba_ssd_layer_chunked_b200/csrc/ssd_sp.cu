@@ -135,12 +135,16 @@ __global__ void __launch_bounds__(kSpThreads) sp_finish_kernel(Dims d, const flo
 
 unsigned blocks_for(int64_t n) { return (unsigned)((n + kSpThreads - 1) / kSpThreads); }
 
+// grids of one thread per float4 of the state arrays stay within 2^31 - 1 blocks
+bool grid_fits(int64_t n) { return (n + kSpThreads - 1) / kSpThreads <= INT32_MAX; }
+
 }  // namespace
 
 cudaError_t launch_sp_combine(const Dims& d, int nranks, int rank, const float* g_loc, const float* g_dec,
                               const int32_t* g_ids, const float* init_states, float* init_local, cudaStream_t st) {
     const int64_t n = (int64_t)d.batch * d.nseq * d.nheads * (d.dstate * d.headdim / 4);
     if (n == 0) return cudaSuccess;
+    if (!grid_fits(n)) return cudaErrorInvalidConfiguration;
     sp_combine_kernel<<<blocks_for(n), kSpThreads, 0, st>>>(d, nranks, rank, (const float4*)g_loc, g_dec, g_ids,
                                                            (const float4*)init_states, (float4*)init_local);
     return cudaGetLastError();
@@ -158,6 +162,7 @@ cudaError_t launch_sp_own_finals(const Dims& d, int nranks, int rank, const int3
                                  cudaStream_t st) {
     const int64_t n = (int64_t)d.batch * d.nseq * d.nheads * (d.dstate * d.headdim / 4);
     if (n == 0) return cudaSuccess;
+    if (!grid_fits(n)) return cudaErrorInvalidConfiguration;
     sp_own_finals_kernel<<<blocks_for(n), kSpThreads, 0, st>>>(d, nranks, rank, g_ids, (float4*)final_states);
     return cudaGetLastError();
 }
