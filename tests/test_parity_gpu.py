@@ -61,6 +61,10 @@ SMALL = {
     "bf16_N16_Q256": (1, 768, 4, 64, 16, 1, 256, "bf16", None, "none", True),
     "bf16_N256_Q256": (1, 512, 2, 64, 256, 1, 256, "bf16", [[200, 312]], "none", True),
     "bf16_groups2": (2, 512, 4, 64, 128, 2, 128, "bf16", None, "normal", False),
+    # one head per group, and an odd number of heads per group (outside the fused family's pairs)
+    "bf16_group_per_head": (1, 512, 4, 64, 64, 4, 128, "bf16", [[300, 212]], "normal", True),
+    "bf16_three_heads_per_group": (1, 640, 6, 64, 128, 2, 256, "bf16", None, "normal", True),
+    "f32_groups3_P32": (2, 256, 6, 32, 32, 3, 64, "f32", [[100, 156], [256]], "normal", True),
     "bf16_boundary_at_chunk_edge": (1, 768, 2, 64, 128, 1, 256, "bf16", [[256, 256, 256]], "none", True),
     "bf16_short_seqs": (1, 512, 2, 64, 64, 1, 256, "bf16", [[1, 1, 3, 250, 1, 256]], "normal", True),
     "f32_varlen_P32_N48_Q64": (2, 320, 3, 32, 48, 1, 64, "f32", [[1, 63, 64, 100, 92], [320]], "normal", True),
