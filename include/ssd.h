@@ -121,7 +121,8 @@ int ssd_path_supported(const ssd_problem* p, ssd_path path);
 /* Bytes of workspace ssd_fwd needs for p, or (size_t)-1 if p is invalid: for
  * the family ssd_fwd runs (p->path, or for AUTO the fused family where it
  * applies, else the chunked ones), the chunked paths' need (the chunk
- * cumulative sums, batch*nchunks*chunk*nheads fp32, and one state per chunk,
+ * cumulative sums, batch*nchunks*chunk*nheads values, fp64 for the SIMT family
+ * and fp32 for the tcgen05 one, and one state per chunk,
  * batch*nchunks*nheads*dstate*headdim fp32) or the fused path's (two states and
  * two decays per work range, see ssd_fused_work_tiles, plus the padded slices
  * when dstate is not 64 or 128), each part 256-byte aligned. */
@@ -187,7 +188,10 @@ size_t ssd_states_bytes(const ssd_problem* p);
 /* Step 1, chunk_cumsum: cs[b, h, c, k] = sum_{j <= k} log_a[b, c*chunk + j, h],
  * the within-chunk inclusive cumulative sum; exp(cs[k] - cs[l]) is the decay
  * prod_{j=l+1..k} a_j of the segment mask L (papernotes design 2, "A_cumsum"
- * and "L = exp(segment_sum(A))"). */
+ * and "L = exp(segment_sum(A))"). Summed in fp64, stored as fp32: a stored
+ * value carries ~6e-8 |cs| of absolute error, so exp(cs[k] - cs[l]) from these
+ * steps is good to ~1e-7 |cs| relative (ssd_fwd's SIMT family keeps the sums in
+ * fp64 internally, which the 1e-5 fp32 parity needs once |cs| nears 100). */
 ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs, void* stream);
 
 /* Step 2, chunk_state: per chunk c, the end state of the chunk's LAST sequence

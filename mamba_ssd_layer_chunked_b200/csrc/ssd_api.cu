@@ -83,9 +83,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // chunks per row: the last one is partial when chunk does not divide seqlen
 int64_t chunk_count(const ssd_problem* p) { return (p->seqlen + p->chunk - 1) / p->chunk; }
 
-size_t cs_bytes(const ssd_problem* p) {
-    return (size_t)p->batch * chunk_count(p) * p->chunk * p->nheads * sizeof(float);
-}
+// entries of the within-chunk cumsum [b, H, nchunks, Q]
+size_t cs_elems(const ssd_problem* p) { return (size_t)p->batch * chunk_count(p) * p->chunk * p->nheads; }
 
 size_t states_bytes(const ssd_problem* p) {
     return (size_t)p->batch * chunk_count(p) * p->nheads * p->dstate * p->headdim * sizeof(float);
@@ -110,7 +109,11 @@ ssd_path fwd_family(const ssd_problem* p) {
     return SSD_PATH_SIMT;
 }
 
-size_t chunked_workspace_bytes(const ssd_problem* p) { return align256(cs_bytes(p)) + align256(states_bytes(p)); }
+// Workspace of the chunked steps inside ssd_fwd: the cumsum (fp64 for the SIMT
+// kernels, fp32 for the tcgen05 ones) and the chunk states.
+size_t chunked_workspace_bytes(const ssd_problem* p, bool simt) {
+    return align256(cs_elems(p) * (simt ? sizeof(double) : sizeof(float))) + align256(states_bytes(p));
+}
 
 // The sequence-parallel summary runs segment_state where the fused family's
 // kernels cover p (and the path allows it), else the chunked steps, which need
@@ -121,7 +124,7 @@ bool sp_fused(const ssd_problem* p) {
 
 size_t sp_workspace_bytes(const ssd_problem* p) {
     if (sp_fused(p)) return 0;
-    return chunked_workspace_bytes(p) +
+    return chunked_workspace_bytes(p, !use_tc(p)) +
            align256((size_t)p->batch * p->nseq * p->nheads * p->dstate * p->headdim * sizeof(float));
 }
 
@@ -244,7 +247,8 @@ size_t ssd_states_bytes(const ssd_problem* p) {
 size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
     if (check_dims(p) != SSD_OK) return (size_t)-1;
     // the family ssd_fwd runs for p (the same host-side decision)
-    return fwd_family(p) == SSD_PATH_FUSED ? fused_layout(p).total : chunked_workspace_bytes(p);
+    const ssd_path fam = fwd_family(p);
+    return fam == SSD_PATH_FUSED ? fused_layout(p).total : chunked_workspace_bytes(p, fam == SSD_PATH_SIMT);
 }
 
 int64_t ssd_fused_work_tiles(const ssd_problem* p) {
@@ -345,17 +349,24 @@ ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_
         const int64_t nt = ((int64_t)p->seqlen + 127) / 128;  // one work range per (batch row, head pair)
         return cuda_status(ssd::launch_segment_state(d, nt, X, log_a, B, seq_idx, loc, dec, st, ids));
     }
+    const bool tc = use_tc(p);
     char* w = static_cast<char*>(workspace);
-    float* cs = reinterpret_cast<float*>(w);
-    float* states = reinterpret_cast<float*>(w + align256(cs_bytes(p)));
-    float* finals = reinterpret_cast<float*>(w + chunked_workspace_bytes(p));
-    cudaError_t e = ssd::launch_chunk_cumsum(d, log_a, cs, st);
-    if (e != cudaSuccess) return cuda_status(e);
-    e = use_tc(p) ? ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, finals, st)
-                  : ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, finals, st);
-    if (e != cudaSuccess) return cuda_status(e);
-    if ((e = ssd::launch_state_passing(d, cs, states, states, nullptr, seq_idx, finals, st)) != cudaSuccess)
-        return cuda_status(e);
+    float* states = reinterpret_cast<float*>(w + align256(cs_elems(p) * (tc ? sizeof(float) : sizeof(double))));
+    float* finals = reinterpret_cast<float*>(w + chunked_workspace_bytes(p, !tc));
+    cudaError_t e;
+    if (tc) {
+        float* cs = reinterpret_cast<float*>(w);
+        if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
+            (e = ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, finals, st)) != cudaSuccess ||
+            (e = ssd::launch_state_passing(d, cs, states, states, nullptr, seq_idx, finals, st)) != cudaSuccess)
+            return cuda_status(e);
+    } else {
+        double* cs = reinterpret_cast<double*>(w);
+        if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
+            (e = ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, finals, st)) != cudaSuccess ||
+            (e = ssd::launch_state_passing(d, cs, states, states, nullptr, seq_idx, finals, st)) != cudaSuccess)
+            return cuda_status(e);
+    }
     return cuda_status(ssd::launch_sp_finish(d, log_a, seq_idx, finals, loc, dec, ids, st));
 }
 
@@ -525,20 +536,30 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
         }
         return cuda_status(e);
     }
-    float* cs = static_cast<float*>(workspace);
-    float* states = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(cs_bytes(p)));
-    cudaError_t e = ssd::launch_chunk_cumsum(d, log_a, cs, st);
-    if (e != cudaSuccess) return cuda_status(e);
     const bool tc = (fam == SSD_PATH_TCGEN05);
-    e = tc ? ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, final_states, st)
-           : ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st);
-    if (e != cudaSuccess) return cuda_status(e);
-    // in place: the chunk states become the incoming states
-    e = ssd::launch_state_passing(d, cs, states, states, init_states, seq_idx, final_states, st);
-    if (e != cudaSuccess) return cuda_status(e);
-    e = tc ? ssd::launch_chunk_scan_tc(d, X, B, C, cs, D, states, init_states, seq_idx, Y, st)
-           : ssd::launch_chunk_scan_simt(d, p->dtype, X, B, C, cs, D, states, init_states, seq_idx, Y, st);
-    return cuda_status(e);
+    char* w = static_cast<char*>(workspace);
+    float* states = reinterpret_cast<float*>(w + align256(cs_elems(p) * (tc ? sizeof(float) : sizeof(double))));
+    cudaError_t e;
+    if (tc) {
+        float* cs = reinterpret_cast<float*>(w);
+        if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
+            (e = ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, final_states, st)) != cudaSuccess ||
+            // in place: the chunk states become the incoming states
+            (e = ssd::launch_state_passing(d, cs, states, states, init_states, seq_idx, final_states, st)) !=
+                cudaSuccess)
+            return cuda_status(e);
+        return cuda_status(ssd::launch_chunk_scan_tc(d, X, B, C, cs, D, states, init_states, seq_idx, Y, st));
+    }
+    // the SIMT kernels take the cumsum in fp64 (fp32 parity for strongly decaying heads)
+    double* cs = reinterpret_cast<double*>(w);
+    if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
+        (e = ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st)) !=
+            cudaSuccess ||
+        (e = ssd::launch_state_passing(d, cs, states, states, init_states, seq_idx, final_states, st)) !=
+            cudaSuccess)
+        return cuda_status(e);
+    return cuda_status(
+        ssd::launch_chunk_scan_simt(d, p->dtype, X, B, C, cs, D, states, init_states, seq_idx, Y, st));
 }
 
 }  // extern "C"

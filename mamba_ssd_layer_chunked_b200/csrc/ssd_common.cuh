@@ -70,18 +70,32 @@ cudaError_t launch_decode_step(int batch, int nheads, int headdim, int dstate, i
                                const void* x, const float* log_a, const void* B, const void* C, const float* D,
                                float* state, void* y, cudaStream_t st);
 
+// The chunked steps take the within-chunk cumsum as fp32 (the step entry
+// points) or fp64 (ssd_fwd's SIMT family, where exp(cs_k - cs_l) needs the
+// difference to fp32 accuracy); the sums are formed in fp64 either way.
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* log_a, float* cs, cudaStream_t st);
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* log_a, double* cs, cudaStream_t st);
 
 cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,
                                     const float* cs, const int32_t* seq_idx, float* states,
+                                    float* final_states, cudaStream_t st);
+cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,
+                                    const double* cs, const int32_t* seq_idx, float* states,
                                     float* final_states, cudaStream_t st);
 
 cudaError_t launch_state_passing(const Dims& d, const float* cs, const float* chunk_states,
                                  float* incoming, const float* init_states,
                                  const int32_t* seq_idx, float* final_states, cudaStream_t st);
+cudaError_t launch_state_passing(const Dims& d, const double* cs, const float* chunk_states,
+                                 float* incoming, const float* init_states,
+                                 const int32_t* seq_idx, float* final_states, cudaStream_t st);
 
 cudaError_t launch_chunk_scan_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,
                                    const void* C, const float* cs, const float* D,
+                                   const float* incoming, const float* init_states,
+                                   const int32_t* seq_idx, void* Y, cudaStream_t st);
+cudaError_t launch_chunk_scan_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,
+                                   const void* C, const double* cs, const float* D,
                                    const float* incoming, const float* init_states,
                                    const int32_t* seq_idx, void* Y, cudaStream_t st);
 

@@ -25,11 +25,16 @@ constexpr int kThreads = 256;
 // --------------------------------------------------------------------------
 // Step 1: chunk_cumsum. cs[b, h, c, k] = sum_{j<=k} log_a[b, c*Q + j, h].
 // grid.x = batch * nchunks, grid.y = head tiles of 32. The [Q x 32] slab of
-// log_a is read coalesced (heads contiguous), then each warp scans one head.
+// log_a is read coalesced (heads contiguous), then each warp scans one head,
+// summing in double. CsT is the stored type: fp32 for the step entry points,
+// fp64 inside ssd_fwd's SIMT family, whose factors exp(cs_k - cs_l) need the
+// difference to fp32 accuracy: a stored fp32 prefix sum carries an absolute
+// error of ~6e-8 |cs|, i.e. ~1e-5 relative in the factor once |cs| nears 150
+// (strongly decaying heads), which is the fp32 parity bound itself.
 // --------------------------------------------------------------------------
-template <int Q>
+template <int Q, typename CsT>
 __global__ void __launch_bounds__(kThreads) chunk_cumsum_kernel(Dims d, const float* __restrict__ log_a,
-                                                                float* __restrict__ cs) {
+                                                                CsT* __restrict__ cs) {
     __shared__ float slab[Q][33];
     const int c = blockIdx.x % d.nchunks;
     const int b = blockIdx.x / d.nchunks;
@@ -45,23 +50,23 @@ __global__ void __launch_bounds__(kThreads) chunk_cumsum_kernel(Dims d, const fl
     constexpr int PER = Q / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int j = warp; j < nh; j += kThreads / 32) {
-        float v[PER];
-        float run = 0.f;
+        double v[PER];
+        double run = 0.0;
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            run += slab[lane * PER + i][j];
+            run += (double)slab[lane * PER + i][j];
             v[i] = run;
         }
-        float x = run;
+        double x = run;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, x, o);
+            const double y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
-        const float excl = x - run;
-        float* out = cs + cs_off(d, b, h0 + j, c) + lane * PER;
+        const double excl = x - run;
+        CsT* out = cs + cs_off(d, b, h0 + j, c) + lane * PER;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) out[i] = v[i] + excl;
+        for (int i = 0; i < PER; ++i) out[i] = (CsT)(v[i] + excl);
     }
 }
 
@@ -69,17 +74,25 @@ __global__ void __launch_bounds__(kThreads) chunk_cumsum_kernel(Dims d, const fl
 // clamped sequence ids and, per position, the start of its sequence piece
 // inside the chunk (pst[k] = first position k' <= k with the same id).
 struct ChunkMeta {
-    float* cs;   // [Q]
+    double* cs;  // [Q] (fp64, so that differences of the stored values are exact)
     int* seq;    // [Q]
     int* pst;    // [Q]
 };
+// shared-memory words (4 bytes) of a ChunkMeta for chunk length Q
+__host__ __device__ constexpr int meta_words(int Q) { return 4 * Q; }
 
-__device__ void load_chunk_meta(const Dims& d, const float* cs, const int32_t* seq_idx, int b, int h,
+__device__ __forceinline__ ChunkMeta chunk_meta_at(float* smem, int Q) {
+    return ChunkMeta{reinterpret_cast<double*>(smem), reinterpret_cast<int*>(smem + 2 * Q),
+                     reinterpret_cast<int*>(smem + 3 * Q)};
+}
+
+template <typename CsT>
+__device__ void load_chunk_meta(const Dims& d, const CsT* cs, const int32_t* seq_idx, int b, int h,
                                 int c, ChunkMeta m) {
     const int Q = d.chunk;
     const int64_t row = (int64_t)b * d.seqlen;
     for (int k = threadIdx.x; k < Q; k += blockDim.x) {
-        m.cs[k] = cs[cs_off(d, b, h, c) + k];
+        m.cs[k] = (double)cs[cs_off(d, b, h, c) + k];
         m.seq[k] = seq_at_padded(seq_idx, row, c * Q + k, d.seqlen, d.nseq);
     }
     __syncthreads();
@@ -129,10 +142,10 @@ __device__ void chunk_pieces(const int* seqbuf, int Q, int* pstart, int* pseq, i
 // every other piece (each ends inside the chunk) into final_states[b, s].
 // grid.x = (b, h, c) flattened, grid.y = tiles of 8192 outputs; 32 outputs per thread.
 // --------------------------------------------------------------------------
-template <typename T>
+template <typename T, typename CsT>
 __global__ void __launch_bounds__(kThreads) chunk_state_simt_kernel(Dims d, const T* __restrict__ X,
                                                                     const T* __restrict__ B,
-                                                                    const float* __restrict__ cs,
+                                                                    const CsT* __restrict__ cs,
                                                                     const int32_t* __restrict__ seq_idx,
                                                                     float* __restrict__ states,
                                                                     float* __restrict__ final_states) {
@@ -141,8 +154,8 @@ __global__ void __launch_bounds__(kThreads) chunk_state_simt_kernel(Dims d, cons
     const int c = blockIdx.x % d.nchunks;
     const int bh = blockIdx.x / d.nchunks;
     const int h = bh % d.nheads, b = bh / d.nheads, g = h / d.heads_per_group;
-    ChunkMeta m{smem, reinterpret_cast<int*>(smem + Q), reinterpret_cast<int*>(smem + 2 * Q)};
-    float* Bs = smem + 3 * Q;  // [32][N]
+    const ChunkMeta m = chunk_meta_at(smem, Q);
+    float* Bs = smem + meta_words(Q);  // [32][N]
     float* Xs = Bs + 32 * N;   // [32][P]
     load_chunk_meta(d, cs, seq_idx, b, h, c, m);
 
@@ -158,7 +171,7 @@ __global__ void __launch_bounds__(kThreads) chunk_state_simt_kernel(Dims d, cons
         float acc[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-        const float cs_end = m.cs[e];
+        const double cs_end = m.cs[e];
         for (int l0 = st; l0 <= e; l0 += 32) {
             const int nl = min(32, e - l0 + 1);
             for (int i = threadIdx.x; i < 32 * N; i += kThreads) {
@@ -169,7 +182,7 @@ __global__ void __launch_bounds__(kThreads) chunk_state_simt_kernel(Dims d, cons
                 const int li = i / P, p = i % P;
                 float v = 0.f;
                 if (li < nl && t0 + l0 + li < d.seqlen)
-                    v = expf(cs_end - m.cs[l0 + li]) * to_f32(X[x_off(d, b, t0 + l0 + li, h) + p]);
+                    v = expf((float)(cs_end - m.cs[l0 + li])) * to_f32(X[x_off(d, b, t0 + l0 + li, h) + p]);
                 Xs[i] = v;
             }
             __syncthreads();
@@ -211,7 +224,8 @@ __device__ __forceinline__ float4 axpy4(float a, float4 x, float4 y) {
     return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
 }
 
-__global__ void __launch_bounds__(kThreads) state_passing_kernel(Dims d, const float* __restrict__ cs,
+template <typename CsT>
+__global__ void __launch_bounds__(kThreads) state_passing_kernel(Dims d, const CsT* __restrict__ cs,
                                                                  const float* chunk_states, float* incoming,
                                                                  const float* __restrict__ init_states,
                                                                  const int32_t* __restrict__ seq_idx,
@@ -236,7 +250,11 @@ __global__ void __launch_bounds__(kThreads) state_passing_kernel(Dims d, const f
     float4 H = zero;
     int s_prev_last = 0;
     for (int c = 0; c < d.nchunks; ++c) {
-        const float* csr = cs + cs_off(d, b, h, c);
+        const CsT* csr = cs + cs_off(d, b, h, c);
+        // decay over positions (st - 1, e] of the chunk, the difference taken in fp64
+        auto piece_decay = [&](int st, int e) {
+            return expf((float)((double)csr[e] - (st > 0 ? (double)csr[st - 1] : 0.0)));
+        };
         if (seq_idx) {
             __syncthreads();
             if (threadIdx.x < Q) seqbuf[threadIdx.x] = seq_at_padded(seq_idx, row, c * Q + threadIdx.x, d.seqlen, d.nseq);
@@ -266,14 +284,14 @@ __global__ void __launch_bounds__(kThreads) state_passing_kernel(Dims d, const f
             for (int j = 0; j + 1 < np; ++j) {
                 const int st = pstart[j], e = pstart[j + 1] - 1, s = pseq[j];
                 const float4 hs = (j == 0) ? hin : init_of(s);
-                const float decay = expf(csr[e] - (st > 0 ? csr[st - 1] : 0.f));
+                const float decay = piece_decay(st, e);
                 float* f = final_states + seqst_off(d, b, s, h) + idx;
                 st4(f, axpy4(decay, hs, ld4(f)));
             }
         }
         const int st_last = seq_idx ? pstart[np - 1] : 0;
         const float4 hstart = (np == 1) ? hin : init_of(s_last);
-        const float decay = expf(csr[Q - 1] - (st_last > 0 ? csr[st_last - 1] : 0.f));
+        const float decay = piece_decay(st_last, Q - 1);
         H = axpy4(decay, hstart, S);
         if (final_states && active) {
             bool ends = (c == d.nchunks - 1);
@@ -297,10 +315,10 @@ __global__ void __launch_bounds__(kThreads) state_passing_kernel(Dims d, const f
 constexpr int kRows = 64;
 constexpr int kMaxOut = kRows * 256 / kThreads;  // 64 outputs per thread at P = 256
 
-template <typename T>
+template <typename T, typename CsT>
 __global__ void __launch_bounds__(kThreads) chunk_scan_simt_kernel(
     Dims d, const T* __restrict__ X, const T* __restrict__ B, const T* __restrict__ C,
-    const float* __restrict__ cs, const float* __restrict__ D, const float* __restrict__ incoming,
+    const CsT* __restrict__ cs, const float* __restrict__ D, const float* __restrict__ incoming,
     const float* __restrict__ init_states, const int32_t* __restrict__ seq_idx, T* __restrict__ Y) {
     extern __shared__ float smem[];
     const int Q = d.chunk, N = d.dstate, P = d.headdim;
@@ -311,9 +329,9 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_simt_kernel(
     const int c = r % d.nchunks;
     r /= d.nchunks;
     const int h = r % d.nheads, b = r / d.nheads, g = h / d.heads_per_group;
-    ChunkMeta m{smem, reinterpret_cast<int*>(smem + Q), reinterpret_cast<int*>(smem + 2 * Q)};
-    const int NS = N + 1;           // padded row stride of Cs and Bs
-    float* Cs = smem + 3 * Q;       // [64][N+1]
+    const ChunkMeta m = chunk_meta_at(smem, Q);
+    const int NS = N + 1;               // padded row stride of Cs and Bs
+    float* Cs = smem + meta_words(Q);   // [64][N+1]
     float* Bs = Cs + kRows * NS;    // [32][N+1]
     float* Xs = Bs + 32 * NS;       // [32][P]
     float* Ws = Xs + 32 * P;        // [64][33]
@@ -369,7 +387,7 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_simt_kernel(
             const int o = j * kThreads + threadIdx.x;
             const int k = k0 + o / P;
             const int pst = m.pst[k];
-            acc[j] *= expf(m.cs[k] - (pst > 0 ? m.cs[pst - 1] : 0.f));
+            acc[j] *= expf((float)(m.cs[k] - (pst > 0 ? m.cs[pst - 1] : 0.0)));
         }
     }
 
@@ -392,7 +410,7 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_simt_kernel(
             if (l <= k && m.pst[l] == m.pst[k]) {
                 float dot = 0.f;
                 for (int n = 0; n < N; ++n) dot = fmaf(Cs[rr * NS + n], Bs[li * NS + n], dot);
-                w = expf(m.cs[k] - m.cs[l]) * dot;
+                w = expf((float)(m.cs[k] - m.cs[l])) * dot;
             }
             Ws[rr * 33 + li] = w;
         }
@@ -447,65 +465,118 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, int slot) {
     return e;
 }
 
-cudaError_t launch_chunk_cumsum(const Dims& d, const float* log_a, float* cs, cudaStream_t st) {
+namespace {
+
+// shared-memory attribute slots: 0-3 with fp32 cs, 4-7 with fp64 cs
+template <typename CsT>
+constexpr int cs_slot() {
+    return sizeof(CsT) == 8 ? 4 : 0;
+}
+
+template <typename CsT>
+cudaError_t chunk_cumsum_impl(const Dims& d, const float* log_a, CsT* cs, cudaStream_t st) {
     dim3 grid(d.batch * d.nchunks, (d.nheads + 31) / 32);
     switch (d.chunk) {
-        case 64: chunk_cumsum_kernel<64><<<grid, kThreads, 0, st>>>(d, log_a, cs); break;
-        case 128: chunk_cumsum_kernel<128><<<grid, kThreads, 0, st>>>(d, log_a, cs); break;
-        case 256: chunk_cumsum_kernel<256><<<grid, kThreads, 0, st>>>(d, log_a, cs); break;
+        case 64: chunk_cumsum_kernel<64, CsT><<<grid, kThreads, 0, st>>>(d, log_a, cs); break;
+        case 128: chunk_cumsum_kernel<128, CsT><<<grid, kThreads, 0, st>>>(d, log_a, cs); break;
+        case 256: chunk_cumsum_kernel<256, CsT><<<grid, kThreads, 0, st>>>(d, log_a, cs); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,
-                                    const float* cs, const int32_t* seq_idx, float* states,
-                                    float* final_states, cudaStream_t st) {
-    const int smem = (3 * d.chunk + 32 * d.dstate + 32 * d.headdim) * 4;
+template <typename CsT>
+cudaError_t chunk_state_simt_impl(const Dims& d, ssd_dtype dt, const void* X, const void* B, const CsT* cs,
+                                  const int32_t* seq_idx, float* states, float* final_states, cudaStream_t st) {
+    const int smem = (meta_words(d.chunk) + 32 * d.dstate + 32 * d.headdim) * 4;
     dim3 grid(d.batch * d.nheads * d.nchunks, (d.dstate * d.headdim + 8191) / 8192);
     cudaError_t e;
     if (dt == SSD_DTYPE_F32) {
-        auto k = chunk_state_simt_kernel<float>;
-        if ((e = ensure_smem_attr((const void*)k, smem, 0)) != cudaSuccess) return e;
+        auto k = chunk_state_simt_kernel<float, CsT>;
+        if ((e = ensure_smem_attr((const void*)k, smem, cs_slot<CsT>() + 0)) != cudaSuccess) return e;
         k<<<grid, kThreads, smem, st>>>(d, (const float*)X, (const float*)B, cs, seq_idx, states, final_states);
     } else {
-        auto k = chunk_state_simt_kernel<__nv_bfloat16>;
-        if ((e = ensure_smem_attr((const void*)k, smem, 1)) != cudaSuccess) return e;
+        auto k = chunk_state_simt_kernel<__nv_bfloat16, CsT>;
+        if ((e = ensure_smem_attr((const void*)k, smem, cs_slot<CsT>() + 1)) != cudaSuccess) return e;
         k<<<grid, kThreads, smem, st>>>(d, (const __nv_bfloat16*)X, (const __nv_bfloat16*)B, cs, seq_idx, states,
                                         final_states);
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_state_passing(const Dims& d, const float* cs, const float* chunk_states, float* incoming,
-                                 const float* init_states, const int32_t* seq_idx, float* final_states,
-                                 cudaStream_t st) {
+template <typename CsT>
+cudaError_t state_passing_impl(const Dims& d, const CsT* cs, const float* chunk_states, float* incoming,
+                               const float* init_states, const int32_t* seq_idx, float* final_states,
+                               cudaStream_t st) {
     dim3 grid(d.batch * d.nheads, (d.dstate * d.headdim + 4 * kThreads - 1) / (4 * kThreads));
-    state_passing_kernel<<<grid, kThreads, 0, st>>>(d, cs, chunk_states, incoming, init_states, seq_idx,
-                                                    final_states);
+    state_passing_kernel<CsT><<<grid, kThreads, 0, st>>>(d, cs, chunk_states, incoming, init_states, seq_idx,
+                                                         final_states);
     return cudaGetLastError();
 }
 
-cudaError_t launch_chunk_scan_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B, const void* C,
-                                   const float* cs, const float* D, const float* incoming,
-                                   const float* init_states, const int32_t* seq_idx, void* Y, cudaStream_t st) {
-    const int smem = (3 * d.chunk + kRows * (d.dstate + 1) + 32 * (d.dstate + 1) + 32 * d.headdim + kRows * 33 +
-                      32 * d.headdim) * 4;
+template <typename CsT>
+cudaError_t chunk_scan_simt_impl(const Dims& d, ssd_dtype dt, const void* X, const void* B, const void* C,
+                                 const CsT* cs, const float* D, const float* incoming, const float* init_states,
+                                 const int32_t* seq_idx, void* Y, cudaStream_t st) {
+    const int smem = (meta_words(d.chunk) + kRows * (d.dstate + 1) + 32 * (d.dstate + 1) + 32 * d.headdim +
+                      kRows * 33 + 32 * d.headdim) * 4;
     dim3 grid(d.batch * d.nheads * d.nchunks * (d.chunk / kRows));
     cudaError_t e;
     if (dt == SSD_DTYPE_F32) {
-        auto k = chunk_scan_simt_kernel<float>;
-        if ((e = ensure_smem_attr((const void*)k, smem, 2)) != cudaSuccess) return e;
+        auto k = chunk_scan_simt_kernel<float, CsT>;
+        if ((e = ensure_smem_attr((const void*)k, smem, cs_slot<CsT>() + 2)) != cudaSuccess) return e;
         k<<<grid, kThreads, smem, st>>>(d, (const float*)X, (const float*)B, (const float*)C, cs, D, incoming,
                                         init_states, seq_idx, (float*)Y);
     } else {
-        auto k = chunk_scan_simt_kernel<__nv_bfloat16>;
-        if ((e = ensure_smem_attr((const void*)k, smem, 3)) != cudaSuccess) return e;
+        auto k = chunk_scan_simt_kernel<__nv_bfloat16, CsT>;
+        if ((e = ensure_smem_attr((const void*)k, smem, cs_slot<CsT>() + 3)) != cudaSuccess) return e;
         k<<<grid, kThreads, smem, st>>>(d, (const __nv_bfloat16*)X, (const __nv_bfloat16*)B,
                                         (const __nv_bfloat16*)C, cs, D, incoming, init_states, seq_idx,
                                         (__nv_bfloat16*)Y);
     }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* log_a, float* cs, cudaStream_t st) {
+    return chunk_cumsum_impl(d, log_a, cs, st);
+}
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* log_a, double* cs, cudaStream_t st) {
+    return chunk_cumsum_impl(d, log_a, cs, st);
+}
+
+cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,
+                                    const float* cs, const int32_t* seq_idx, float* states,
+                                    float* final_states, cudaStream_t st) {
+    return chunk_state_simt_impl(d, dt, X, B, cs, seq_idx, states, final_states, st);
+}
+cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B,
+                                    const double* cs, const int32_t* seq_idx, float* states,
+                                    float* final_states, cudaStream_t st) {
+    return chunk_state_simt_impl(d, dt, X, B, cs, seq_idx, states, final_states, st);
+}
+
+cudaError_t launch_state_passing(const Dims& d, const float* cs, const float* chunk_states, float* incoming,
+                                 const float* init_states, const int32_t* seq_idx, float* final_states,
+                                 cudaStream_t st) {
+    return state_passing_impl(d, cs, chunk_states, incoming, init_states, seq_idx, final_states, st);
+}
+cudaError_t launch_state_passing(const Dims& d, const double* cs, const float* chunk_states, float* incoming,
+                                 const float* init_states, const int32_t* seq_idx, float* final_states,
+                                 cudaStream_t st) {
+    return state_passing_impl(d, cs, chunk_states, incoming, init_states, seq_idx, final_states, st);
+}
+
+cudaError_t launch_chunk_scan_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B, const void* C,
+                                   const float* cs, const float* D, const float* incoming,
+                                   const float* init_states, const int32_t* seq_idx, void* Y, cudaStream_t st) {
+    return chunk_scan_simt_impl(d, dt, X, B, C, cs, D, incoming, init_states, seq_idx, Y, st);
+}
+cudaError_t launch_chunk_scan_simt(const Dims& d, ssd_dtype dt, const void* X, const void* B, const void* C,
+                                   const double* cs, const float* D, const float* incoming,
+                                   const float* init_states, const int32_t* seq_idx, void* Y, cudaStream_t st) {
+    return chunk_scan_simt_impl(d, dt, X, B, C, cs, D, incoming, init_states, seq_idx, Y, st);
 }
 
 }  // namespace ssd

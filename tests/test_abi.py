@@ -45,7 +45,7 @@ def test_status_strings():
 def test_workspace_bytes_formula():
     p = prob()
     align = lambda x: (x + 255) // 256 * 256
-    cs = 2 * 512 * 4 * 4
+    cs = 2 * 512 * 4 * 4  # fp32 cumsum (the tcgen05 family); the SIMT family keeps it in fp64
     st = 2 * (512 // 256) * 4 * 128 * 64 * 4
     # fused: rows (batch, head pair) = 4, 4 tiles each; ranges of wt tiles
     wt = ssd.fused_work_tiles(p)
@@ -55,12 +55,13 @@ def test_workspace_bytes_formula():
     assert ssd.fused_work_count(p, wt) == nwork
     fused = 2 * align(nwork * 2 * 128 * 64 * 4) + align(nwork * 2 * 4)
     assert ssd.workspace_bytes(p) == fused  # AUTO runs the fused family for this problem
-    assert ssd.workspace_bytes(prob(path=1)) == align(cs) + align(st)  # the SIMT family: the chunked need
+    assert ssd.workspace_bytes(prob(path=1)) == align(2 * cs) + align(st)  # the SIMT family: the chunked need
+    assert ssd.workspace_bytes(prob(path=2)) == align(cs) + align(st)  # the chunked tcgen05 family
     assert ssd.states_bytes(p) == st
     # outside the fused domain (fp32) only the chunked need counts
     q = prob(dtype=ssd.ssd.SSD_DTYPE_F32)
     assert ssd.fused_work_tiles(q) == -1
-    assert ssd.workspace_bytes(q) == align(cs) + align(st)
+    assert ssd.workspace_bytes(q) == align(2 * cs) + align(st)
 
 
 def test_fused_work_count():
@@ -131,13 +132,15 @@ def test_sp_summary_workspace_formula():
     size = lambda q: lib.ssd_sp_summary_workspace_bytes(ctypes.byref(q))
     # segment_state covers bf16, P 64, N 64 or 128: no workspace
     assert size(prob()) == 0 and size(prob(dstate=64)) == 0
-    # the chunked steps: cumsum, chunk states, final states from zero
-    for q, (b, T, H, P, N, Q, S) in ((prob(dtype=ssd.ssd.SSD_DTYPE_F32, headdim=16, dstate=16, chunk=64),
-                                      (2, 512, 4, 16, 16, 64, 1)),
-                                     (prob(dstate=256), (2, 512, 4, 64, 256, 256, 1)),
-                                     (prob(seqlen=500, nseq=3, path=1), (2, 500, 4, 64, 128, 256, 3))):
+    # the chunked steps: cumsum (fp64 for the SIMT kernels, fp32 for the tcgen05 ones),
+    # chunk states, final states from zero
+    for q, (b, T, H, P, N, Q, S, csb) in ((prob(dtype=ssd.ssd.SSD_DTYPE_F32, headdim=16, dstate=16, chunk=64),
+                                           (2, 512, 4, 16, 16, 64, 1, 8)),
+                                          (prob(dstate=256), (2, 512, 4, 64, 256, 256, 1, 8)),
+                                          (prob(seqlen=500, nseq=3, path=1), (2, 500, 4, 64, 128, 256, 3, 8)),
+                                          (prob(path=2), (2, 512, 4, 64, 128, 256, 1, 4))):
         nc = -(-T // Q)
-        want = align(b * nc * Q * H * 4) + align(b * nc * H * N * P * 4) + align(b * S * H * N * P * 4)
+        want = align(b * nc * Q * H * csb) + align(b * nc * H * N * P * 4) + align(b * S * H * N * P * 4)
         assert size(q) == want
     assert size(prob(batch=0)) == ctypes.c_size_t(-1).value
 
