@@ -62,3 +62,48 @@ def test_random_problem_every_family(i):
         assert_close(F, Fr, TAU[dtype], f"final_states ({path}; {desc})")
         ran += 1
     assert ran >= 2  # auto and at least the SIMT family
+
+
+NLARGE = 8
+
+
+def _draw_large(i):
+    """Larger bf16 problems in the fused family's domain, long enough that its
+    work ranges cut rows and chain the pieces before each cut."""
+    rng = np.random.default_rng(9000 + i)
+    b = int(rng.integers(1, 4))
+    T = int(rng.integers(1000, 4097))
+    H = int(rng.choice([2, 4, 6, 8]))
+    G = int(rng.choice([g for g in (1, 2) if (H // g) % 2 == 0 and H % g == 0]))
+    N = int(rng.choice([64, 128]))
+    Q = int(rng.choice([128, 256]))
+    lengths = None
+    if rng.random() < 0.5:
+        nseq = int(rng.integers(1, 9))
+        lengths = []
+        for _ in range(b):
+            cuts = np.sort(rng.integers(0, T + 1, size=nseq - 1))
+            lengths.append(np.diff(np.concatenate([[0], cuts, [T]])).astype(int).tolist())
+    D = str(rng.choice(["none", "normal"]))
+    init = bool(rng.random() < 0.5)
+    nseq = None if lengths is None else max(len(r) for r in lengths)
+    d = make_custom(b, T, H, 64, N, ngroups=G, dtype="bf16", seed=int(rng.integers(0, 10000)), has_D=D,
+                    has_init=init, lengths=lengths, nseq=nseq)
+    return d, Q, f"bf16 b{b} T{T} H{H} G{G} N{N} Q{Q} nseq={nseq} D={D} init={init}"
+
+
+@pytest.mark.parametrize("i", range(NLARGE))
+def test_random_large_problem_fused_and_chunked(i):
+    import mamba_ssd_layer_chunked_b200 as ssd
+    d, Q, desc = _draw_large(i)
+    Yr, Fr = run_oracle(d)
+    X = d["X"]
+    p = ssd.make_problem(X.shape[0], X.shape[1], X.shape[2], 64, d["B"].shape[3], d["B"].shape[2], Q, d["nseq"],
+                         torch.bfloat16)
+    assert ssd.path_supported(p, "fused")
+    for path in ("auto", "fused", "tcgen05"):
+        if not ssd.path_supported(p, path) and path != "auto":
+            continue
+        Y, F = run_gpu(d, "bf16", Q, path)
+        assert_close(Y, Yr, TAU["bf16"], f"Y ({path}; {desc})")
+        assert_close(F, Fr, TAU["bf16"], f"final_states ({path}; {desc})")
