@@ -34,21 +34,35 @@ constexpr int kSpThreads = 256;
 // earlier ranks j: start_j = E_{j-1} when segment j is one sequence piece that
 // continues rank j-1's last sequence, else the initial state of its last
 // sequence; E_j = dec_j start_j + loc_j.
+// Index split of thread i over [b, s, h, NP4] in the index type I (32-bit
+// where the element count fits: a 64-bit division by a runtime divisor costs
+// more than the rest of these threads' work).
+template <typename I>
+struct BshIndex {
+    int b, s, h, e4;
+    __device__ BshIndex(I i, const Dims& d, I NP4) {
+        const I bsh = i / NP4;
+        e4 = (int)(i - bsh * NP4);
+        const I bs = bsh / (I)d.nheads;
+        h = (int)(bsh - bs * (I)d.nheads);
+        const I bb = bs / (I)d.nseq;
+        s = (int)(bs - bb * (I)d.nseq);
+        b = (int)bb;
+    }
+};
+
+template <typename I>
 __global__ void __launch_bounds__(kSpThreads) sp_combine_kernel(Dims d, int nranks, int rank,
                                                                 const float4* __restrict__ g_loc,
                                                                 const float* __restrict__ g_dec,
                                                                 const int32_t* __restrict__ g_ids,
                                                                 const float4* __restrict__ init_states,
-                                                                float4* __restrict__ init_local) {
+                                                                float4* __restrict__ init_local, I n_all) {
     const int NP4 = d.dstate * d.headdim / 4;
-    const int64_t n_all = (int64_t)d.batch * d.nseq * d.nheads * NP4;
-    const int64_t i = (int64_t)blockIdx.x * kSpThreads + threadIdx.x;
+    const I i = (I)blockIdx.x * kSpThreads + threadIdx.x;
     if (i >= n_all) return;
-    const int e4 = (int)(i % NP4);
-    const int64_t bsh = i / NP4;
-    const int h = (int)(bsh % d.nheads);
-    const int s = (int)((bsh / d.nheads) % d.nseq);
-    const int b = (int)(bsh / ((int64_t)d.nheads * d.nseq));
+    const BshIndex<I> x(i, d, (I)NP4);
+    const int b = x.b, s = x.s, h = x.h, e4 = x.e4;
     auto init_of = [&](int sq) -> float4 {
         return init_states ? init_states[seqst_off(d, b, sq, h) / 4 + e4] : make_float4(0.f, 0.f, 0.f, 0.f);
     };
@@ -75,16 +89,15 @@ __global__ void __launch_bounds__(kSpThreads) sp_combine_kernel(Dims d, int nran
 
 // zero final_states[b, s] unless rank is its owner: the last rank whose first
 // id is <= s (rank 0 when there is none)
+template <typename I>
 __global__ void __launch_bounds__(kSpThreads) sp_own_finals_kernel(Dims d, int nranks, int rank,
                                                                    const int32_t* __restrict__ g_ids,
-                                                                   float4* __restrict__ final_states) {
+                                                                   float4* __restrict__ final_states, I n_all) {
     const int NP4 = d.dstate * d.headdim / 4;
-    const int64_t n_all = (int64_t)d.batch * d.nseq * d.nheads * NP4;
-    const int64_t i = (int64_t)blockIdx.x * kSpThreads + threadIdx.x;
+    const I i = (I)blockIdx.x * kSpThreads + threadIdx.x;
     if (i >= n_all) return;
-    const int64_t bsh = i / NP4;
-    const int s = (int)((bsh / d.nheads) % d.nseq);
-    const int b = (int)(bsh / ((int64_t)d.nheads * d.nseq));
+    const BshIndex<I> x(i, d, (I)NP4);
+    const int b = x.b, s = x.s;
     int owner = 0;
     for (int j = 0; j < nranks; ++j)
         if (g_ids[2 * ((int64_t)j * d.batch + b)] <= s) owner = j;
@@ -145,8 +158,13 @@ cudaError_t launch_sp_combine(const Dims& d, int nranks, int rank, const float* 
     const int64_t n = (int64_t)d.batch * d.nseq * d.nheads * (d.dstate * d.headdim / 4);
     if (n == 0) return cudaSuccess;
     if (!grid_fits(n)) return cudaErrorInvalidConfiguration;
-    sp_combine_kernel<<<blocks_for(n), kSpThreads, 0, st>>>(d, nranks, rank, (const float4*)g_loc, g_dec, g_ids,
-                                                           (const float4*)init_states, (float4*)init_local);
+    if (n + kSpThreads < (int64_t)UINT32_MAX)
+        sp_combine_kernel<uint32_t><<<blocks_for(n), kSpThreads, 0, st>>>(
+            d, nranks, rank, (const float4*)g_loc, g_dec, g_ids, (const float4*)init_states, (float4*)init_local,
+            (uint32_t)n);
+    else
+        sp_combine_kernel<int64_t><<<blocks_for(n), kSpThreads, 0, st>>>(
+            d, nranks, rank, (const float4*)g_loc, g_dec, g_ids, (const float4*)init_states, (float4*)init_local, n);
     return cudaGetLastError();
 }
 
@@ -163,7 +181,12 @@ cudaError_t launch_sp_own_finals(const Dims& d, int nranks, int rank, const int3
     const int64_t n = (int64_t)d.batch * d.nseq * d.nheads * (d.dstate * d.headdim / 4);
     if (n == 0) return cudaSuccess;
     if (!grid_fits(n)) return cudaErrorInvalidConfiguration;
-    sp_own_finals_kernel<<<blocks_for(n), kSpThreads, 0, st>>>(d, nranks, rank, g_ids, (float4*)final_states);
+    if (n + kSpThreads < (int64_t)UINT32_MAX)
+        sp_own_finals_kernel<uint32_t><<<blocks_for(n), kSpThreads, 0, st>>>(d, nranks, rank, g_ids,
+                                                                             (float4*)final_states, (uint32_t)n);
+    else
+        sp_own_finals_kernel<int64_t><<<blocks_for(n), kSpThreads, 0, st>>>(d, nranks, rank, g_ids,
+                                                                            (float4*)final_states, n);
     return cudaGetLastError();
 }
 
