@@ -23,7 +23,7 @@ namespace ssd {
 
 namespace {
 
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 128;  // small CTAs: 16 per SM, a finer last wave
 
 template <typename T>
 __device__ __forceinline__ float4 load4(const T* p);
