@@ -5,6 +5,8 @@ off), each run through every family that covers it and compared with the CPU
 fp64 oracle under the parity rule max|gpu - oracle| <= tau * max|oracle|
 (tau = 1e-5 for fp32 inputs, 2e-2 for bf16 inputs with fp32 state).
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -14,7 +16,8 @@ from workloads import make_custom
 
 pytestmark = pytest.mark.gpu
 
-NPROBLEMS = 64
+# more problems for a longer stress run: SSD_RANDOM_PROBLEMS=400 pytest ...
+NPROBLEMS = int(os.environ.get("SSD_RANDOM_PROBLEMS", "64"))
 
 
 def _draw(i):
