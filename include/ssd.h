@@ -28,7 +28,10 @@
  *    is set once. Every call is asynchronous on `stream` (a cudaStream_t passed
  *    as void*; NULL means the legacy default stream) and is thread-safe.
  *  - Layouts are dense row-major (C order) with the last dimension contiguous.
- *    Every pointer must be 16-byte aligned.
+ *    Every pointer must be 16-byte aligned, except log_a, D and seq_idx,
+ *    which are read one element at a time and need only their natural 4-byte
+ *    alignment (a segment of a batch-1 tensor starts wherever its first token
+ *    does); the exceptions each entry point states.
  *  - Arguments are validated on the host before anything is launched; on an
  *    error status nothing has been enqueued. SSD_ERR_CUDA reports a launch
  *    error (the message of cudaGetLastError is available from

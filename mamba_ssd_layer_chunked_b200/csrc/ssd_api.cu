@@ -208,6 +208,17 @@ bool all_aligned(Ptrs... ps) {
     return true;
 }
 
+// log a, D and seq_idx are read one element at a time: their natural 4-byte
+// alignment suffices (a segment of a batch-1 tensor, for one, starts wherever
+// its first token does)
+template <typename... Ptrs>
+bool all_aligned4(Ptrs... ps) {
+    const void* arr[] = {static_cast<const void*>(ps)...};
+    for (const void* q : arr)
+        if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return false;
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -269,7 +280,7 @@ ssd_status ssd_segment_state(const ssd_problem* p, int64_t work_tiles, const voi
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !work_local || !work_decay) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, seq_idx, work_local, work_decay)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, B, work_local, work_decay) || !all_aligned4(log_a, seq_idx)) return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = make_dims(p);
     if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
     if ((s = check_device()) != SSD_OK) return s;
@@ -284,7 +295,8 @@ ssd_status ssd_segment_passing(const ssd_problem* p, int64_t work_tiles, const f
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!work_local || !work_decay || !work_incoming) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(work_local, work_decay, init_states, seq_idx, work_incoming)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(work_local, work_decay, init_states, work_incoming) || !all_aligned4(seq_idx))
+        return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = make_dims(p);
     if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
     if ((s = check_device()) != SSD_OK) return s;
@@ -299,7 +311,7 @@ ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* 
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, C, D, work_incoming, init_states, seq_idx, Y, final_states))
+    if (!all_aligned(X, B, C, work_incoming, init_states, Y, final_states) || !all_aligned4(log_a, D, seq_idx))
         return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = make_dims(p);
     if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
@@ -317,7 +329,7 @@ ssd_status ssd_fused_scan_chained(const ssd_problem* p, int64_t work_tiles, cons
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, C, D, work_local, work_decay, init_states, seq_idx, Y, final_states))
+    if (!all_aligned(X, B, C, work_local, work_decay, init_states, Y, final_states) || !all_aligned4(log_a, D, seq_idx))
         return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = make_dims(p);
     if (!ssd::fused_work_ok(d, work_tiles)) return SSD_ERR_INVALID_ARG;
@@ -339,7 +351,7 @@ ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !loc || !dec || !ids) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, seq_idx, loc, dec, ids, workspace)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, B, loc, dec, ids, workspace) || !all_aligned4(log_a, seq_idx)) return SSD_ERR_INVALID_ARG;
     const size_t need = sp_workspace_bytes(p);
     if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
     if ((s = check_runnable(p)) != SSD_OK) return s;
@@ -441,7 +453,7 @@ ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs,
     ssd_status s = check_dims(p);  // log a only: nseq and seq_idx play no part here
     if (s != SSD_OK) return s;
     if (!log_a || !cs) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(log_a, cs)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(cs) || !all_aligned4(log_a)) return SSD_ERR_INVALID_ARG;
     if ((s = check_device()) != SSD_OK) return s;
     return cuda_status(ssd::launch_chunk_cumsum(make_dims(p), log_a, cs, (cudaStream_t)stream));
 }
@@ -451,7 +463,7 @@ ssd_status ssd_chunk_state(const ssd_problem* p, const void* X, const void* B, c
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !B || !cs || !states) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, B, cs, seq_idx, states, final_states)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, B, cs, states, final_states) || !all_aligned4(seq_idx)) return SSD_ERR_INVALID_ARG;
     if ((s = check_runnable(p)) != SSD_OK) return s;
     const ssd::Dims d = make_dims(p);
     cudaStream_t st = (cudaStream_t)stream;
@@ -465,7 +477,8 @@ ssd_status ssd_state_passing(const ssd_problem* p, const float* cs, const float*
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!cs || !chunk_states || !incoming) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(cs, chunk_states, incoming, init_states, seq_idx, final_states)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(cs, chunk_states, incoming, init_states, final_states) || !all_aligned4(seq_idx))
+        return SSD_ERR_INVALID_ARG;
     if ((s = check_runnable(p)) != SSD_OK) return s;
     return cuda_status(ssd::launch_state_passing(make_dims(p), cs, chunk_states, incoming, init_states, seq_idx,
                                                  final_states, (cudaStream_t)stream));
@@ -477,7 +490,7 @@ ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, co
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !B || !C || !cs || !incoming || !Y) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, B, C, cs, D, incoming, init_states, seq_idx, Y)) return SSD_ERR_INVALID_ARG;
+    if (!all_aligned(X, B, C, cs, incoming, init_states, Y) || !all_aligned4(D, seq_idx)) return SSD_ERR_INVALID_ARG;
     if ((s = check_runnable(p)) != SSD_OK) return s;
     const ssd::Dims d = make_dims(p);
     cudaStream_t st = (cudaStream_t)stream;
@@ -493,7 +506,7 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
-    if (!all_aligned(X, log_a, B, C, D, init_states, seq_idx, Y, final_states, workspace))
+    if (!all_aligned(X, B, C, init_states, Y, final_states, workspace) || !all_aligned4(log_a, D, seq_idx))
         return SSD_ERR_INVALID_ARG;
     const size_t need = ssd_fwd_workspace_bytes(p);
     if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;

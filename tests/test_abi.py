@@ -115,11 +115,9 @@ def test_null_required_pointer(arg):
 
 @pytest.mark.parametrize("arg", ["X", "la", "B", "C", "D", "init", "seq", "Y", "fin", "ws"])
 def test_misaligned_pointer(arg):
+    # 16-byte alignment, except log a, D and seq_idx: 4-byte (read one element at a time)
     p = prob(nseq=2) if arg == "seq" else prob()
-    kw = {arg: FAKE + 4}
-    if arg == "seq":
-        kw = {"seq": FAKE + 4}
-    assert _fwd(p, **kw) == INVALID
+    assert _fwd(p, **{arg: FAKE + (2 if arg in ("la", "D", "seq") else 4)}) == INVALID
 
 
 def test_nseq_needs_seq_idx():
@@ -156,7 +154,8 @@ def test_step_entry_points_validate_on_host():
     lib = ssd.lib()
     p = prob()
     assert lib.ssd_chunk_cumsum(ctypes.byref(p), None, FAKE, None) == INVALID
-    assert lib.ssd_chunk_cumsum(ctypes.byref(p), FAKE + 8, FAKE, None) == INVALID
+    assert lib.ssd_chunk_cumsum(ctypes.byref(p), FAKE + 2, FAKE, None) == INVALID  # log a: 4-byte
+    assert lib.ssd_chunk_cumsum(ctypes.byref(p), FAKE, FAKE + 8, None) == INVALID  # cs: 16-byte
     assert lib.ssd_chunk_state(ctypes.byref(p), None, FAKE, FAKE, None, FAKE, None, None) == INVALID
     assert lib.ssd_state_passing(ctypes.byref(p), FAKE, None, FAKE, None, None, None, None) == INVALID
     assert lib.ssd_chunk_scan(ctypes.byref(p), FAKE, FAKE, None, FAKE, None, FAKE, None, None, FAKE,

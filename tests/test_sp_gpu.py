@@ -168,3 +168,37 @@ def test_sp_summary_is_the_state_after_the_last_piece(name):
             assert_close(dec[bb].cpu().numpy().astype(np.float64), dref, 1e-4, f"dec r={r} b={bb}", atol=1e-30)
             want = (0, 0) if row is None else (int(row[a]), int(row[b - 1]))
             assert tuple(ids[bb].tolist()) == want
+
+
+def _draw_sp(i):
+    """Random sequence-parallel problem i: (inputs, segments, dtype, chunk)."""
+    rng = np.random.default_rng(5100 + i)
+    dtype = "bf16" if rng.random() < 0.7 else "f32"
+    b = int(rng.integers(1, 3))
+    T = int(rng.integers(64, 1500))
+    H = int(rng.choice([2, 4, 6]))
+    P = int(rng.choice([32, 64, 64]))
+    N = int(rng.choice([16, 64, 128, 128, 256]))
+    Q = int(rng.choice([64, 128, 256]))
+    R = int(rng.integers(2, 5))
+    cuts = np.sort(rng.choice(np.arange(1, T), size=R - 1, replace=False))
+    seg = np.diff(np.concatenate([[0], cuts, [T]])).astype(int).tolist()
+    lengths = None
+    if rng.random() < 0.6:
+        nseq = int(rng.integers(1, 6))
+        lengths = [np.diff(np.concatenate([[0], np.sort(rng.integers(0, T + 1, size=nseq - 1)), [T]])).astype(int).tolist()
+                   for _ in range(b)]
+    nseq = None if lengths is None else max(len(r) for r in lengths)
+    d = make_custom(b, T, H, P, N, 1, dtype, seed=int(rng.integers(0, 10000)), has_D=str(rng.choice(["none", "normal"])),
+                    has_init=bool(rng.random() < 0.5), lengths=lengths, nseq=nseq)
+    return d, seg, dtype, Q
+
+
+@pytest.mark.parametrize("i", range(12))
+def test_sp_random_problem(i):
+    d, seg, dtype, Q = _draw_sp(i)
+    Y, finals = _run_threads(d, seg, dtype, Q)
+    Yr, Fr = run_oracle(d)
+    assert_close(Y, Yr, TAU[dtype], f"Y (segments {seg})")
+    for r, F in enumerate(finals):
+        assert_close(F, Fr, TAU[dtype], f"final_states on rank {r} (segments {seg})")
