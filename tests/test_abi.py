@@ -3,6 +3,7 @@ include/ssd.h declares, and rejects bad arguments on the host before any
 launch. Calls here use fake device addresses only where a host check is sure to
 reject the call first, so the tests are also safe on a GPU machine."""
 import ctypes
+import os
 
 import pytest
 
@@ -210,3 +211,28 @@ def test_sequence_parallel_entry_points_validate_on_host():
     assert lib.ssd_sp_combine(ctypes.byref(p), 2, 1, FAKE, FAKE, FAKE, None, None, None) == INVALID
     assert lib.ssd_sp_own_finals(ctypes.byref(p), 2, 1, None, FAKE, None) == INVALID
     assert lib.ssd_sp_own_finals(ctypes.byref(p), 2, 1, FAKE, FAKE + 4, None) == INVALID
+
+
+def test_header_is_plain_c_and_a_c_program_links(tmp_path):
+    """include/ssd.h compiles as C99 and a C program links against the library
+    and calls its host-only functions (no device needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "ssd.h"\n'
+        "int main(void) {\n"
+        "    ssd_problem p = {2, 512, 4, 64, 128, 1, 256, 1, SSD_DTYPE_BF16, SSD_PATH_SIMT};\n"
+        '    printf("%s %zu %zu\\n", ssd_status_string(SSD_OK), ssd_fwd_workspace_bytes(&p), ssd_states_bytes(&p));\n'
+        "    return ssd_check_problem(NULL) == SSD_ERR_INVALID_ARG ? 0 : 1;\n}\n")
+    lib_dir = os.path.dirname(ssd.ssd.LIB_PATH)
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"), str(src),
+                    "-o", str(exe), ssd.ssd.LIB_PATH, "-Wl,-rpath," + lib_dir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    align = lambda x: (x + 255) // 256 * 256
+    st = 2 * 2 * 4 * 128 * 64 * 4
+    assert out == ["ok", str(align(2 * 2 * 512 * 4 * 4) + align(st)), str(st)]
