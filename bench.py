@@ -2,7 +2,7 @@
 """Benchmark of the SSD chunked-scan forward on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                [--workload NAME] [--path auto|simt|tcgen05|fused]
+                [--workload NAME] [--path auto|simt|fused]
 
 One step = one ssd_fwd call, the whole forward path over one batch of the
 workload with its inputs resident in HBM: on the fused family (the default
@@ -356,12 +356,9 @@ def run_reference(args, w):
 
 def family(ssd, p, path):
     """Kernel family ssd_fwd runs for problem p under the requested path."""
-    if path in ("simt", "tcgen05", "fused"):
+    if path in ("simt", "fused"):
         return path
-    for f in ("fused", "tcgen05"):
-        if ssd.path_supported(p, f):
-            return f
-    return "simt"
+    return "fused" if ssd.path_supported(p, "fused") else "simt"
 
 
 def workload_config(w, args):
@@ -462,7 +459,7 @@ def run_ours(args, w):
                                                            vp(wloc) if cuts else None, vp(wdec) if cuts else None,
                                                            vp(init), vp(seq), vp(Y), vp(F), sp))
     else:
-        pk = ssd.problem_from(X, B, w.chunk, inputs["nseq"], "tcgen05" if fam == "tcgen05" else "simt")
+        pk = ssd.problem_from(X, B, w.chunk, inputs["nseq"], "simt")
         pr = ctypes.byref(pk)
         nc = -(-T // w.chunk)
         cs = wsp[: b * nc * w.chunk * H * 4].view(torch.float32)
@@ -845,7 +842,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05", "fused"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "fused"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")

@@ -67,7 +67,8 @@ typedef enum {
     SSD_ERR_INVALID_ARG = 1,  /* null required pointer, bad dims, misaligned pointer */
     SSD_ERR_UNSUPPORTED = 2,  /* valid problem this build or device cannot run */
     SSD_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
-    SSD_ERR_CUDA = 4          /* a CUDA call or kernel launch failed */
+    SSD_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
+    SSD_ERR_DEVICE_TIMEOUT = 5  /* ssd_device_error: a kernel's bounded wait gave up */
 } ssd_status;
 
 typedef enum {
@@ -77,19 +78,16 @@ typedef enum {
 
 /* Kernel family.
  *   SIMT     the four steps as fp32 SIMT kernels (any supported shape, fp32 or bf16);
- *   TCGEN05  the four steps with chunk_state and chunk_scan on the tensor cores
- *            (bf16, headdim 64, dstate 64 or 128, chunk 128 or 256, an even
- *            number of heads per group);
- *   FUSED    the two-level path of ssd_segment_state / ssd_segment_passing /
- *            ssd_fused_scan (bf16, headdim 64, dstate 64 or 128, an even number
- *            of heads per group; any chunk): the state stays on chip within a
- *            work range and crosses HBM only where a range boundary cuts a row.
- * AUTO picks FUSED, else TCGEN05, else SIMT, by what the problem allows. An
- * explicit family outside its domain returns SSD_ERR_UNSUPPORTED. */
+ *   FUSED    the two-level tensor-core path of ssd_segment_state /
+ *            ssd_segment_passing / ssd_fused_scan (bf16, headdim 64, dstate a
+ *            multiple of 16 up to 256, an even number of heads per group; any
+ *            chunk): the state stays on chip within a work range and crosses HBM
+ *            only where a range boundary cuts a row.
+ * AUTO picks FUSED where the problem allows it, else SIMT. An explicit family
+ * outside its domain returns SSD_ERR_UNSUPPORTED. (Value 2 is not used.) */
 typedef enum {
     SSD_PATH_AUTO = 0,
     SSD_PATH_SIMT = 1,
-    SSD_PATH_TCGEN05 = 2,
     SSD_PATH_FUSED = 3
 } ssd_path;
 
@@ -114,18 +112,43 @@ const char* ssd_status_string(ssd_status s);
  * ("" if none). */
 const char* ssd_last_cuda_error_string(void);
 
+/*
+ * ssd_device_error: the failure report of the kernels' bounded waits. The
+ * tensor-core kernels wait on shared-memory barriers for their copies and
+ * matrix products; every such wait is bounded (about 2 s), and a wait that
+ * gives up sets a bit in a device-wide 32-bit error word, after which its CTA
+ * runs to its end without hanging or faulting: the outputs of that call are
+ * then INVALID, although the call itself returned SSD_OK (the library does not
+ * synchronise, so the launch cannot see it). The word is per device and shared
+ * by every call and stream since it was last cleared.
+ * This entry point enqueues a read of the word on `stream`, then its clearing,
+ * and SYNCHRONISES `stream` (the one entry point that does). *code (if
+ * code is non-NULL) receives the word: 0, or bit 0 for a barrier wait that
+ * gave up. Returns SSD_OK when the word was 0, SSD_ERR_DEVICE_TIMEOUT when it
+ * was not, SSD_ERR_CUDA if the read failed. The pages have no counterpart.
+ */
+ssd_status ssd_device_error(uint32_t* code, void* stream);
+
+/* ssd_selftest_wait_timeout: checks the report above end to end. Launches one
+ * small kernel whose single wait, limited to limit_ns (1000 .. 10^9, else
+ * SSD_ERR_INVALID_ARG), is on a barrier that nothing completes: the wait gives
+ * up and sets the error word exactly as a production kernel's would, and the
+ * kernel ends normally (no copy or product is in flight). The next
+ * ssd_device_error then returns SSD_ERR_DEVICE_TIMEOUT and clears the word.
+ * Asynchronous on `stream`. The pages have no counterpart. */
+ssd_status ssd_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 /* Host-side validation of a problem (no device access besides querying the
  * current device's compute capability). */
 ssd_status ssd_check_problem(const ssd_problem* p);
 
-/* 1 if `path` (SIMT, TCGEN05 or FUSED) can run problem p on the current device. */
+/* 1 if `path` (SIMT or FUSED) can run problem p on the current device. */
 int ssd_path_supported(const ssd_problem* p, ssd_path path);
 
 /* Bytes of workspace ssd_fwd needs for p, or (size_t)-1 if p is invalid: for
  * the family ssd_fwd runs (p->path, or for AUTO the fused family where it
- * applies, else the chunked ones), the chunked paths' need (the chunk
- * cumulative sums, batch*nchunks*chunk*nheads values, fp64 for the SIMT family
- * and fp32 for the tcgen05 one, and one state per chunk,
+ * applies, else the chunked SIMT one), the chunked need (the chunk cumulative
+ * sums, batch*nchunks*chunk*nheads fp64 values, and one state per chunk,
  * batch*nchunks*nheads*dstate*headdim fp32) or the fused path's (two states and
  * two decays per work range, see ssd_fused_work_tiles, plus the padded slices
  * when dstate is not 64 or 128), each part 256-byte aligned. */

@@ -18,13 +18,16 @@ from .ssd import (  # noqa: F401
     chunk_state,
     decode_step,
     discretize,
+    check_device_error,
     declared_functions,
+    device_error,
     fused_scan,
     fused_scan_chained,
     fused_work_count,
     fused_work_tiles,
     segment_passing,
     segment_state,
+    selftest_wait_timeout,
     sp_combine,
     sp_own_finals,
     sp_summary,

@@ -3,11 +3,39 @@
 // sequence chunk_cumsum -> chunk_state -> state_passing -> chunk_scan on the
 // caller's stream. Nothing here allocates, synchronises or reads device memory.
 
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 
 #include "ssd_common.cuh"
 #include "ssd_tc.cuh"
+
+// The library's device error word: a kernel whose bounded wait gives up ORs a
+// code into it (the output of that call is then invalid). One per device; read
+// and cleared by ssd_device_error.
+__device__ unsigned int g_ssd_device_error = 0u;
+
+namespace ssd {
+
+cudaError_t device_error_word(unsigned int** out) {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<unsigned int*> addr[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    unsigned int* a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
+        void* p = nullptr;
+        if ((e = cudaGetSymbolAddress(&p, g_ssd_device_error)) != cudaSuccess) return e;
+        a = static_cast<unsigned int*>(p);
+        addr[dev].store(a, std::memory_order_release);  // a race only repeats the lookup
+    }
+    *out = a;
+    return cudaSuccess;
+}
+
+}  // namespace ssd
 
 namespace {
 
@@ -29,8 +57,7 @@ ssd_status check_dims(const ssd_problem* p) {
         return SSD_ERR_INVALID_ARG;
     if (p->nheads % p->ngroups != 0) return SSD_ERR_INVALID_ARG;
     if (p->dtype != SSD_DTYPE_F32 && p->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
-    if (p->path != SSD_PATH_AUTO && p->path != SSD_PATH_SIMT && p->path != SSD_PATH_TCGEN05 &&
-        p->path != SSD_PATH_FUSED)
+    if (p->path != SSD_PATH_AUTO && p->path != SSD_PATH_SIMT && p->path != SSD_PATH_FUSED)
         return SSD_ERR_INVALID_ARG;
     if (p->chunk != 64 && p->chunk != 128 && p->chunk != 256) return SSD_ERR_UNSUPPORTED;
     if (p->headdim % 16 != 0 || p->headdim > 256 || p->dstate % 16 != 0 || p->dstate > 256)
@@ -90,29 +117,21 @@ size_t states_bytes(const ssd_problem* p) {
     return (size_t)p->batch * chunk_count(p) * p->nheads * p->dstate * p->headdim * sizeof(float);
 }
 
-// kernels of the chunked steps (chunk_state, chunk_scan)
-bool use_tc(const ssd_problem* p) {
-    if (p->path == SSD_PATH_SIMT) return false;
-    return ssd::tc_supported(p);
-}
-
 // family ssd_fwd runs
 ssd_path fwd_family(const ssd_problem* p) {
     switch (p->path) {
         case SSD_PATH_SIMT: return SSD_PATH_SIMT;
-        case SSD_PATH_TCGEN05: return SSD_PATH_TCGEN05;
         case SSD_PATH_FUSED: return SSD_PATH_FUSED;
         default: break;
     }
     if (ssd::fused_fwd_supported(p)) return SSD_PATH_FUSED;
-    if (ssd::tc_supported(p)) return SSD_PATH_TCGEN05;
     return SSD_PATH_SIMT;
 }
 
-// Workspace of the chunked steps inside ssd_fwd: the cumsum (fp64 for the SIMT
-// kernels, fp32 for the tcgen05 ones) and the chunk states.
-size_t chunked_workspace_bytes(const ssd_problem* p, bool simt) {
-    return align256(cs_elems(p) * (simt ? sizeof(double) : sizeof(float))) + align256(states_bytes(p));
+// Workspace of the chunked steps inside ssd_fwd: the cumsum (fp64: the SIMT
+// kernels take exp(cs_k - cs_l) from it) and the chunk states.
+size_t chunked_workspace_bytes(const ssd_problem* p) {
+    return align256(cs_elems(p) * sizeof(double)) + align256(states_bytes(p));
 }
 
 // The sequence-parallel summary runs segment_state where the fused family's
@@ -124,7 +143,7 @@ bool sp_fused(const ssd_problem* p) {
 
 size_t sp_workspace_bytes(const ssd_problem* p) {
     if (sp_fused(p)) return 0;
-    return chunked_workspace_bytes(p, !use_tc(p)) +
+    return chunked_workspace_bytes(p) +
            align256((size_t)p->batch * p->nseq * p->nheads * p->dstate * p->headdim * sizeof(float));
 }
 
@@ -195,7 +214,6 @@ ssd_status check_common(const ssd_problem* p, const int32_t* seq_idx) {
 ssd_status check_runnable(const ssd_problem* p) {
     ssd_status s = check_device();
     if (s != SSD_OK) return s;
-    if (p->path == SSD_PATH_TCGEN05 && !ssd::tc_supported(p)) return SSD_ERR_UNSUPPORTED;
     if (p->path == SSD_PATH_FUSED && !ssd::fused_fwd_supported(p)) return SSD_ERR_UNSUPPORTED;
     return SSD_OK;
 }
@@ -230,11 +248,29 @@ const char* ssd_status_string(ssd_status s) {
         case SSD_ERR_UNSUPPORTED: return "unsupported problem or device";
         case SSD_ERR_WORKSPACE: return "workspace missing or too small";
         case SSD_ERR_CUDA: return "CUDA error";
+        case SSD_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up (outputs invalid)";
     }
     return "unknown status";
 }
 
 const char* ssd_last_cuda_error_string(void) { return g_cuda_err; }
+
+ssd_status ssd_device_error(uint32_t* code, void* stream) {
+    ssd_status s = check_device();
+    if (s != SSD_OK) return s;
+    unsigned int* word = nullptr;
+    cudaError_t e = ssd::device_error_word(&word);
+    if (e != cudaSuccess) return cuda_status(e);
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned int v = 0u;
+    // the read, then the clear, in stream order; the stream is then drained
+    if ((e = cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaMemsetAsync(word, 0, sizeof(v), st)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
+        return cuda_status(e);
+    if (code) *code = v;
+    return v ? SSD_ERR_DEVICE_TIMEOUT : SSD_OK;
+}
 
 ssd_status ssd_check_problem(const ssd_problem* p) {
     ssd_status s = check_dims(p);
@@ -245,7 +281,6 @@ ssd_status ssd_check_problem(const ssd_problem* p) {
 int ssd_path_supported(const ssd_problem* p, ssd_path path) {
     if (check_dims(p) != SSD_OK || check_device() != SSD_OK) return 0;
     if (path == SSD_PATH_SIMT) return 1;
-    if (path == SSD_PATH_TCGEN05) return ssd::tc_supported(p) ? 1 : 0;
     if (path == SSD_PATH_FUSED) return ssd::fused_fwd_supported(p) ? 1 : 0;
     return 0;
 }
@@ -259,7 +294,7 @@ size_t ssd_fwd_workspace_bytes(const ssd_problem* p) {
     if (check_dims(p) != SSD_OK) return (size_t)-1;
     // the family ssd_fwd runs for p (the same host-side decision)
     const ssd_path fam = fwd_family(p);
-    return fam == SSD_PATH_FUSED ? fused_layout(p).total : chunked_workspace_bytes(p, fam == SSD_PATH_SIMT);
+    return fam == SSD_PATH_FUSED ? fused_layout(p).total : chunked_workspace_bytes(p);
 }
 
 int64_t ssd_fused_work_tiles(const ssd_problem* p) {
@@ -361,24 +396,15 @@ ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_
         const int64_t nt = ((int64_t)p->seqlen + 127) / 128;  // one work range per (batch row, head pair)
         return cuda_status(ssd::launch_segment_state(d, nt, X, log_a, B, seq_idx, loc, dec, st, ids));
     }
-    const bool tc = use_tc(p);
     char* w = static_cast<char*>(workspace);
-    float* states = reinterpret_cast<float*>(w + align256(cs_elems(p) * (tc ? sizeof(float) : sizeof(double))));
-    float* finals = reinterpret_cast<float*>(w + chunked_workspace_bytes(p, !tc));
+    float* states = reinterpret_cast<float*>(w + align256(cs_elems(p) * sizeof(double)));
+    float* finals = reinterpret_cast<float*>(w + chunked_workspace_bytes(p));
+    double* cs = reinterpret_cast<double*>(w);
     cudaError_t e;
-    if (tc) {
-        float* cs = reinterpret_cast<float*>(w);
-        if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
-            (e = ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, finals, st)) != cudaSuccess ||
-            (e = ssd::launch_state_passing(d, cs, states, states, nullptr, seq_idx, finals, st)) != cudaSuccess)
-            return cuda_status(e);
-    } else {
-        double* cs = reinterpret_cast<double*>(w);
-        if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
-            (e = ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, finals, st)) != cudaSuccess ||
-            (e = ssd::launch_state_passing(d, cs, states, states, nullptr, seq_idx, finals, st)) != cudaSuccess)
-            return cuda_status(e);
-    }
+    if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
+        (e = ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, finals, st)) != cudaSuccess ||
+        (e = ssd::launch_state_passing(d, cs, states, states, nullptr, seq_idx, finals, st)) != cudaSuccess)
+        return cuda_status(e);
     return cuda_status(ssd::launch_sp_finish(d, log_a, seq_idx, finals, loc, dec, ids, st));
 }
 
@@ -467,7 +493,6 @@ ssd_status ssd_chunk_state(const ssd_problem* p, const void* X, const void* B, c
     if ((s = check_runnable(p)) != SSD_OK) return s;
     const ssd::Dims d = make_dims(p);
     cudaStream_t st = (cudaStream_t)stream;
-    if (use_tc(p)) return cuda_status(ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, final_states, st));
     return cuda_status(ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st));
 }
 
@@ -494,8 +519,6 @@ ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, co
     if ((s = check_runnable(p)) != SSD_OK) return s;
     const ssd::Dims d = make_dims(p);
     cudaStream_t st = (cudaStream_t)stream;
-    if (use_tc(p))
-        return cuda_status(ssd::launch_chunk_scan_tc(d, X, B, C, cs, D, incoming, init_states, seq_idx, Y, st));
     return cuda_status(
         ssd::launch_chunk_scan_simt(d, p->dtype, X, B, C, cs, D, incoming, init_states, seq_idx, Y, st));
 }
@@ -549,21 +572,11 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
         }
         return cuda_status(e);
     }
-    const bool tc = (fam == SSD_PATH_TCGEN05);
     char* w = static_cast<char*>(workspace);
-    float* states = reinterpret_cast<float*>(w + align256(cs_elems(p) * (tc ? sizeof(float) : sizeof(double))));
+    float* states = reinterpret_cast<float*>(w + align256(cs_elems(p) * sizeof(double)));
     cudaError_t e;
-    if (tc) {
-        float* cs = reinterpret_cast<float*>(w);
-        if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
-            (e = ssd::launch_chunk_state_tc(d, X, B, cs, seq_idx, states, final_states, st)) != cudaSuccess ||
-            // in place: the chunk states become the incoming states
-            (e = ssd::launch_state_passing(d, cs, states, states, init_states, seq_idx, final_states, st)) !=
-                cudaSuccess)
-            return cuda_status(e);
-        return cuda_status(ssd::launch_chunk_scan_tc(d, X, B, C, cs, D, states, init_states, seq_idx, Y, st));
-    }
-    // the SIMT kernels take the cumsum in fp64 (fp32 parity for strongly decaying heads)
+    // the SIMT kernels take the cumsum in fp64 (fp32 parity for strongly decaying heads);
+    // state_passing works in place: the chunk states become the incoming states
     double* cs = reinterpret_cast<double*>(w);
     if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
         (e = ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st)) !=

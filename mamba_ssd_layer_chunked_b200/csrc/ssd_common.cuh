@@ -102,4 +102,9 @@ cudaError_t launch_chunk_scan_simt(const Dims& d, ssd_dtype dt, const void* X, c
 // Sets cudaFuncAttributeMaxDynamicSharedMemorySize once per (kernel, device).
 cudaError_t ensure_smem_attr(const void* func, int bytes, int slot);
 
+// Device address of the library's error word on the current device (looked up
+// once per device): kernels with bounded waits OR a code into it when a wait
+// gives up; ssd_device_error reads and clears it.
+cudaError_t device_error_word(unsigned int** out);
+
 }  // namespace ssd

@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     segment_state_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b, Dims d,
                          Work wk, const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
                          float* __restrict__ work_local, float* __restrict__ work_decay, int whole_rows,
-                         int32_t* __restrict__ row_ids) {
+                         int32_t* __restrict__ row_ids, unsigned int* __restrict__ err) {
     constexpr uint32_t kXB = 2 * kBox, kBB = (N / 64) * kBox, kStage = kXB + kBB;
     // three stages: tile it scaled, tile it - 1 multiplied, tile it + 1 loading
     constexpr int kStages = 3;
@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     __shared__ __align__(8) uint64_t bar_load[kStages], bar_mma[kStages], bar_scaled[kStages];
     __shared__ uint32_t tmem_base;
 
+    wait_guard_init(err);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the scan that follows may start its setup and first tile now: it waits
     // for this grid before it reads the range states
@@ -473,7 +474,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                       const float* __restrict__ work_in, const float* __restrict__ init_states,
                       const int32_t* __restrict__ seq_idx, __nv_bfloat16* __restrict__ Y,
                       float* __restrict__ final_states, const float* __restrict__ work_local,
-                      const float* __restrict__ work_decay) {
+                      const float* __restrict__ work_decay, unsigned int* __restrict__ err) {
     using S = FusedSmem<N>;
     constexpr int NQ = N / 4;  // state columns per thread
     extern __shared__ uint8_t smem_raw[];
@@ -493,6 +494,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         bar_st, bar_free, bar_csfull[kCsBufs], bar_csfree[kCsBufs];
     __shared__ uint32_t tmem_base;
 
+    wait_guard_init(err);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int i_work = blockIdx.x;
 
@@ -1281,6 +1283,8 @@ cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* 
                                  int32_t* row_ids) {
     CUtensorMap mx, mb;
     cudaError_t e;
+    unsigned int* err = nullptr;
+    if ((e = device_error_word(&err)) != cudaSuccess) return e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
     if ((e = bc_map(&mb, d, B, 128)) != cudaSuccess) return e;
     const Work w = make_work(d, work_tiles);
@@ -1290,12 +1294,12 @@ cudaError_t launch_segment_state(const Dims& d, int64_t work_tiles, const void* 
         auto k = segment_state_kernel<64>;
         if ((e = set_smem_attr(k, smem, 30)) != cudaSuccess) return e;
         k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay, row_ids != nullptr,
-                                           row_ids);
+                                           row_ids, err);
     } else if (d.dstate == 128) {
         auto k = segment_state_kernel<128>;
         if ((e = set_smem_attr(k, smem, 31)) != cudaSuccess) return e;
         k<<<grid, kSegThreads, smem, st>>>(mx, mb, d, w, log_a, seq_idx, work_local, work_decay, row_ids != nullptr,
-                                           row_ids);
+                                           row_ids, err);
     } else {
         return cudaErrorNotSupported;
     }
@@ -1318,6 +1322,8 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
     if (Yacc && Yacc != Y) return cudaErrorInvalidValue;  // the slices accumulate in place
     CUtensorMap mx, mb, mc, my;
     cudaError_t e;
+    unsigned int* err = nullptr;
+    if ((e = device_error_word(&err)) != cudaSuccess) return e;
     if ((e = x_map(&mx, d, X, 128)) != cudaSuccess) return e;
     if ((e = bc_map(&mb, d, B, 128)) != cudaSuccess) return e;
     if ((e = bc_map(&mc, d, C, 128)) != cudaSuccess) return e;
@@ -1342,13 +1348,13 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
         cfg.dynamicSmemBytes = fused_smem_bytes<64>();
         if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, Yacc ? 34 : 32)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
-                               final_states, work_local, work_decay);
+                               final_states, work_local, work_decay, err);
     } else if (d.dstate == 128) {
         auto k = Yacc ? fused_scan_kernel<128, true> : fused_scan_kernel<128, false>;
         cfg.dynamicSmemBytes = fused_smem_bytes<128>();
         if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, Yacc ? 35 : 33)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
-                               final_states, work_local, work_decay);
+                               final_states, work_local, work_decay, err);
     } else {
         return cudaErrorNotSupported;
     }

@@ -1,5 +1,6 @@
-// ssd_tc.cuh -- tensor-core (tcgen05 / TMEM / TMA) kernels of the SSD chunked
-// scan for sm_100a: chunk_state and chunk_scan. Internal, not part of the C ABI.
+// ssd_tc.cuh -- the tensor-core (tcgen05 / TMEM / TMA) kernels of the SSD
+// forward for sm_100a: the fused path's launchers and the TMA tensor maps they
+// use. Internal, not part of the C ABI.
 #pragma once
 
 #include <cuda.h>
@@ -8,21 +9,9 @@
 
 namespace ssd {
 
-// TMA tensor maps (bf16, 128-byte swizzle, boxes of 64 x 1 x box_tok x 1)
+// TMA tensor maps (ssd_tmap.cu; bf16, 128-byte swizzle, boxes of 64 x 1 x box_tok x 1)
 cudaError_t x_map(CUtensorMap* m, const Dims& d, const void* X, uint32_t box_tok);
 cudaError_t bc_map(CUtensorMap* m, const Dims& d, const void* Bp, uint32_t box_tok);
-
-// True when the tcgen05 kernels cover problem p (dtype, head/state sizes, chunk).
-bool tc_supported(const ssd_problem* p);
-
-cudaError_t launch_chunk_state_tc(const Dims& d, const void* X, const void* B, const float* cs,
-                                  const int32_t* seq_idx, float* states, float* final_states,
-                                  cudaStream_t st);
-
-cudaError_t launch_chunk_scan_tc(const Dims& d, const void* X, const void* B, const void* C,
-                                 const float* cs, const float* D, const float* incoming,
-                                 const float* init_states, const int32_t* seq_idx, void* Y,
-                                 cudaStream_t st);
 
 // ---- fused path (ssd_fused.cu) ----
 // The rows (batch row, head pair) x 128-token tiles laid end to end, cut into

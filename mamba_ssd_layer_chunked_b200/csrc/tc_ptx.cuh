@@ -12,13 +12,34 @@ namespace ssd {
 namespace tc {
 
 // ---------------------------------------------------------------------------
-// error word: a wait that gives up records a code here and the kernel carries
-// on to its end (no trap, no hang). One copy per translation unit that
-// includes this header (only the tensor-core kernels do).
+// Bounded waits and their error report. Every kernel that waits on an
+// mbarrier calls wait_guard_init(err) on entry, before its first
+// __syncthreads, with err the library's device error word (one 32-bit word per
+// device, read and cleared by ssd_device_error on the host). A wait that gives
+// up ORs its code into that word, marks its CTA, and returns false; the kernel
+// then runs to its end without trapping or hanging, and its output is invalid.
+// Later waits of the same CTA give up at once, so a CTA that lost its schedule
+// still ends within one wait limit; the mark lives in shared memory, so it ends
+// with the launch and never touches later launches.
 // ---------------------------------------------------------------------------
-static __device__ unsigned int g_tc_error = 0;
+enum : unsigned { kErrBarrierTimeout = 1u };
 
-enum : unsigned { kErrBarrierTimeout = 1u, kErrTmaStoreTimeout = 2u };
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // ~2 s per wait
+
+static __shared__ unsigned int* s_wait_err;    // the device error word (may be null)
+static __shared__ unsigned int s_wait_gave_up;  // a wait of this CTA gave up
+
+__device__ __forceinline__ void wait_guard_init(unsigned int* err) {
+    if (threadIdx.x == 0) {
+        s_wait_err = err;
+        s_wait_gave_up = 0u;
+    }
+}
+
+__device__ __forceinline__ void wait_report(unsigned int code) {
+    s_wait_gave_up = 1u;
+    if (s_wait_err) atomicOr(s_wait_err, code);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -58,19 +79,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete, for at most ~2 s.
-// On timeout: record the error and return false (the caller carries on to the
-// end of the kernel). Once any wait has timed out, later waits give up at
-// once, so a kernel that lost its schedule still ends within seconds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete, for at most limit_ns
+// (by %globaltimer). On timeout: report it (see wait_guard_init) and return
+// false; the caller carries on to the end of the kernel.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0u) {  // the clock and the error word are read rarely
-            if (*reinterpret_cast<volatile unsigned int*>(&g_tc_error) != 0u) return false;
-            if (globaltimer_ns() - t0 > 2000000000ull) {
-                atomicOr(&g_tc_error, kErrBarrierTimeout);
+        if ((it & 63u) == 0u) {  // the clock and the CTA's mark are read rarely
+            if (*reinterpret_cast<volatile unsigned int*>(&s_wait_gave_up) != 0u) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                wait_report(kErrBarrierTimeout);
                 return false;
             }
         }

@@ -20,9 +20,9 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libssd_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "ssd.h")
 
-SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA = range(5)
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA, SSD_ERR_DEVICE_TIMEOUT = range(6)
 SSD_DTYPE_F32, SSD_DTYPE_BF16 = 0, 1
-PATHS = {"auto": 0, "simt": 1, "tcgen05": 2, "fused": 3}
+PATHS = {"auto": 0, "simt": 1, "fused": 3}
 
 
 class SSDError(RuntimeError):
@@ -73,6 +73,8 @@ def _declare(lib):
         "ssd_sp_summary_workspace_bytes": ([P], ctypes.c_size_t),
         "ssd_sp_combine": ([P, ctypes.c_int, ctypes.c_int] + [vp] * 6, ctypes.c_int),
         "ssd_sp_own_finals": ([P, ctypes.c_int, ctypes.c_int, vp, vp, vp], ctypes.c_int),
+        "ssd_device_error": ([ctypes.POINTER(ctypes.c_uint32), vp], ctypes.c_int),
+        "ssd_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
     }
     for name, (argtypes, restype) in sig.items():
         f = getattr(lib, name)
@@ -157,6 +159,29 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream) -> ctypes.c_void_p:
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def device_error(stream=None) -> int:
+    """Read and clear the library's device error word (synchronises `stream`):
+    0 when no bounded wait of a kernel has given up since the last read; else
+    the word's bits (the outputs of the calls since then are invalid)."""
+    code = ctypes.c_uint32(0)
+    st = lib().ssd_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (SSD_OK, SSD_ERR_DEVICE_TIMEOUT):
+        _check(st, "ssd_device_error")
+    return int(code.value)
+
+
+def check_device_error(stream=None):
+    """Raise SSDError when a kernel's bounded wait gave up since the last read."""
+    code = device_error(stream)
+    if code:
+        raise SSDError(SSD_ERR_DEVICE_TIMEOUT, "ssd_device_error", f"error word 0x{code:x}")
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None):
+    """Launch the self-test kernel whose one wait gives up after limit_ns."""
+    _check(lib().ssd_selftest_wait_timeout(int(limit_ns), _stream(stream)), "ssd_selftest_wait_timeout")
 
 
 def _check_shapes(X, log_a, B, C, D, init_states, seq_idx, nseq):

@@ -29,6 +29,7 @@ def run_gpu(d, dtype, chunk, path="auto"):
                            seq_idx=g["seq_idx"], nseq=g["nseq"] if g["seq_idx"] is not None else None,
                            path=path)
     torch.cuda.synchronize()
+    ssd.check_device_error()  # no bounded wait of any kernel gave up
     return Y.float().cpu().numpy().astype(np.float64), final.cpu().numpy().astype(np.float64)
 
 

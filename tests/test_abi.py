@@ -30,7 +30,8 @@ def test_library_exports_every_declared_function():
     assert set(names) >= {"ssd_status_string", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
                           "ssd_chunk_scan", "ssd_check_problem", "ssd_path_supported", "ssd_states_bytes",
                           "ssd_last_cuda_error_string", "ssd_segment_state", "ssd_segment_passing",
-                          "ssd_fused_scan", "ssd_fused_work_tiles", "ssd_fused_work_count"}
+                          "ssd_fused_scan", "ssd_fused_work_tiles", "ssd_fused_work_count", "ssd_device_error",
+                          "ssd_selftest_wait_timeout"}
 
 
 def test_problem_struct_layout():
@@ -38,7 +39,8 @@ def test_problem_struct_layout():
 
 
 def test_status_strings():
-    for s, text in [(OK, "ok"), (INVALID, "invalid argument"), (WORKSPACE, "workspace missing or too small")]:
+    for s, text in [(OK, "ok"), (INVALID, "invalid argument"), (WORKSPACE, "workspace missing or too small"),
+                    (5, "a device-side wait gave up (outputs invalid)")]:
         assert ssd.status_string(s) == text
     assert ssd.status_string(99) == "unknown status"
 
@@ -46,7 +48,7 @@ def test_status_strings():
 def test_workspace_bytes_formula():
     p = prob()
     align = lambda x: (x + 255) // 256 * 256
-    cs = 2 * 512 * 4 * 4  # fp32 cumsum (the tcgen05 family); the SIMT family keeps it in fp64
+    cs = 2 * 512 * 4 * 4  # cumsum values x 4 bytes; the SIMT family keeps them in fp64 (x 2)
     st = 2 * (512 // 256) * 4 * 128 * 64 * 4
     # fused: rows (batch, head pair) = 4, 4 tiles each; ranges of wt tiles
     wt = ssd.fused_work_tiles(p)
@@ -57,7 +59,9 @@ def test_workspace_bytes_formula():
     fused = 2 * align(nwork * 2 * 128 * 64 * 4) + align(nwork * 2 * 4)
     assert ssd.workspace_bytes(p) == fused  # AUTO runs the fused family for this problem
     assert ssd.workspace_bytes(prob(path=1)) == align(2 * cs) + align(st)  # the SIMT family: the chunked need
-    assert ssd.workspace_bytes(prob(path=2)) == align(cs) + align(st)  # the chunked tcgen05 family
+    # value 2 of ssd_path (the retired chunked tensor-core family) is not a path
+    assert ssd.lib().ssd_fwd_workspace_bytes(ctypes.byref(prob(path=2))) == ctypes.c_size_t(-1).value
+    assert ssd.lib().ssd_check_problem(ctypes.byref(prob(path=2))) == INVALID
     assert ssd.states_bytes(p) == st
     # outside the fused domain (fp32) only the chunked need counts
     q = prob(dtype=ssd.ssd.SSD_DTYPE_F32)
@@ -131,13 +135,12 @@ def test_sp_summary_workspace_formula():
     size = lambda q: lib.ssd_sp_summary_workspace_bytes(ctypes.byref(q))
     # segment_state covers bf16, P 64, N 64 or 128: no workspace
     assert size(prob()) == 0 and size(prob(dstate=64)) == 0
-    # the chunked steps: cumsum (fp64 for the SIMT kernels, fp32 for the tcgen05 ones),
-    # chunk states, final states from zero
+    # the chunked steps: cumsum (fp64), chunk states, final states from zero
     for q, (b, T, H, P, N, Q, S, csb) in ((prob(dtype=ssd.ssd.SSD_DTYPE_F32, headdim=16, dstate=16, chunk=64),
                                            (2, 512, 4, 16, 16, 64, 1, 8)),
                                           (prob(dstate=256), (2, 512, 4, 64, 256, 256, 1, 8)),
                                           (prob(seqlen=500, nseq=3, path=1), (2, 500, 4, 64, 128, 256, 3, 8)),
-                                          (prob(path=2), (2, 512, 4, 64, 128, 256, 1, 4))):
+                                          (prob(path=1), (2, 512, 4, 64, 128, 256, 1, 8))):
         nc = -(-T // Q)
         want = align(b * nc * Q * H * csb) + align(b * nc * H * N * P * 4) + align(b * S * H * N * P * 4)
         assert size(q) == want

@@ -57,7 +57,7 @@ def test_random_problem_every_family(i):
     p = ssd.make_problem(X.shape[0], X.shape[1], X.shape[2], X.shape[3], d["B"].shape[3], d["B"].shape[2], Q,
                          d["nseq"], torch.bfloat16 if dtype == "bf16" else torch.float32)
     ran = 0
-    for path in ("auto", "simt", "tcgen05", "fused"):
+    for path in ("auto", "simt", "fused"):
         if path != "auto" and not ssd.path_supported(p, path):
             continue
         Y, F = run_gpu(d, dtype, Q, path)
@@ -104,7 +104,7 @@ def test_random_large_problem_fused_and_chunked(i):
     p = ssd.make_problem(X.shape[0], X.shape[1], X.shape[2], 64, d["B"].shape[3], d["B"].shape[2], Q, d["nseq"],
                          torch.bfloat16)
     assert ssd.path_supported(p, "fused")
-    for path in ("auto", "fused", "tcgen05"):
+    for path in ("auto", "fused"):
         if not ssd.path_supported(p, path) and path != "auto":
             continue
         Y, F = run_gpu(d, "bf16", Q, path)
