@@ -45,11 +45,14 @@ DEFAULT_WORKLOAD = "mamba2_2p7b_layer"
 # Algorithmic work (the per-unit figures of the design notes)
 # --------------------------------------------------------------------------- #
 
-def algorithmic_flops(w) -> float:
+def algorithmic_flops(w, q=None) -> float:
     """F = b * C_n * [H (Q(Q+1) P + 4 Q N P) + G Q(Q+1) N]: the masked quadratic
-    term and C B^T on the lower triangle, the chunk state and the state read-out."""
-    cn = w.seqlen // w.chunk
-    Q, N, P = w.chunk, w.dstate, w.headdim
+    term and C B^T on the lower triangle, the chunk state and the state read-out,
+    at the workload's chunk Q (the primary count) or at block length q (the
+    fused kernels work in 128-token tiles, whose masked work is that of q = 128)."""
+    Q = w.chunk if q is None else q
+    cn = w.seqlen / Q
+    N, P = w.dstate, w.headdim
     return w.batch * cn * (w.nheads * (Q * (Q + 1) * P + 4 * Q * N * P) + w.ngroups * Q * (Q + 1) * N)
 
 
@@ -113,10 +116,11 @@ def kernel_model(w, wt=None):
       segment_passing (the step entry point; ssd_fwd folds it into fused_scan)
                       reads those states and decays, writes one incoming state
                       per range start inside a row and head; 2 N P flops each.
-      fused_scan      reads X, B, C, log a, D, the states and decays of the pieces
-                      before its cut (one piece per cut at the bench shapes) and
-                      the initial states; writes Y and the final states; per
-                      (b, tile, h) 128*129 P + 4*128 N P flops, per (b, tile, g) 128*129 N.
+      fused_scan      reads X, B, C, log a, D and the initial states; writes Y
+                      and the final states (the algorithmic bytes: the range
+                      states it also reads at each cut are a state spill, which
+                      the count leaves out); per (b, tile, h) 128*129 P +
+                      4*128 N P flops, per (b, tile, g) 128*129 N.
     """
     e = _esize(w)
     b, T, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
@@ -144,30 +148,31 @@ def kernel_model(w, wt=None):
             "segment_state": dict(bytes=walked * (P * e + 4) + cut_tokens * N * e + ncuts * (st2 + 8),
                                   flops=walked * 2 * N * P),
             "segment_passing": dict(bytes=ncuts * (2 * st2 + 8), flops=ncuts * 2 * 2 * N * P),
-            "fused_scan": dict(bytes=2 * xb + 2 * bcb + csb + ncuts * st2 + init + fin,
+            "fused_scan": dict(bytes=2 * xb + 2 * bcb + csb + (H * 4 if w.has_D != "none" else 0) + init + fin,
                                flops=b * ntile * (H * (128 * 129 * P + 4 * 128 * N * P) + G * 128 * 129 * N)),
         })
     return out
 
 
 def profiled_traffic(kernel):
-    """dram bytes read + written per launch of `kernel` from the committed ncu
-    summary of the fused path, or None when that summary was taken on another
-    version of the kernel source (or covers no such kernel)."""
+    """dram bytes read + written per launch of `kernel`, from the committed ncu
+    summary of the fused path (profiles/fused_path_mamba2_2p7b_layer.json), or
+    None when that capture was taken on another version of the kernel source
+    (or covers no such kernel)."""
     import hashlib
-    import re
-    prof = os.path.join(ROOT, "profiles", "fused_path_mamba2_2p7b_layer.md")
-    src = os.path.join(ROOT, "mamba_ssd_layer_chunked_b200", "csrc", "ssd_fused.cu")
-    if not (os.path.exists(prof) and os.path.exists(src)):
+    prof = os.path.join(ROOT, "profiles", "fused_path_mamba2_2p7b_layer.json")
+    if not os.path.exists(prof):
         return None
-    text = open(prof).read()
-    m = re.search(r"sha256 prefix `([0-9a-f]+)`", text)
+    with open(prof) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, rec.get("kernel_source", ""))
+    if not os.path.isfile(src):
+        return None
     with open(src, "rb") as f:
-        if not m or hashlib.sha256(f.read()).hexdigest()[: len(m.group(1))] != m.group(1):
+        if hashlib.sha256(f.read()).hexdigest()[: len(rec["sha256_prefix"])] != rec["sha256_prefix"]:
             return None
-    m = re.search(r"dram_bytes_per_launch (.*)", text)
-    vals = dict(kv.split("=") for kv in m.group(1).split()) if m else {}
-    return int(vals[kernel]) if kernel in vals else None
+    v = rec.get("dram_bytes_per_launch", {}).get(kernel)
+    return int(v) if v is not None else None
 
 
 def load_peaks():
@@ -288,11 +293,12 @@ def cpu_model() -> str:
     return platform.processor() or platform.machine()
 
 
-def oracle_sample(w, inputs, budget_s: float = 12.0, threads: int = 0):
+def oracle_sample(w, inputs, budget_s: float = 12.0, threads: int = 0, outputs=None):
     """Time the oracle on whole (batch row, head) pairs of the workload, one
     batch row and `cores` heads per call (cores = threads, or every host core
     when threads is 0), until about budget_s seconds of CPU work or the whole
-    workload; return (token·heads/s, cores, sample, seconds)."""
+    workload; return (token·heads/s, cores, sample, seconds). With `outputs` (a
+    list), each call's (batch row, heads, Y) is appended to it."""
     import oracle
     cores = threads if threads > 0 else max(1, oracle.max_threads())
     done, t_total = 0, 0.0
@@ -309,9 +315,11 @@ def oracle_sample(w, inputs, budget_s: float = 12.0, threads: int = 0):
             if w.ngroups != 1:
                 raise NotImplementedError("oracle sampling assumes one group")
             t0 = time.perf_counter()
-            oracle.ssd_reference(X, la, inputs["B"][b:b + 1], inputs["C"][b:b + 1], D, init, seq,
-                                 nseq=inputs["nseq"], nthreads=cores)
+            Yr, _ = oracle.ssd_reference(X, la, inputs["B"][b:b + 1], inputs["C"][b:b + 1], D, init, seq,
+                                         nseq=inputs["nseq"], nthreads=cores)
             t_total += time.perf_counter() - t0
+            if outputs is not None:
+                outputs.append((b, hs, Yr))
             done += X.shape[2]
     return done * w.seqlen / t_total, cores, f"{done} (batch row, head) pairs x {w.seqlen} tokens of {w.name}", t_total
 
@@ -420,14 +428,16 @@ def run_ours(args, w):
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs_step = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     barrier()
-    ev0.record(stream)
-    for _ in range(args.steps):
+    evs_step[0].record(stream)
+    for i in range(args.steps):
         step()
-    ev1.record(stream)
+        evs_step[i + 1].record(stream)
     barrier()
-    t_dev = ev0.elapsed_time(ev1) / 1e3
+    t_dev = evs_step[0].elapsed_time(evs_step[-1]) / 1e3
+    step_ms = sorted(evs_step[i].elapsed_time(evs_step[i + 1]) for i in range(args.steps))
+    pct = lambda q: step_ms[min(len(step_ms) - 1, int(round(q * (len(step_ms) - 1))))]
     units = w.tokens_heads * args.steps
     value, t_max = aggregate(units, t_dev, dev if ws > 1 else None)
     ms_per_step = t_max / args.steps * 1e3
@@ -567,6 +577,12 @@ def run_ours(args, w):
         "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, args),
         "tflops": flops * ws / step_s / 1e12,
         "pct_bf16_peak": flops / step_s / 1e12 / peaks["bf16_tflops"],
+        "tflops_note": "algorithmic count at the workload's chunk Q; tflops_at_tile128 counts the masked work "
+                       "of the 128-token tiles the fused kernels compute in",
+        "tflops_at_tile128": algorithmic_flops(w, 128) * ws / step_s / 1e12,
+        "pct_bf16_peak_at_tile128": algorithmic_flops(w, 128) / step_s / 1e12 / peaks["bf16_tflops"],
+        "step_ms": {"median": statistics.median(step_ms), "p10": pct(0.1), "p90": pct(0.9),
+                    "note": "rank 0, CUDA events between consecutive steps"},
         "pct_hbm": algorithmic_bytes(w) / step_s / 1e9 / peaks["hbm_gbs"],
         "path": fam,
         "work_tiles": wt,
@@ -577,8 +593,18 @@ def run_ours(args, w):
         "gpu_launches": len(launches) * args.steps,
         "clocks": clk,
     }
+    result["parity"] = None
     if rank == 0 and not args.no_cpu_baseline:
-        v, cores, sample, secs = oracle_sample(w, inputs, budget_s=args.cpu_budget)
+        outs = []
+        v, cores, sample, secs = oracle_sample(w, inputs, budget_s=args.cpu_budget, outputs=outs)
+        # parity of the timed output on the rows the oracle computed: max|dY| / max|Y_ref|
+        err = scale = 0.0
+        for b_, hs, Yr in outs:
+            Yg = Y[b_:b_ + 1, :, hs].float().cpu().numpy().astype(np.float64)
+            err = max(err, float(np.max(np.abs(Yg - Yr))))
+            scale = max(scale, float(np.max(np.abs(Yr))))
+        result["parity"] = {"max_abs_err_over_max_abs_y": err / scale if scale else 0.0,
+                            "tau": 2e-2 if w.dtype == "bf16" else 1e-5, "rows": sample}
         v1, _, sample1, secs1 = oracle_sample(w, inputs, budget_s=max(1.0, args.cpu_budget / 4), threads=1)
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                                   "seconds": secs, "cpu_model": cpu_model(),

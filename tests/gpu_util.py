@@ -52,16 +52,3 @@ def assert_close(got, ref, tau, what, atol=0.0):
     err, scale = rel_err(got, ref)
     assert err <= tau * scale + atol, f"{what}: max|d| = {err:.3e} > {tau:g} * max|ref| + {atol:g} = {tau * scale + atol:.3e}"
     return err / scale if scale else 0.0
-
-
-def slice_heads(d, b, h):
-    """Inputs of one (batch row, head) pair, for sampled oracle checks."""
-    H = d["X"].shape[2]
-    G = d["B"].shape[2]
-    g = h // (H // G)
-    out = dict(X=d["X"][b:b + 1, :, h:h + 1], log_a=d["log_a"][b:b + 1, :, h:h + 1],
-               B=d["B"][b:b + 1, :, g:g + 1], C=d["C"][b:b + 1, :, g:g + 1],
-               D=None if d["D"] is None else d["D"][h:h + 1],
-               init_states=None if d["init_states"] is None else d["init_states"][b:b + 1, :, h:h + 1],
-               seq_idx=None if d["seq_idx"] is None else d["seq_idx"][b:b + 1], nseq=d["nseq"])
-    return out

@@ -281,6 +281,105 @@ def test_chunk_states_with_resets():
             np.testing.assert_allclose(loc[b, c], f[0, 0], rtol=1e-12, atol=1e-13)
 
 
+def test_chunk_states_and_block_decay_on_the_chunk_split_example(golden):
+    """The page's split after step 2, with no padding: the second block is a
+    short last block of one token. Its incoming state is the first block's end
+    state, its zero-start local end state is its own output (C = 1, N = P = 1),
+    its block decay is the product of its a_t, and decay * incoming + local is
+    the last output (the block scan of the same page)."""
+    g = golden("worked_example_a05.txt")
+    q, a = int(g["split_after"][0]), g["a"][0]
+    X, la, B, C = scalar_inputs(g["x"], a=a)
+    inc, loc = oracle.chunk_states(X, la, B, chunk=q)
+    assert inc.shape[1] == 2  # ceil(3 / 2) blocks, the last one short
+    assert inc[0, 0].item() == 0.0
+    assert abs(inc[0, 1].item() - g["first_block_end_state"][0]) < 1e-12
+    assert abs(loc[0, 0].item() - g["first_block_end_state"][0]) < 1e-12
+    assert abs(loc[0, 1].item() - g["second_block_local_output"][0]) < 1e-12
+    dec = oracle.segment_decay(la, q)
+    assert abs(dec[0, 0, 0] - a * a) < 1e-15          # product of the first block's two a_t
+    assert abs(dec[0, 1, 0] - a) < 1e-15              # the short block holds one a_t
+    # the carried contribution and the scan step of the page
+    assert abs(dec[0, 1, 0] * inc[0, 1].item() - g["second_block_incoming_output"][0]) < 1e-12
+    assert abs(dec[0, 1, 0] * inc[0, 1].item() + loc[0, 1].item() - g["y"][-1]) < 1e-12
+
+
+def _last_piece_start(seq_row, t0, t1):
+    """First token of the last sequence piece of the block [t0, t1)."""
+    p0 = t1 - 1
+    while p0 > t0 and seq_row[p0 - 1] == seq_row[t1 - 1]:
+        p0 -= 1
+    return p0
+
+
+RAGGED = [(4, [[3, 9, 1, 3, 3], [19]]), (8, [[5, 6, 2, 6], [10, 9]]), (8, [[19], [17, 1, 1]])]
+
+
+@pytest.mark.parametrize("Q,lens", RAGGED)
+def test_chunk_states_ragged_last_chunk_against_recurrence_on_slices(Q, lens):
+    """T = 19 is not a multiple of Q: the last block is short. Every block's
+    incoming and local states equal the step recurrence run on row slices: from
+    the sequence's start (with its initial state) to the block start, and from
+    zero over the block's last sequence piece."""
+    nseq = max(len(r) for r in lens)
+    d = make_custom(2, 19, 2, 3, 4, dtype="f32", seed=50 + Q, has_init=True, lengths=lens, nseq=nseq)
+    inc, loc = oracle.chunk_states(d["X"], d["log_a"], d["B"], Q, d["init_states"], d["seq_idx"], nseq=nseq)
+    seq = d["seq_idx"]
+    nch = -(-19 // Q)
+    assert inc.shape[1] == nch and 19 % Q != 0
+    sl_args = lambda b, sl, init=None: (d["X"][b:b + 1, sl], d["log_a"][b:b + 1, sl], d["B"][b:b + 1, sl],
+                                        d["C"][b:b + 1, sl], None, init)
+    for b in range(2):
+        for c in range(nch):
+            t0, t1 = c * Q, min(19, (c + 1) * Q)
+            s0 = seq[b, t0]
+            start = t0
+            while start > 0 and seq[b, start - 1] == s0:
+                start -= 1
+            if t0 > start:
+                _, f = oracle.ssd_reference(*sl_args(b, slice(start, t0), d["init_states"][b:b + 1, s0:s0 + 1]))
+                np.testing.assert_allclose(inc[b, c], f[0, 0], rtol=1e-12, atol=1e-13)
+            else:
+                np.testing.assert_array_equal(inc[b, c], d["init_states"][b, s0])
+            p0 = _last_piece_start(seq[b], t0, t1)
+            _, f = oracle.ssd_reference(*sl_args(b, slice(p0, t1)))
+            np.testing.assert_allclose(loc[b, c], f[0, 0], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("Q,lens", RAGGED)
+def test_segment_decay_is_the_product_over_the_last_piece(Q, lens):
+    """The block decay of the page's block scan for blocks that may hold a
+    sequence start and may be short: (a) the explicit product of a_t over the
+    block's last sequence piece; (b) the factor the step recurrence applies to
+    a state carried into that piece (no input, initial state of ones); and a
+    piece start off by one either way fails both."""
+    nseq = max(len(r) for r in lens)
+    d = make_custom(2, 19, 3, 2, 2, dtype="f32", seed=60 + Q, lengths=lens, nseq=nseq)
+    la, seq = d["log_a"].astype(np.float64), d["seq_idx"]
+    dec = oracle.segment_decay(la, Q, seq)
+    nch = -(-19 // Q)
+    assert dec.shape == (2, nch, 3)
+    for b in range(2):
+        for c in range(nch):
+            t0, t1 = c * Q, min(19, (c + 1) * Q)
+            p0 = _last_piece_start(seq[b], t0, t1)
+            for h in range(3):
+                prod = 1.0
+                for t in range(p0, t1):
+                    prod *= math.exp(la[b, t, h])
+                assert abs(dec[b, c, h] - prod) <= 1e-14 * prod
+                # off-by-one piece starts give other values
+                for q0 in (p0 - 1, p0 + 1):
+                    if t0 <= q0 < t1 and q0 != p0:
+                        wrong = math.prod(math.exp(la[b, t, h]) for t in range(q0, t1))
+                        assert abs(wrong - dec[b, c, h]) > 1e-6 * dec[b, c, h]
+            sl = slice(p0, t1)
+            zeros = np.zeros_like(d["X"][b:b + 1, sl])
+            ones = np.ones((1, 1, 3, 2, 2))
+            _, f = oracle.ssd_reference(zeros, la[b:b + 1, sl], d["B"][b:b + 1, sl], d["C"][b:b + 1, sl], None, ones)
+            np.testing.assert_allclose(f[0, 0, :, 0, 0], dec[b, c], rtol=1e-12)
+
+
 def test_groups_with_identical_B_C_equal_one_group():
     d = _rand(T=9, H=4, G=1, seed=43, has_D="normal")
     B2 = np.repeat(d["B"], 2, axis=2)

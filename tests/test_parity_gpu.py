@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import TAU, assert_close, run_gpu, run_oracle, slice_heads, to_device
+from gpu_util import TAU, assert_close, run_gpu, run_oracle, to_device
 from workloads import WORKLOADS, make_custom, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -371,8 +371,8 @@ def test_host_buffer_entry_point():
 
 
 # --------------------------------------------------------------------------- #
-# Full-size workloads, in the configuration the benchmark times, on sampled
-# (batch row, head) pairs the oracle computes one by one
+# Full-size workloads, in the launch configuration the benchmark times, compared
+# with the oracle element by element over the whole Y and final-state tensors
 # --------------------------------------------------------------------------- #
 
 FULL = ["mamba2_130m_layer", "mamba2_2p7b_layer", "long16k_N16", "long16k_N64", "long16k_N128", "long16k_N256",
@@ -380,15 +380,42 @@ FULL = ["mamba2_130m_layer", "mamba2_2p7b_layer", "long16k_N16", "long16k_N64", 
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(name):
+def test_full_size_whole_tensor(name):
     w = WORKLOADS[name]
     d = make_inputs(w)
     Y, F = run_gpu(d, w.dtype, w.chunk, "auto")
-    rng = np.random.default_rng(99)
-    pairs = {(int(rng.integers(w.batch)), int(rng.integers(w.nheads))) for _ in range(6)}
-    pairs |= {(0, 0), (w.batch - 1, w.nheads - 1)}
-    for b, h in sorted(pairs):
-        s = slice_heads(d, b, h)
-        Yr, Fr = run_oracle(s)
-        assert_close(Y[b:b + 1, :, h:h + 1], Yr, TAU[w.dtype], f"Y[b={b},h={h}]")
-        assert_close(F[b:b + 1, :, h:h + 1], Fr, TAU[w.dtype], f"final[b={b},h={h}]")
+    Yr, Fr = run_oracle(d)  # every (batch row, head), all host cores
+    assert_close(Y, Yr, TAU[w.dtype], f"Y ({name})")
+    assert_close(F, Fr, TAU[w.dtype], f"final_states ({name})")
+
+
+# --------------------------------------------------------------------------- #
+# segment_state stops its backward walk once the decay over the rest of the
+# piece is below e^-40 (those terms reach the cut scaled by < 4.3e-18). Put the
+# largest inputs exactly there: 2^40 times the rest, in the tiles the walk
+# skips, with a cut inside the row; the outputs after the cut must still match
+# the oracle to the tolerance relative to their own magnitude.
+# --------------------------------------------------------------------------- #
+
+def test_segment_walk_cut_with_large_early_inputs():
+    ssd = _ssd()
+    T, wt, cut = 8192, 40, 40 * 128  # ranges [0, 40) and [40, 64) of one row: a cut at token 5120
+    d = make_custom(1, T, 2, 64, 128, dtype="bf16", seed=404, has_D="normal", has_init=True)
+    d["log_a"] = np.full_like(d["log_a"], -0.04)  # the walk stops ~8 tiles back from the cut
+    big = 30 * 128
+    d["X"] = d["X"].copy()
+    d["X"][:, :big] *= 2.0 ** 40  # exact in bf16: a power of two
+    g = to_device(d, "bf16")
+    loc, dec = ssd.segment_state(g["X"], g["log_a"], g["B"], wt)
+    torch.cuda.synchronize()
+    assert float(dec[0].abs().max()) == 0.0, "the walk did not stop early: the case does not exercise the cut"
+    F = torch.full((1, 1, 2, 128, 64), float("nan"), dtype=torch.float32, device="cuda")
+    Yg = ssd.fused_scan_chained(g["X"], g["log_a"], g["B"], g["C"], wt, loc, dec, D=g["D"],
+                                init_states=g["init_states"], final_states=F)
+    torch.cuda.synchronize()
+    ssd.check_device_error()
+    Y = Yg.float().cpu().numpy().astype(np.float64)
+    Yr, Fr = run_oracle(d)
+    assert_close(Y, Yr, TAU["bf16"], "Y")
+    assert_close(Y[:, cut:], Yr[:, cut:], TAU["bf16"], "Y after the cut (its own scale)")
+    assert_close(F.cpu().numpy().astype(np.float64), Fr, TAU["bf16"], "final_states")
