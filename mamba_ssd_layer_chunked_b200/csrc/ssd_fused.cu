@@ -442,6 +442,133 @@ struct __align__(16) CsBuf {
 // every buffer's c rows are read and written as float4
 static_assert(sizeof(CsBuf) % 16 == 0, "CsBuf must keep 16-byte alignment in an array");
 
+// ---------------------------------------------------------------------------
+// The decay warp of the scan kernels. Walks range i_work's pieces (one per row
+// it covers) in tiles of at most 128 tokens that never cross a sequence start,
+// one tile ahead of the buffers it fills: per tile its descriptor, the
+// within-tile inclusive cumsum of log a (log2 units) for both heads, and the
+// whole-tile decays. Lane j holds tokens 4j .. 4j+3 of a tile.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const int i_work, const int lane,
+                                        const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
+                                        CsBuf* csb, uint64_t* bar_csfull, uint64_t* bar_csfree) {
+    const int64_t fb = work_begin(wk, i_work), fe = work_end(wk, i_work);
+    int r = (int)(fb / wk.nt);
+    int s0, s1;
+    row_piece(wk, d.seqlen, fb, fe, r, s0, s1);
+    int pos = s0;
+    bool first = true;
+    auto next_tile = [&](TileDesc& td) {
+        const int b = r / wk.npairs, hp = r % wk.npairs;
+        const int64_t row = (int64_t)b * d.seqlen;
+        int v = min(128, s1 - pos);
+        int sid = 0, psid = pos > 0 ? 0 : -1;
+        bool change = false;  // the sequence changes right after the tile
+        if (seq_idx) {
+            sid = seq_clamped(seq_idx, row, pos, d.nseq);
+            if (pos > 0) psid = seq_clamped(seq_idx, row, pos - 1, d.nseq);
+            // first offset j in [1, min(128, s1 - pos - 1)] whose id differs
+            const int jmax = min(128, s1 - pos - 1);
+            int jm = 1 << 30;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int jj = 4 * lane + 1 + e;
+                if (jj <= jmax && seq_clamped(seq_idx, row, pos + jj, d.nseq) != sid) jm = min(jm, jj);
+            }
+            jm = __reduce_min_sync(0xffffffffu, jm);
+            if (jm <= jmax) {
+                v = jm;
+                change = true;
+            }
+        }
+        const int pend = pos + v;
+        const bool piece_end = pend == s1;
+        const bool last_piece = (int64_t)(r + 1) * wk.nt >= fe;
+        bool seq_end = false;
+        if (pend == d.seqlen) seq_end = true;
+        else if (change) seq_end = true;
+        else if (piece_end && seq_idx) seq_end = seq_clamped(seq_idx, row, pend, d.nseq) != sid;
+        int flags = 0;
+        if (piece_end || change) flags |= kTileLast;
+        if ((piece_end || change) && seq_end) flags |= kTileSeqEnd;
+        if (pend == d.seqlen) flags |= kTileRowEnd;
+        if (piece_end && last_piece) flags |= kTileFinal;
+        if (first && s0 > 0) flags |= kTileFromWork;
+        td.b = b;
+        td.hp = hp;
+        td.ts = pos;
+        td.v = v;
+        td.sid = sid;
+        td.psid = psid;
+        td.flags = flags;
+        first = false;
+        pos = pend;
+        if (piece_end && !last_piece) {
+            ++r;
+            row_piece(wk, d.seqlen, fb, fe, r, s0, s1);
+            pos = s0;
+        }
+    };
+    auto load4 = [&](const TileDesc& td, float (&v)[2][4]) {
+        const int64_t row = (int64_t)td.b * d.seqlen;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = 4 * lane + e;
+                v[hh][e] = tok < td.v ? log_a[(row + td.ts + tok) * d.nheads + 2 * td.hp + hh] : 0.f;
+            }
+    };
+    TileDesc cur;
+    next_tile(cur);
+    float lcur[2][4];
+    load4(cur, lcur);
+    for (int t = 0;; ++t) {
+        const bool fin = (cur.flags & kTileFinal) != 0;
+        TileDesc nxt = cur;
+        float lnxt[2][4];
+        if (!fin) {
+            next_tile(nxt);
+            load4(nxt, lnxt);
+        }
+        const int bi = t & (kCsBufs - 1);
+        if (t >= kCsBufs) mbar_wait(&bar_csfree[bi], ((t / kCsBufs) - 1) & 1);
+        const int last = cur.v - 1;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float x0 = lcur[hh][0] * kLog2e;
+            float x1 = fmaf(lcur[hh][1], kLog2e, x0);
+            float x2 = fmaf(lcur[hh][2], kLog2e, x1);
+            float x3 = fmaf(lcur[hh][3], kLog2e, x2);
+            float tot = x3;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, tot, o);
+                if (lane >= o) tot += y;
+            }
+            const float pre = tot - x3;
+            x0 += pre;
+            x1 += pre;
+            x2 += pre;
+            x3 += pre;
+            *reinterpret_cast<float4*>(&csb[bi].c[hh][4 * lane]) = make_float4(x0, x1, x2, x3);
+            const int el = last & 3;
+            const float mine = el == 0 ? x0 : el == 1 ? x1 : el == 2 ? x2 : x3;
+            const float cend = __shfl_sync(0xffffffffu, mine, last >> 2);
+            if (lane == 0) csb[bi].dec[hh] = ex2_approx(cend);
+        }
+        if (lane == 0) csb[bi].td = cur;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_csfull[bi]);
+        if (fin) break;
+        cur = nxt;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) lcur[hh][e] = lnxt[hh][e];
+    }
+}
+
 // Thread layout of the 16 compute warps: warp w owns the TMEM lane quarter
 // w % 4 and the column quarter w / 4 of every 128-column accumulator it
 // touches; the four warps of a lane quarter split the columns.
@@ -669,124 +796,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         __syncwarp();
     } else if (warp == kComputeWarps + 1) {
         // =================== decay warp ===================
-        // Walks the range's pieces (one per row it covers) in tiles of at most
-        // 128 tokens that never cross a sequence start, one tile ahead of the
-        // buffers it fills. Lane j holds tokens 4j .. 4j+3 of a tile.
-        const int64_t fb = work_begin(wk, i_work), fe = work_end(wk, i_work);
-        int r = (int)(fb / wk.nt);
-        int s0, s1;
-        row_piece(wk, d.seqlen, fb, fe, r, s0, s1);
-        int pos = s0;
-        bool first = true;
-        auto next_tile = [&](TileDesc& td) {
-            const int b = r / wk.npairs, hp = r % wk.npairs;
-            const int64_t row = (int64_t)b * d.seqlen;
-            int v = min(128, s1 - pos);
-            int sid = 0, psid = pos > 0 ? 0 : -1;
-            bool change = false;  // the sequence changes right after the tile
-            if (seq_idx) {
-                sid = seq_clamped(seq_idx, row, pos, d.nseq);
-                if (pos > 0) psid = seq_clamped(seq_idx, row, pos - 1, d.nseq);
-                // first offset j in [1, min(128, s1 - pos - 1)] whose id differs
-                const int jmax = min(128, s1 - pos - 1);
-                int jm = 1 << 30;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int jj = 4 * lane + 1 + e;
-                    if (jj <= jmax && seq_clamped(seq_idx, row, pos + jj, d.nseq) != sid) jm = min(jm, jj);
-                }
-                jm = __reduce_min_sync(0xffffffffu, jm);
-                if (jm <= jmax) {
-                    v = jm;
-                    change = true;
-                }
-            }
-            const int pend = pos + v;
-            const bool piece_end = pend == s1;
-            const bool last_piece = (int64_t)(r + 1) * wk.nt >= fe;
-            bool seq_end = false;
-            if (pend == d.seqlen) seq_end = true;
-            else if (change) seq_end = true;
-            else if (piece_end && seq_idx) seq_end = seq_clamped(seq_idx, row, pend, d.nseq) != sid;
-            int flags = 0;
-            if (piece_end || change) flags |= kTileLast;
-            if ((piece_end || change) && seq_end) flags |= kTileSeqEnd;
-            if (pend == d.seqlen) flags |= kTileRowEnd;
-            if (piece_end && last_piece) flags |= kTileFinal;
-            if (first && s0 > 0) flags |= kTileFromWork;
-            td.b = b;
-            td.hp = hp;
-            td.ts = pos;
-            td.v = v;
-            td.sid = sid;
-            td.psid = psid;
-            td.flags = flags;
-            first = false;
-            pos = pend;
-            if (piece_end && !last_piece) {
-                ++r;
-                row_piece(wk, d.seqlen, fb, fe, r, s0, s1);
-                pos = s0;
-            }
-        };
-        auto load4 = [&](const TileDesc& td, float (&v)[2][4]) {
-            const int64_t row = (int64_t)td.b * d.seqlen;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int tok = 4 * lane + e;
-                    v[hh][e] = tok < td.v ? log_a[(row + td.ts + tok) * d.nheads + 2 * td.hp + hh] : 0.f;
-                }
-        };
-        TileDesc cur;
-        next_tile(cur);
-        float lcur[2][4];
-        load4(cur, lcur);
-        for (int t = 0;; ++t) {
-            const bool fin = (cur.flags & kTileFinal) != 0;
-            TileDesc nxt = cur;
-            float lnxt[2][4];
-            if (!fin) {
-                next_tile(nxt);
-                load4(nxt, lnxt);
-            }
-            const int bi = t & (kCsBufs - 1);
-            if (t >= kCsBufs) mbar_wait(&bar_csfree[bi], ((t / kCsBufs) - 1) & 1);
-            const int last = cur.v - 1;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float x0 = lcur[hh][0] * kLog2e;
-                float x1 = fmaf(lcur[hh][1], kLog2e, x0);
-                float x2 = fmaf(lcur[hh][2], kLog2e, x1);
-                float x3 = fmaf(lcur[hh][3], kLog2e, x2);
-                float tot = x3;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, tot, o);
-                    if (lane >= o) tot += y;
-                }
-                const float pre = tot - x3;
-                x0 += pre;
-                x1 += pre;
-                x2 += pre;
-                x3 += pre;
-                *reinterpret_cast<float4*>(&csb[bi].c[hh][4 * lane]) = make_float4(x0, x1, x2, x3);
-                const int el = last & 3;
-                const float mine = el == 0 ? x0 : el == 1 ? x1 : el == 2 ? x2 : x3;
-                const float cend = __shfl_sync(0xffffffffu, mine, last >> 2);
-                if (lane == 0) csb[bi].dec[hh] = ex2_approx(cend);
-            }
-            if (lane == 0) csb[bi].td = cur;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_csfull[bi]);
-            if (fin) break;
-            cur = nxt;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) lcur[hh][e] = lnxt[hh][e];
-        }
+        decay_walk(d, wk, i_work, lane, log_a, seq_idx, csb, bar_csfull, bar_csfree);
     } else {
         // =================== compute warps ===================
         const int q4 = warp & 3, cq = warp >> 2;
