@@ -358,10 +358,11 @@ __global__ void __launch_bounds__(256) segment_passing_kernel(Dims d, Work wk, c
             row_piece(wk, d.seqlen, work_begin(wk, j0 + l), work_end(wk, j0 + l), r, s0, s1);
             int sl = 0, cont_last = (s0 > 0);
             if (seq_idx) {
+                // the piece's last sequence starts at s0 when s0 already has its id
+                // (ids never decrease), and continues when s0 - 1 has it too
                 sl = seq_clamped(seq_idx, row, s1 - 1, d.nseq);
-                const int st = lower_bound_global(seq_idx, row, s0, s1 - 1, sl, d.nseq);
                 const int prev = s0 > 0 ? seq_clamped(seq_idx, row, s0 - 1, d.nseq) : -1;
-                cont_last = (st == s0) && prev == sl;
+                cont_last = seq_clamped(seq_idx, row, s0, d.nseq) == sl && prev == sl;
             }
             sl_s[l] = sl;
             cl_s[l] = cont_last;
@@ -400,6 +401,7 @@ constexpr int kComputeThreads = 32 * kComputeWarps;
 // four SM sub-partitions, which still fits 96 registers a thread
 constexpr int kFusedThreads = kComputeThreads + 128;
 constexpr int kCsBufs = 4;                           // decay buffers in flight
+constexpr int kChainBatch = 64;                      // pieces resolved together in the scan prologue
 
 template <int N>
 struct FusedSmem {
@@ -617,6 +619,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     __shared__ __align__(16) float cf8[kComputeWarps][2][2][8];
     // per-thread row factors of the next tile: rf (head 0, 1), rg (head 0, 1)
     __shared__ float rowf_s[4][kComputeThreads];
+    // the prologue's chain over the pieces before a cut: per piece its last
+    // sequence id and whether that sequence continues from the piece before
+    __shared__ int chain_sl[kChainBatch];
+    __shared__ int chain_cont[kChainBatch];
     __shared__ __align__(8) uint64_t bar_c, bar_bx[2], bar_g, bar_yo, bar_yd, bar_s, bar_sfree[2], bar_lg, bar_epi,
         bar_st, bar_free, bar_csfull[kCsBufs], bar_csfree[kCsBufs];
     __shared__ uint32_t tmem_base;
@@ -1033,27 +1039,48 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const int b = r / wk.npairs, hp = r % wk.npairs;
                 const int64_t row = (int64_t)b * d.seqlen;
                 const int s_cut = (int)(128 * (fb - rb));
-                griddep_wait();  // the range states come from the kernel before this one
 #pragma unroll
                 for (int i = 0; i < NQ; ++i) hv[i] = 0.f;
-                for (int j = (int)(rb / wk.wt); j < i_work; ++j) {
-                    int s0, s1;
-                    row_piece(wk, d.seqlen, work_begin(wk, j), work_end(wk, j), r, s0, s1);
-                    int sl = 0;
-                    bool cont = s0 > 0;
-                    if (seq_idx) {
-                        sl = seq_clamped(seq_idx, row, s1 - 1, d.nseq);
-                        const int st = lower_bound_global(seq_idx, row, s0, s1 - 1, sl, d.nseq);
-                        cont = st == s0 && s0 > 0 && seq_clamped(seq_idx, row, s0 - 1, d.nseq) == sl;
+                // Pieces are taken kChainBatch at a time: first every piece's last
+                // sequence id and whether that sequence continues from the piece
+                // before (its first token seq(s0) has that id, and so does the token
+                // before s0: ids never decrease), one piece per thread; then the
+                // chain itself, element by element. The ids come from seq_idx alone,
+                // so they are read before the wait for the range states.
+                const int jbeg = (int)(rb / wk.wt);
+                bool waited = false;
+                for (int j0 = jbeg; j0 < i_work; j0 += kChainBatch) {
+                    const int nl = min(kChainBatch, i_work - j0);
+                    named_bar_sync(1, kComputeThreads);  // the previous batch is consumed
+                    if (tid < nl) {
+                        int s0, s1;
+                        row_piece(wk, d.seqlen, work_begin(wk, j0 + tid), work_end(wk, j0 + tid), r, s0, s1);
+                        int sl = 0, cont = s0 > 0;
+                        if (seq_idx) {
+                            sl = seq_clamped(seq_idx, row, s1 - 1, d.nseq);
+                            cont = s0 > 0 && seq_clamped(seq_idx, row, s0, d.nseq) == sl &&
+                                   seq_clamped(seq_idx, row, s0 - 1, d.nseq) == sl;
+                        }
+                        chain_sl[tid] = sl;
+                        chain_cont[tid] = cont;
                     }
-                    const float a = work_decay[(int64_t)j * 2 + sh];
-                    const float* loc = work_local + ((int64_t)j * 2 + sh) * N * kP;
-                    const float* is = cont ? nullptr : init_src(b, hp, sl);
+                    named_bar_sync(1, kComputeThreads);
+                    if (!waited) {
+                        griddep_wait();  // the range states come from the kernel before this one
+                        waited = true;
+                    }
+                    for (int l = 0; l < nl; ++l) {
+                        const int j = j0 + l;
+                        const bool cont = chain_cont[l] != 0;
+                        const float a = work_decay[(int64_t)j * 2 + sh];
+                        const float* loc = work_local + ((int64_t)j * 2 + sh) * N * kP;
+                        const float* is = cont ? nullptr : init_src(b, hp, chain_sl[l]);
 #pragma unroll
-                    for (int i = 0; i < NQ; ++i) {
-                        const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
-                        const float start = cont ? hv[i] : (is ? is[o] : 0.f);
-                        hv[i] = fmaf(a, start, loc[o]);
+                        for (int i = 0; i < NQ; ++i) {
+                            const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
+                            const float start = cont ? hv[i] : (is ? is[o] : 0.f);
+                            hv[i] = fmaf(a, start, loc[o]);
+                        }
                     }
                 }
                 if (seq_idx) {
