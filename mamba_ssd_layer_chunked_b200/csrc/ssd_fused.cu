@@ -28,11 +28,12 @@
 // change the output), so the tiles here are aligned to sequence starts: no tile
 // mixes two sequences.
 //
-// fused_scan is warp-specialised: 16 compute warps (warp w reaches the TMEM
-// lane quarter w % 4), one control warp that issues TMA copies and tcgen05.mma,
-// and one decay warp that walks the range ahead of the others and publishes,
-// per tile, its coordinates and the within-tile cumsum of log a; the roles
-// handshake through mbarriers.
+// fused_scan has 20 warps: 16 compute warps (warp w reaches the TMEM lane
+// quarter w % 4) that run each tile's epilogue, L o G build and state update in
+// turn; three issuing threads, one warp each (the L o G-side MMAs, the
+// state-side MMAs and the Y store, the TMA loads); and one decay warp that walks
+// the range ahead of the others and publishes, per tile, its coordinates and
+// the within-tile cumsum of log a. The roles handshake through mbarriers.
 
 #include <cuda.h>
 
