@@ -81,6 +81,33 @@ __device__ __forceinline__ void row_piece(const Work& w, int seqlen, int64_t fb,
     s1 = (int)min((int64_t)128 * (fe - rb), (int64_t)seqlen);
 }
 
+// The two 64-column slots of pair row hp (rows r = b * npairs + hp): slot s
+// carries head h from column p0 of that head's dimension. The heads of a group
+// are paired in order; in a group with an odd number of heads the last pair's
+// slot 1 has no head of its own (valid = false): it mirrors slot 0's head and
+// nothing of it is written. With headdim 128 a row is one head, and its two
+// slots are the two halves of the head dimension.
+struct Slot {
+    int h, p0;
+    bool valid;
+};
+__device__ __forceinline__ Slot slot_of(const Dims& d, int hp, int s) {
+    Slot o;
+    if (d.headdim == 2 * kP) {
+        o.h = hp;
+        o.p0 = kP * s;
+        o.valid = true;
+        return o;
+    }
+    const int npg = (d.heads_per_group + 1) >> 1;  // pairs per group
+    const int g = hp / npg, j = hp - g * npg;
+    const int h0 = g * d.heads_per_group + 2 * j;
+    o.valid = s == 0 || 2 * j + 1 < d.heads_per_group;
+    o.h = o.valid ? h0 + s : h0;
+    o.p0 = 0;
+    return o;
+}
+
 // ===========================================================================
 // segment_state
 // ===========================================================================
@@ -122,7 +149,8 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     row_piece(wk, d.seqlen, work_begin(wk, i_work), fe, r, s0, s1);
     if (s1 >= d.seqlen && !whole_rows) return;  // ends at the row end: nothing feeds a next range
     const int hp = r % wk.npairs, b = r / wk.npairs;
-    const int h0 = 2 * hp, g = h0 / d.heads_per_group;
+    const Slot sl0 = slot_of(d, hp, 0), sl1 = slot_of(d, hp, 1);
+    const int g = sl0.h / d.heads_per_group;
     const int64_t row = (int64_t)b * d.seqlen;
     if (whole_rows && hp == 0 && tid == 0) {
         row_ids[2 * b] = seq_idx ? seq_clamped(seq_idx, row, 0, d.nseq) : 0;
@@ -202,7 +230,7 @@ __global__ void __launch_bounds__(kSegThreads, 1)
         auto load_la = [&](int i) -> float {
             const int ts = st + 128 * i;
             const int v = min(128, s1 - ts);
-            return log_a[(row + ts + min(rr, v - 1)) * d.nheads + h0 + hh];
+            return log_a[(row + ts + min(rr, v - 1)) * d.nheads + (hh ? sl1.h : sl0.h)];
         };
         // tile i's X (two heads) and B into stage sg
         auto issue_load = [&](int i, int sg) {
@@ -210,8 +238,8 @@ __global__ void __launch_bounds__(kSegThreads, 1)
             uint8_t* xs = smem + sg * kStage;
             uint8_t* bs = xs + kXB;
             mbar_arrive_expect_tx(&bar_load[sg], kStage);
-            tma_load_4d(xs, &tm_x, &bar_load[sg], 0, h0, ts, b);
-            tma_load_4d(xs + kBox, &tm_x, &bar_load[sg], 0, h0 + 1, ts, b);
+            tma_load_4d(xs, &tm_x, &bar_load[sg], sl0.p0, sl0.h, ts, b);
+            tma_load_4d(xs + kBox, &tm_x, &bar_load[sg], sl1.p0, sl1.h, ts, b);
 #pragma unroll
             for (int q = 0; q < N / 64; ++q) tma_load_4d(bs + q * kBox, &tm_b, &bar_load[sg], 64 * q, g, ts, b);
         };
@@ -424,15 +452,19 @@ struct FusedSmem {
 // One tile of a range, as the decay warp publishes it: batch row, head pair,
 // first token, valid rows, the sequence id of its tokens, the id of the token
 // before it in the row (-1 at the row start) and flags.
+// Also the row's slot mapping (slot_of), worked out once per tile: the heads
+// of slots 0 and 1, the first column of slot 1 in its head, the B/C group.
 struct TileDesc {
     int b, hp, ts, v, sid, psid, flags;
+    int h0, h1, p1, g;
 };
 enum : int {
-    kTileLast = 1,      // last tile of its sequence piece in this range
-    kTileSeqEnd = 2,    // ... and the sequence ends there (its final state is due)
-    kTileRowEnd = 4,    // the tile ends its row
-    kTileFinal = 8,     // last tile of the range
-    kTileFromWork = 16  // first tile of a range that starts inside its row
+    kTileLast = 1,       // last tile of its sequence piece in this range
+    kTileSeqEnd = 2,     // ... and the sequence ends there (its final state is due)
+    kTileRowEnd = 4,     // the tile ends its row
+    kTileFinal = 8,      // last tile of the range
+    kTileFromWork = 16,  // first tile of a range that starts inside its row
+    kTileNoSlot1 = 32    // slot 1 has no head (odd heads per group): nothing of it is written
 };
 
 // 16-row block of the tokens held by lane half hi (lanes 16 hi .. 16 hi + 15)
@@ -446,7 +478,7 @@ __device__ __forceinline__ int row_block(int q, int hi) { return 2 * q + hi; }
 struct __align__(16) CsBuf {
     float c[2][128];
     float dec[2];
-    int pad[2];
+    int pad[3];
     TileDesc td;
 };
 // every buffer's c rows are read and written as float4
@@ -459,6 +491,7 @@ static_assert(sizeof(CsBuf) % 16 == 0, "CsBuf must keep 16-byte alignment in an 
 // within-tile inclusive cumsum of log a (log2 units) for both heads, and the
 // whole-tile decays. Lane j holds tokens 4j .. 4j+3 of a tile.
 // ---------------------------------------------------------------------------
+template <bool kGen>
 __device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const int i_work, const int lane,
                                         const float* __restrict__ log_a, const int32_t* __restrict__ seq_idx,
                                         CsBuf* csb, uint64_t* bar_csfull, uint64_t* bar_csfree) {
@@ -504,6 +537,15 @@ __device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const in
         if (pend == d.seqlen) flags |= kTileRowEnd;
         if (piece_end && last_piece) flags |= kTileFinal;
         if (first && s0 > 0) flags |= kTileFromWork;
+        Slot q0, q1;
+        if constexpr (kGen) {
+            q0 = slot_of(d, hp, 0);
+            q1 = slot_of(d, hp, 1);
+            if (!q1.valid) flags |= kTileNoSlot1;
+        } else {  // a plain head pair
+            q0 = {2 * hp, 0, true};
+            q1 = {2 * hp + 1, 0, true};
+        }
         td.b = b;
         td.hp = hp;
         td.ts = pos;
@@ -511,6 +553,10 @@ __device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const in
         td.sid = sid;
         td.psid = psid;
         td.flags = flags;
+        td.h0 = q0.h;
+        td.h1 = q1.h;
+        td.p1 = q1.p0;
+        td.g = q0.h / d.heads_per_group;
         first = false;
         pos = pend;
         if (piece_end && !last_piece) {
@@ -526,7 +572,7 @@ __device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const in
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int tok = 4 * lane + e;
-                v[hh][e] = tok < td.v ? log_a[(row + td.ts + tok) * d.nheads + 2 * td.hp + hh] : 0.f;
+                v[hh][e] = tok < td.v ? log_a[(row + td.ts + tok) * d.nheads + (hh ? td.h1 : td.h0)] : 0.f;
             }
     };
     TileDesc cur;
@@ -603,7 +649,7 @@ __device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const in
 // kAcc: a later state slice, whose epilogue adds its Y to the Y already there
 // (each thread reads the elements it then writes); a separate instantiation so
 // that the common case keeps its epilogue unchanged.
-template <int N, bool kAcc>
+template <int N, bool kAcc, bool kGen>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, Dims d,
@@ -675,6 +721,25 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                    tm_h = tmem_base + 384;
 
     const uint32_t ca = smem_u32(Cs), ha = smem_u32(Hs);
+    // slot s of a tile's row: its head, first column in that head, and whether it
+    // has a head (kGen: the mapping the decay warp worked out; else a plain head
+    // pair 2 hp, 2 hp + 1)
+    auto head_of = [&](const TileDesc& td, int s) -> int {
+        if constexpr (kGen) return s ? td.h1 : td.h0;
+        else return 2 * td.hp + s;
+    };
+    auto p0_of = [&](const TileDesc& td, int s) -> int {
+        if constexpr (kGen) return s ? td.p1 : 0;
+        else return 0;
+    };
+    auto valid_of = [&](const TileDesc& td, int s) -> bool {
+        if constexpr (kGen) return s == 0 || !(td.flags & kTileNoSlot1);
+        else return true;
+    };
+    auto group_row = [&](const TileDesc& td) -> int {
+        if constexpr (kGen) return td.g;
+        else return 2 * td.hp / d.heads_per_group;
+    };
     auto stage_x = [&](int t) { return smem_u32(smem + S::oX + (t & 1) * S::kX); };
     auto stage_b = [&](int t) { return smem_u32(smem + S::oB + (t & 1) * S::kB); };
     // tile t's descriptor, once the decay warp has published it
@@ -747,8 +812,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 tc_fence_after();
                 const bool full = cur.v == 128;
                 if (full) {
-                    tma_store_4d(&tm_y, Hs, 0, 2 * cur.hp, cur.ts, cur.b);
-                    tma_store_4d(&tm_y, Hs + kBox, 0, 2 * cur.hp + 1, cur.ts, cur.b);
+                    tma_store_4d(&tm_y, Hs, p0_of(cur, 0), head_of(cur, 0), cur.ts, cur.b);
+                    if (valid_of(cur, 1)) tma_store_4d(&tm_y, Hs + kBox, p0_of(cur, 1), head_of(cur, 1), cur.ts, cur.b);
                     tma_store_commit();
                 }
                 const uint32_t xa = stage_x(t), ba = stage_b(t);
@@ -769,18 +834,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // =================== TMA loads: C(t), B(t), X(t) ===================
         if (lane == 0) {
             auto load_bx = [&](const TileDesc& td, int st) {
-                const int h0 = 2 * td.hp, g = h0 / d.heads_per_group;
+                const int g = group_row(td);
                 uint8_t* Bsg = smem + S::oB + st * S::kB;
                 uint8_t* Xsg = smem + S::oX + st * S::kX;
                 mbar_arrive_expect_tx(&bar_bx[st], S::kB + S::kX);
 #pragma unroll
                 for (int q = 0; q < N / 64; ++q)
                     tma_load_4d(Bsg + q * kBox, &tm_b, &bar_bx[st], 64 * q, g, td.ts, td.b);
-                tma_load_4d(Xsg, &tm_x, &bar_bx[st], 0, h0, td.ts, td.b);
-                tma_load_4d(Xsg + kBox, &tm_x, &bar_bx[st], 0, h0 + 1, td.ts, td.b);
+                tma_load_4d(Xsg, &tm_x, &bar_bx[st], p0_of(td, 0), head_of(td, 0), td.ts, td.b);
+                tma_load_4d(Xsg + kBox, &tm_x, &bar_bx[st], p0_of(td, 1), head_of(td, 1), td.ts, td.b);
             };
             auto load_c = [&](const TileDesc& td) {
-                const int g = 2 * td.hp / d.heads_per_group;
+                const int g = group_row(td);
                 mbar_arrive_expect_tx(&bar_c, S::kC);
 #pragma unroll
                 for (int q = 0; q < N / 64; ++q) tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, td.ts, td.b);
@@ -810,7 +875,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         __syncwarp();
     } else if (warp == kComputeWarps + 1) {
         // =================== decay warp ===================
-        decay_walk(d, wk, i_work, lane, log_a, seq_idx, csb, bar_csfull, bar_csfree);
+        decay_walk<kGen>(d, wk, i_work, lane, log_a, seq_idx, csb, bar_csfull, bar_csfree);
     } else {
         // =================== compute warps ===================
         const int q4 = warp & 3, cq = warp >> 2;
@@ -920,7 +985,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const CsBuf& cs = csb[t & (kCsBufs - 1)];
             const int hi = lane >> 4;
             const int rb = row_block(q4, hi);
-            const int hp = cs.td.hp;
             const uint32_t tcol = tm_lg + lane_off + 32 * cq;  // this warp's 32 columns
             __syncwarp();
             mbar_wait(&bar_g, t & 1);
@@ -934,7 +998,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 tmem_wait_ld();
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
-                    const HeadF f = {rowf_s[hh][tid], rowf_s[2 + hh][tid], cs.c[hh][k], Dv ? Dv[2 * hp + hh] : 0.f};
+                    const HeadF f = {rowf_s[hh][tid], rowf_s[2 + hh][tid], cs.c[hh][k],
+                                     Dv ? Dv[head_of(cs.td, hh)] : 0.f};
                     uint32_t w0[8], w1[8];
                     if (cq == q4) {
                         // lane half hi's diagonal block is column block hi; block 0
@@ -987,10 +1052,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if constexpr (NQ == 32) tmem_st32(tm_h + lane_off + NQ * cq, reinterpret_cast<const uint32_t(&)[32]>(v));
             else tmem_st16(tm_h + lane_off + NQ * cq, reinterpret_cast<const uint32_t(&)[16]>(v));
         };
-        auto load_state = [&](float (&v)[NQ], const float* src) {  // src: [N][P] of head sh, or null
+        // src: this slot's columns of an [N][stride] state (stride = headdim for the
+        // caller's states, 64 for the range buffers), or null for zero
+        auto load_state = [&](float (&v)[NQ], const float* src, int stride) {
 #pragma unroll
-            for (int i = 0; i < NQ; ++i) v[i] = src ? src[(int64_t)(cq * NQ + i) * kP + sp] : 0.f;
+            for (int i = 0; i < NQ; ++i) v[i] = src ? src[(int64_t)(cq * NQ + i) * stride + sp] : 0.f;
         };
+        const int P = kGen ? d.headdim : kP;  // row stride of the caller's states
         auto write_hs = [&](const float (&v)[NQ]) {  // bf16 state, row m, K-major over n
 #pragma unroll
             for (int c8 = 0; c8 < NQ / 8; ++c8) {
@@ -1001,9 +1069,26 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             }
         };
 
-        // the initial state (or zero) of sequence sid of batch row b for head pair hp
+        // this slot's columns of the initial state of sequence sid of batch row b
+        // in pair row hp, or null (zero) without initial states or for a slot
+        // without a head
         auto init_src = [&](int b, int hp, int sid) -> const float* {
-            return init_states ? init_states + seqst_off(d, b, sid, 2 * hp + sh) : nullptr;
+            if constexpr (kGen) {
+                const Slot o = slot_of(d, hp, sh);
+                return init_states && o.valid ? init_states + seqst_off(d, b, sid, o.h) + o.p0 : nullptr;
+            } else {
+                return init_states ? init_states + seqst_off(d, b, sid, 2 * hp + sh) : nullptr;
+            }
+        };
+        // this slot's columns of the final state of sequence sid, or null for a
+        // slot without a head
+        auto final_dst = [&](int b, int hp, int sid) -> float* {
+            if constexpr (kGen) {
+                const Slot o = slot_of(d, hp, sh);
+                return o.valid ? final_states + seqst_off(d, b, sid, o.h) + o.p0 : nullptr;
+            } else {
+                return final_states + seqst_off(d, b, sid, 2 * hp + sh);
+            }
         };
 
         // ids that never occur between the sequence before tile td and its own
@@ -1011,11 +1096,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         auto fill_gap = [&](const TileDesc& td) {
             if (!final_states || !seq_idx) return;
             for (int sq = td.psid + 1; sq < td.sid; ++sq) {
-                float* f = final_states + seqst_off(d, td.b, sq, 2 * td.hp + sh);
+                float* f = final_dst(td.b, td.hp, sq);
+                if (!f) continue;
                 const float* src = init_src(td.b, td.hp, sq);
 #pragma unroll 1
                 for (int i = 0; i < NQ; ++i) {
-                    const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
+                    const int64_t o = (int64_t)(cq * NQ + i) * P + sp;
                     f[o] = src ? src[o] : 0.f;
                 }
             }
@@ -1030,9 +1116,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const TileDesc& td0 = csb[0].td;
             float hv[NQ];
             if (!(td0.flags & kTileFromWork)) {
-                load_state(hv, init_src(td0.b, td0.hp, td0.sid));
+                load_state(hv, init_src(td0.b, td0.hp, td0.sid), P);
             } else if (work_in) {
-                load_state(hv, work_in + ((int64_t)i_work * 2 + sh) * N * kP);
+                load_state(hv, work_in + ((int64_t)i_work * 2 + sh) * N * kP, kP);
             } else {
                 // The range starts inside its row: the state entering its first
                 // token from the pieces of the row before the cut (ranges i0 ..
@@ -1085,15 +1171,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         const float* is = cont ? nullptr : init_src(b, hp, chain_sl[l]);
 #pragma unroll
                         for (int i = 0; i < NQ; ++i) {
-                            const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
-                            const float start = cont ? hv[i] : (is ? is[o] : 0.f);
-                            hv[i] = fmaf(a, start, loc[o]);
+                            const int64_t n = cq * NQ + i;
+                            const float start = cont ? hv[i] : (is ? is[n * P + sp] : 0.f);
+                            hv[i] = fmaf(a, start, loc[n * kP + sp]);
                         }
                     }
                 }
                 if (seq_idx) {
                     const int sf = seq_clamped(seq_idx, row, s_cut, d.nseq);
-                    if (seq_clamped(seq_idx, row, s_cut - 1, d.nseq) != sf) load_state(hv, init_src(b, hp, sf));
+                    if (seq_clamped(seq_idx, row, s_cut - 1, d.nseq) != sf) load_state(hv, init_src(b, hp, sf), P);
                 }
             }
             write_hs(hv);
@@ -1131,13 +1217,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             tc_fence_after();
             {
                 const __nv_bfloat162 wx2 = __floats2bfloat162_rn(wx, wx);
-                const int64_t yoff = ((rowt + cur.ts + k) * d.nheads + 2 * cur.hp + eh) * (int64_t)kP + p0;
+                const bool yvalid = valid_of(cur, eh);
+                const int64_t yoff = ((rowt + cur.ts + k) * d.nheads + head_of(cur, eh)) * (int64_t)P +
+                                     p0_of(cur, eh) + p0;
                 __nv_bfloat16* yrow = Y + yoff;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     // a later state slice: the Y this thread's outputs add to
                     uint4 ya[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-                    if (kAcc && k < cur.v) {
+                    if (kAcc && k < cur.v && yvalid) {
 #pragma unroll
                         for (int c = 0; c < 2; ++c) ya[c] = *reinterpret_cast<const uint4*>(Y + yoff + 8 * (2 * hf + c));
                     }
@@ -1171,7 +1259,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         }
                         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
                         if (cur.v == 128) *reinterpret_cast<uint4*>(Hs + eh * kBox + off) = ov;  // Y_off(t) has read Hs
-                        else if (k < cur.v) *reinterpret_cast<uint4*>(yrow + 8 * (c16 - (p0 >> 3))) = ov;
+                        else if (k < cur.v && yvalid) *reinterpret_cast<uint4*>(yrow + 8 * (c16 - (p0 >> 3))) = ov;
                         *reinterpret_cast<uint4*>(Xst + off) = xv;
                     }
                 }
@@ -1191,25 +1279,26 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 float hv[NQ];
                 ld_state(hv);
                 if (cur.flags & kTileLast) {
-                    if (final_states && (cur.flags & kTileSeqEnd)) {
-                        float* f = final_states + seqst_off(d, cur.b, cur.sid, 2 * cur.hp + sh);
+                    float* f = final_states && (cur.flags & kTileSeqEnd) ? final_dst(cur.b, cur.hp, cur.sid) : nullptr;
+                    if (f) {
 #pragma unroll
-                        for (int i = 0; i < NQ; ++i) f[(int64_t)(cq * NQ + i) * kP + sp] = hv[i];
+                        for (int i = 0; i < NQ; ++i) f[(int64_t)(cq * NQ + i) * P + sp] = hv[i];
                     }
                     // the next tile starts a new sequence or a new row
                     if (!fin) {
-                        load_state(hv, init_src(nx.b, nx.hp, nx.sid));
+                        load_state(hv, init_src(nx.b, nx.hp, nx.sid), P);
                         fill_gap(nx);
                     }
                 }
                 // ids after the row's last sequence never occur: they keep their initial state
                 if ((cur.flags & kTileRowEnd) && final_states && seq_idx) {
                     for (int sq = cur.sid + 1; sq < d.nseq; ++sq) {
-                        float* f = final_states + seqst_off(d, cur.b, sq, 2 * cur.hp + sh);
+                        float* f = final_dst(cur.b, cur.hp, sq);
+                        if (!f) continue;
                         const float* src = init_src(cur.b, cur.hp, sq);
 #pragma unroll 1
                         for (int i = 0; i < NQ; ++i) {
-                            const int64_t o = (int64_t)(cq * NQ + i) * kP + sp;
+                            const int64_t o = (int64_t)(cq * NQ + i) * P + sp;
                             f[o] = src ? src[o] : 0.f;
                         }
                     }
@@ -1268,9 +1357,16 @@ int num_sms() {
     return v;
 }
 
+// pair rows per batch row: head pairs of each group (the last one half empty
+// when a group has an odd number of heads), or single heads with headdim 128
+int pair_rows(const Dims& d) {
+    if (d.headdim == 2 * kP) return d.nheads;
+    return d.ngroups * ((d.heads_per_group + 1) / 2);
+}
+
 Work make_work(const Dims& d, int64_t work_tiles) {
     Work w;
-    w.npairs = d.nheads / 2;
+    w.npairs = pair_rows(d);
     w.nt = (d.seqlen + 127) / 128;
     w.total = (int64_t)d.batch * w.npairs * w.nt;
     w.wt = (int)work_tiles;
@@ -1288,14 +1384,14 @@ bool fused_supported(const ssd_problem* p) {
 }
 
 bool fused_fwd_supported(const ssd_problem* p) {
-    if (p->dtype != SSD_DTYPE_BF16 || p->headdim != kP) return false;
+    if (p->dtype != SSD_DTYPE_BF16) return false;
+    if (p->headdim != kP && p->headdim != 2 * kP) return false;  // pairs of 64-column slots
     if (p->dstate % 16 != 0 || p->dstate > 256) return false;
-    if ((p->nheads / p->ngroups) % 2 != 0) return false;
     return true;
 }
 
 bool fused_work_ok(const Dims& d, int64_t work_tiles) {
-    const int64_t total = (int64_t)d.batch * (d.nheads / 2) * ((d.seqlen + 127) / 128);
+    const int64_t total = (int64_t)d.batch * pair_rows(d) * ((d.seqlen + 127) / 128);
     if (work_tiles < 1 || work_tiles > total) return false;
     return (total + work_tiles - 1) / work_tiles <= (int64_t)1 << 30;
 }
@@ -1312,7 +1408,7 @@ bool fused_needs_cut_states(const Dims& d, int64_t work_tiles) {
 // per CTA, which need no cut states, measured slower on the 130M-shaped layer:
 // 72.4 against 69.5 us with 96 of 148 SMs busy.)
 int fused_default_work_tiles(const Dims& d) {
-    const int64_t total = (int64_t)d.batch * (d.nheads / 2) * ((d.seqlen + 127) / 128);
+    const int64_t total = (int64_t)d.batch * pair_rows(d) * ((d.seqlen + 127) / 128);
     const int64_t g = std::min<int64_t>(num_sms(), total);
     return (int)((total + g - 1) / g);
 }
@@ -1390,16 +1486,22 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
     cfg.attrs = attr;
     cfg.numAttrs = after_segment_state ? 1 : 0;
     __nv_bfloat16* Yb = (__nv_bfloat16*)Y;
+    // the general slot mapping (headdim 128, or an odd number of heads per group) is
+    // its own instantiation, so that the plain head pairs keep their code
+    const bool gen = d.headdim != kP || d.heads_per_group % 2 != 0;
+    const int slot = (Yacc ? 2 : 0) + (gen ? 4 : 0);
     if (d.dstate == 64) {
-        auto k = Yacc ? fused_scan_kernel<64, true> : fused_scan_kernel<64, false>;
+        auto k = gen ? (Yacc ? fused_scan_kernel<64, true, true> : fused_scan_kernel<64, false, true>)
+                     : (Yacc ? fused_scan_kernel<64, true, false> : fused_scan_kernel<64, false, false>);
         cfg.dynamicSmemBytes = fused_smem_bytes<64>();
-        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, Yacc ? 34 : 32)) != cudaSuccess) return e;
+        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 40 + slot)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
                                final_states, work_local, work_decay, err);
     } else if (d.dstate == 128) {
-        auto k = Yacc ? fused_scan_kernel<128, true> : fused_scan_kernel<128, false>;
+        auto k = gen ? (Yacc ? fused_scan_kernel<128, true, true> : fused_scan_kernel<128, false, true>)
+                     : (Yacc ? fused_scan_kernel<128, true, false> : fused_scan_kernel<128, false, false>);
         cfg.dynamicSmemBytes = fused_smem_bytes<128>();
-        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, Yacc ? 35 : 33)) != cudaSuccess) return e;
+        if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 41 + slot)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
                                final_states, work_local, work_decay, err);
     } else {

@@ -80,6 +80,12 @@ SMALL = {
     "f32_ragged_T300_Q64": (2, 300, 3, 32, 48, 1, 64, "f32", [[100, 200], [300]], "normal", True),
     "f32_ragged_T70_Q128": (1, 70, 2, 16, 16, 1, 128, "f32", None, "ones", True),
     "bf16_ragged_boundary_in_last_chunk": (1, 700, 4, 64, 128, 1, 256, "bf16", [[600, 100]], "normal", True),
+    # head dimension 128: one head per row of the fused family, its two 64-column halves as the slots
+    "bf16_P128_varlen_N128": (2, 900, 3, 128, 128, 1, 256, "bf16", [[250, 650], [900]], "normal", True),
+    "bf16_P128_groups2_N64": (1, 640, 4, 128, 64, 2, 128, "bf16", None, "normal", False),
+    "bf16_P128_N256_slices": (1, 512, 2, 128, 256, 1, 256, "bf16", [[200, 312]], "normal", True),
+    # an odd number of heads per group with ranges that cut rows (the half-empty last pair)
+    "bf16_odd_heads_varlen": (2, 1500, 5, 64, 128, 1, 256, "bf16", [[700, 800], [1500]], "normal", True),
 }
 
 

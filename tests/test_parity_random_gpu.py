@@ -110,3 +110,53 @@ def test_random_large_problem_fused_and_chunked(i):
         Y, F = run_gpu(d, "bf16", Q, path)
         assert_close(Y, Yr, TAU["bf16"], f"Y ({path}; {desc})")
         assert_close(F, Fr, TAU["bf16"], f"final_states ({path}; {desc})")
+
+
+NWIDE = 16
+
+
+def _draw_wide(i):
+    """Problems that the fused family runs as 64-column slots other than a plain
+    head pair: head dimension 128 (one head per row), or an odd number of heads
+    per group (the last pair of each group half empty). Long enough, for some,
+    that the work ranges cut rows."""
+    rng = np.random.default_rng(11000 + i)
+    b = int(rng.integers(1, 3))
+    T = int(rng.choice([int(rng.integers(1, 600)), int(rng.integers(1500, 3500))]))
+    if i % 2 == 0:
+        P, H = 128, int(rng.integers(1, 5))
+        G = int(rng.choice([g for g in range(1, H + 1) if H % g == 0]))
+    else:
+        P = 64
+        G = int(rng.integers(1, 3))
+        H = G * int(rng.choice([1, 3, 5]))
+    N = int(rng.choice([32, 64, 128, 128, 256]))
+    Q = int(rng.choice([64, 128, 256]))
+    lengths = None
+    if rng.random() < 0.6:
+        nseq = int(rng.integers(1, 6))
+        lengths = []
+        for _ in range(b):
+            cuts = np.sort(rng.integers(0, T + 1, size=nseq - 1))
+            lengths.append(np.diff(np.concatenate([[0], cuts, [T]])).astype(int).tolist())
+    D = str(rng.choice(["none", "normal"]))
+    init = bool(rng.random() < 0.5)
+    nseq = None if lengths is None else max(len(r) for r in lengths)
+    d = make_custom(b, T, H, P, N, ngroups=G, dtype="bf16", seed=int(rng.integers(0, 10000)), has_D=D,
+                    has_init=init, lengths=lengths, nseq=nseq)
+    return d, Q, f"bf16 b{b} T{T} H{H} G{G} P{P} N{N} Q{Q} nseq={nseq} D={D} init={init}"
+
+
+@pytest.mark.parametrize("i", range(NWIDE))
+def test_random_wide_slots_fused(i):
+    import mamba_ssd_layer_chunked_b200 as ssd
+    d, Q, desc = _draw_wide(i)
+    X = d["X"]
+    p = ssd.make_problem(X.shape[0], X.shape[1], X.shape[2], X.shape[3], d["B"].shape[3], d["B"].shape[2], Q,
+                         d["nseq"], torch.bfloat16)
+    assert ssd.path_supported(p, "fused"), desc
+    Yr, Fr = run_oracle(d)
+    for path in ("auto", "fused"):
+        Y, F = run_gpu(d, "bf16", Q, path)
+        assert_close(Y, Yr, TAU["bf16"], f"Y ({path}; {desc})")
+        assert_close(F, Fr, TAU["bf16"], f"final_states ({path}; {desc})")
