@@ -79,10 +79,12 @@ typedef enum {
 /* Kernel family.
  *   SIMT     the four steps as fp32 SIMT kernels (any supported shape, fp32 or bf16);
  *   FUSED    the two-level tensor-core path of ssd_segment_state /
- *            ssd_segment_passing / ssd_fused_scan (bf16, headdim 64, dstate a
- *            multiple of 16 up to 256, an even number of heads per group; any
- *            chunk): the state stays on chip within a work range and crosses HBM
- *            only where a range boundary cuts a row.
+ *            ssd_segment_passing / ssd_fused_scan (bf16, headdim 64 or 128, dstate
+ *            a multiple of 16 up to 256, any number of heads per group; any chunk):
+ *            the state stays on chip within a work range and crosses HBM only
+ *            where a range boundary cuts a row. (The fused step entry points
+ *            below take headdim 64, dstate 64 or 128 and an even number of heads
+ *            per group; ssd_fwd covers the rest of the family's domain.)
  * AUTO picks FUSED where the problem allows it, else SIMT. An explicit family
  * outside its domain returns SSD_ERR_UNSUPPORTED. (Value 2 is not used.) */
 typedef enum {
@@ -269,9 +271,9 @@ ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, co
  *   work_local / work_incoming  [nwork, 2, dstate, headdim] fp32 (the two heads
  *                               of the row the range ends / starts in)
  *   work_decay                  [nwork, 2] fp32
- * These entry points cover the FUSED family's domain only
- * (SSD_ERR_UNSUPPORTED elsewhere); 1 <= work_tiles <= the number of tiles,
- * else SSD_ERR_INVALID_ARG. */
+ * These entry points take bf16, headdim 64, dstate 64 or 128 and an even
+ * number of heads per group (SSD_ERR_UNSUPPORTED elsewhere); 1 <= work_tiles
+ * <= the number of tiles, else SSD_ERR_INVALID_ARG. */
 
 /* Tiles per range ssd_fwd uses for p on the current device (about one range
  * per SM), or -1 if p is invalid or outside the fused domain. */
