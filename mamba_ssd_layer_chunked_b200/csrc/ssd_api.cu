@@ -3,6 +3,8 @@
 // sequence chunk_cumsum -> chunk_state -> state_passing -> chunk_scan on the
 // caller's stream. Nothing here allocates, synchronises or reads device memory.
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -40,6 +42,18 @@ cudaError_t device_error_word(unsigned int** out) {
 namespace {
 
 thread_local char g_cuda_err[256] = "";
+
+// An NVTX range around the host-side enqueue of one entry point or one kernel
+// launch, named after it ("ssd_fwd", "fused_scan", ...): a profiler attaches
+// the kernels launched inside a range to its name (Nsight Systems' timeline,
+// `ncu --nvtx --nvtx-include`). With no tool attached a push or pop costs one
+// check of a function pointer.
+struct TraceRange {
+    explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange&) = delete;
+    TraceRange& operator=(const TraceRange&) = delete;
+};
 
 ssd_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return SSD_OK;
@@ -197,8 +211,12 @@ cudaError_t run_fused(const ssd::Dims& d, const void* X, const float* log_a, con
     const bool cuts = ssd::fused_needs_cut_states(d, wt);
     cudaError_t e = cudaSuccess;
     (void)work_in;  // the fused scan chains the pieces before each cut itself
-    if (cuts && (e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st)) != cudaSuccess)
-        return e;
+    if (cuts) {
+        TraceRange r("segment_state");
+        if ((e = ssd::launch_segment_state(d, wt, X, log_a, B, seq_idx, work_local, work_decay, st)) != cudaSuccess)
+            return e;
+    }
+    TraceRange r("fused_scan");
     return ssd::launch_fused_scan(d, wt, X, log_a, B, C, D, nullptr, init_states, seq_idx, Y, final_states, st,
                                   cuts ? work_local : nullptr, cuts ? work_decay : nullptr, cuts, Yacc);
 }
@@ -312,6 +330,7 @@ int64_t ssd_fused_work_count(const ssd_problem* p, int64_t work_tiles) {
 ssd_status ssd_segment_state(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a,
                              const void* B, const int32_t* seq_idx, float* work_local, float* work_decay,
                              void* stream) {
+    TraceRange trace("ssd_segment_state");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !work_local || !work_decay) return SSD_ERR_INVALID_ARG;
@@ -327,6 +346,7 @@ ssd_status ssd_segment_state(const ssd_problem* p, int64_t work_tiles, const voi
 ssd_status ssd_segment_passing(const ssd_problem* p, int64_t work_tiles, const float* work_local,
                                const float* work_decay, const float* init_states, const int32_t* seq_idx,
                                float* work_incoming, void* stream) {
+    TraceRange trace("ssd_segment_passing");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!work_local || !work_decay || !work_incoming) return SSD_ERR_INVALID_ARG;
@@ -343,6 +363,7 @@ ssd_status ssd_segment_passing(const ssd_problem* p, int64_t work_tiles, const f
 ssd_status ssd_fused_scan(const ssd_problem* p, int64_t work_tiles, const void* X, const float* log_a, const void* B,
                           const void* C, const float* D, const float* work_incoming, const float* init_states,
                           const int32_t* seq_idx, void* Y, float* final_states, void* stream) {
+    TraceRange trace("ssd_fused_scan");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
@@ -361,6 +382,7 @@ ssd_status ssd_fused_scan_chained(const ssd_problem* p, int64_t work_tiles, cons
                                   const void* B, const void* C, const float* D, const float* work_local,
                                   const float* work_decay, const float* init_states, const int32_t* seq_idx,
                                   void* Y, float* final_states, void* stream) {
+    TraceRange trace("ssd_fused_scan_chained");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
@@ -383,6 +405,7 @@ size_t ssd_sp_summary_workspace_bytes(const ssd_problem* p) {
 ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_a, const void* B,
                           const int32_t* seq_idx, float* loc, float* dec, int32_t* ids, void* workspace,
                           size_t workspace_bytes, void* stream) {
+    TraceRange trace("ssd_sp_summary");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !loc || !dec || !ids) return SSD_ERR_INVALID_ARG;
@@ -410,6 +433,7 @@ ssd_status ssd_sp_summary(const ssd_problem* p, const void* X, const float* log_
 
 ssd_status ssd_sp_combine(const ssd_problem* p, int nranks, int rank, const float* g_loc, const float* g_dec,
                           const int32_t* g_ids, const float* init_states, float* init_local, void* stream) {
+    TraceRange trace("ssd_sp_combine");
     ssd_status s = check_dims(p);
     if (s != SSD_OK) return s;
     if (nranks < 1 || rank < 0 || rank >= nranks) return SSD_ERR_INVALID_ARG;
@@ -423,6 +447,7 @@ ssd_status ssd_sp_combine(const ssd_problem* p, int nranks, int rank, const floa
 
 ssd_status ssd_sp_own_finals(const ssd_problem* p, int nranks, int rank, const int32_t* g_ids, float* final_states,
                              void* stream) {
+    TraceRange trace("ssd_sp_own_finals");
     ssd_status s = check_dims(p);
     if (s != SSD_OK) return s;
     if (nranks < 1 || rank < 0 || rank >= nranks) return SSD_ERR_INVALID_ARG;
@@ -436,6 +461,7 @@ ssd_status ssd_sp_own_finals(const ssd_problem* p, int nranks, int rank, const i
 
 ssd_status ssd_discretize(const ssd_problem* p, const float* dt, const float* dt_bias, const float* A,
                           const void* x, int zoh, float* log_a, void* X, void* stream) {
+    TraceRange trace("ssd_discretize");
     if (!p) return SSD_ERR_INVALID_ARG;
     if (p->batch < 1 || p->seqlen < 1 || p->nheads < 1 || p->headdim < 1) return SSD_ERR_INVALID_ARG;
     if (p->dtype != SSD_DTYPE_F32 && p->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
@@ -455,6 +481,7 @@ ssd_status ssd_discretize(const ssd_problem* p, const float* dt, const float* dt
 
 ssd_status ssd_decode_step(const ssd_problem* p, const void* x, const float* log_a, const void* B, const void* C,
                            const float* D, float* state, void* y, void* stream) {
+    TraceRange trace("ssd_decode_step");
     if (!p) return SSD_ERR_INVALID_ARG;
     if (p->batch < 1 || p->nheads < 1 || p->headdim < 1 || p->dstate < 1 || p->ngroups < 1 ||
         p->nheads % p->ngroups != 0)
@@ -476,6 +503,7 @@ ssd_status ssd_decode_step(const ssd_problem* p, const void* x, const float* log
 }
 
 ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs, void* stream) {
+    TraceRange trace("ssd_chunk_cumsum");
     ssd_status s = check_dims(p);  // log a only: nseq and seq_idx play no part here
     if (s != SSD_OK) return s;
     if (!log_a || !cs) return SSD_ERR_INVALID_ARG;
@@ -486,6 +514,7 @@ ssd_status ssd_chunk_cumsum(const ssd_problem* p, const float* log_a, float* cs,
 
 ssd_status ssd_chunk_state(const ssd_problem* p, const void* X, const void* B, const float* cs,
                            const int32_t* seq_idx, float* states, float* final_states, void* stream) {
+    TraceRange trace("ssd_chunk_state");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !B || !cs || !states) return SSD_ERR_INVALID_ARG;
@@ -499,6 +528,7 @@ ssd_status ssd_chunk_state(const ssd_problem* p, const void* X, const void* B, c
 ssd_status ssd_state_passing(const ssd_problem* p, const float* cs, const float* chunk_states, float* incoming,
                              const float* init_states, const int32_t* seq_idx, float* final_states,
                              void* stream) {
+    TraceRange trace("ssd_state_passing");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!cs || !chunk_states || !incoming) return SSD_ERR_INVALID_ARG;
@@ -512,6 +542,7 @@ ssd_status ssd_state_passing(const ssd_problem* p, const float* cs, const float*
 ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, const void* C, const float* cs,
                           const float* D, const float* incoming, const float* init_states,
                           const int32_t* seq_idx, void* Y, void* stream) {
+    TraceRange trace("ssd_chunk_scan");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !B || !C || !cs || !incoming || !Y) return SSD_ERR_INVALID_ARG;
@@ -526,6 +557,7 @@ ssd_status ssd_chunk_scan(const ssd_problem* p, const void* X, const void* B, co
 ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, const void* B, const void* C,
                    const float* D, const float* init_states, const int32_t* seq_idx, void* Y,
                    float* final_states, void* workspace, size_t workspace_bytes, void* stream) {
+    TraceRange trace("ssd_fwd");
     ssd_status s = check_common(p, seq_idx);
     if (s != SSD_OK) return s;
     if (!X || !log_a || !B || !C || !Y) return SSD_ERR_INVALID_ARG;
@@ -578,12 +610,23 @@ ssd_status ssd_fwd(const ssd_problem* p, const void* X, const float* log_a, cons
     // the SIMT kernels take the cumsum in fp64 (fp32 parity for strongly decaying heads);
     // state_passing works in place: the chunk states become the incoming states
     double* cs = reinterpret_cast<double*>(w);
-    if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess ||
-        (e = ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st)) !=
-            cudaSuccess ||
-        (e = ssd::launch_state_passing(d, cs, states, states, init_states, seq_idx, final_states, st)) !=
+    {
+        TraceRange r("chunk_cumsum");
+        if ((e = ssd::launch_chunk_cumsum(d, log_a, cs, st)) != cudaSuccess) return cuda_status(e);
+    }
+    {
+        TraceRange r("chunk_state");
+        if ((e = ssd::launch_chunk_state_simt(d, p->dtype, X, B, cs, seq_idx, states, final_states, st)) !=
             cudaSuccess)
-        return cuda_status(e);
+            return cuda_status(e);
+    }
+    {
+        TraceRange r("state_passing");
+        if ((e = ssd::launch_state_passing(d, cs, states, states, init_states, seq_idx, final_states, st)) !=
+            cudaSuccess)
+            return cuda_status(e);
+    }
+    TraceRange r("chunk_scan");
     return cuda_status(
         ssd::launch_chunk_scan_simt(d, p->dtype, X, B, C, cs, D, states, init_states, seq_idx, Y, st));
 }
