@@ -648,8 +648,11 @@ __device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const in
 // Y_off [256,384); the carried state H [384,512) (rows (head, p), N columns).
 // kAcc: a later state slice, whose epilogue adds its Y to the Y already there
 // (each thread reads the elements it then writes); a separate instantiation so
-// that the common case keeps its epilogue unchanged.
-template <int N, bool kAcc, bool kGen>
+// that the common case keeps its epilogue unchanged. kSeq: sequence ids are
+// given, and the prologue's chain over the pieces before a cut starts at the
+// last piece in which a sequence starts (also an instantiation of its own: the
+// kernel without ids keeps its code unchanged).
+template <int N, bool kAcc, bool kGen, bool kSeq>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, Dims d,
@@ -1163,7 +1166,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         griddep_wait();  // the range states come from the kernel before this one
                         waited = true;
                     }
-                    for (int l = 0; l < nl; ++l) {
+                    int l0 = 0;
+                    if constexpr (kSeq) {  // the pieces before the last sequence start drop out
+                        l0 = nl - 1;
+                        while (l0 > 0 && chain_cont[l0]) --l0;
+                    }
+                    for (int l = l0; l < nl; ++l) {
                         const int j = j0 + l;
                         const bool cont = chain_cont[l] != 0;
                         const float a = work_decay[(int64_t)j * 2 + sh];
@@ -1333,6 +1341,17 @@ cudaError_t set_smem_attr(K kernel, int bytes, int slot) {
     return ensure_smem_attr(reinterpret_cast<const void*>(kernel), bytes, slot);
 }
 
+// the scan instantiation for (accumulate into Y, general slot mapping, sequence ids)
+template <int N>
+auto scan_instance(bool acc, bool gen, bool sq) {
+    decltype(&fused_scan_kernel<N, false, false, false>) const k[2][2][2] = {
+        {{fused_scan_kernel<N, false, false, false>, fused_scan_kernel<N, false, false, true>},
+         {fused_scan_kernel<N, false, true, false>, fused_scan_kernel<N, false, true, true>}},
+        {{fused_scan_kernel<N, true, false, false>, fused_scan_kernel<N, true, false, true>},
+         {fused_scan_kernel<N, true, true, false>, fused_scan_kernel<N, true, true, true>}}};
+    return k[acc][gen][sq];
+}
+
 template <int N>
 int fused_smem_bytes() {
     return (int)FusedSmem<N>::oTail + 1024;
@@ -1489,17 +1508,16 @@ cudaError_t launch_fused_scan(const Dims& d, int64_t work_tiles, const void* X, 
     // the general slot mapping (headdim 128, or an odd number of heads per group) is
     // its own instantiation, so that the plain head pairs keep their code
     const bool gen = d.headdim != kP || d.heads_per_group % 2 != 0;
-    const int slot = (Yacc ? 2 : 0) + (gen ? 4 : 0);
+    const bool sq = seq_idx != nullptr;
+    const int slot = (Yacc ? 2 : 0) + (gen ? 4 : 0) + (sq ? 8 : 0);
     if (d.dstate == 64) {
-        auto k = gen ? (Yacc ? fused_scan_kernel<64, true, true> : fused_scan_kernel<64, false, true>)
-                     : (Yacc ? fused_scan_kernel<64, true, false> : fused_scan_kernel<64, false, false>);
+        auto k = scan_instance<64>(Yacc != nullptr, gen, sq);
         cfg.dynamicSmemBytes = fused_smem_bytes<64>();
         if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 40 + slot)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
                                final_states, work_local, work_decay, err);
     } else if (d.dstate == 128) {
-        auto k = gen ? (Yacc ? fused_scan_kernel<128, true, true> : fused_scan_kernel<128, false, true>)
-                     : (Yacc ? fused_scan_kernel<128, true, false> : fused_scan_kernel<128, false, false>);
+        auto k = scan_instance<128>(Yacc != nullptr, gen, sq);
         cfg.dynamicSmemBytes = fused_smem_bytes<128>();
         if ((e = set_smem_attr(k, (int)cfg.dynamicSmemBytes, 41 + slot)) != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k, mx, mb, mc, my, d, w, log_a, D, work_in, init_states, seq_idx, Yb,
