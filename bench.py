@@ -421,13 +421,15 @@ def run_ours(args, w):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize(dev)
 
-    for _ in range(args.warmup):
-        step()
-    barrier()
+    # the clock sampler starts first, so that the warm-up steps run right before
+    # the timed ones (an idle GPU lowers its clocks; the first timed step would
+    # pay for the ramp)
     clocks = ClockSampler(local) if rank == 0 and not args.no_clocks else None
     if clocks:
         clocks.start()
         time.sleep(0.3)
+    for _ in range(args.warmup):
+        step()
     evs_step = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     barrier()
     evs_step[0].record(stream)
