@@ -649,19 +649,22 @@ __device__ __forceinline__ void decay_walk(const Dims d, const Work wk, const in
 // kAcc: a later state slice, whose epilogue adds its Y to the Y already there
 // (each thread reads the elements it then writes); a separate instantiation so
 // that the common case keeps its epilogue unchanged. kSeq: sequence ids are
-// given, and the prologue's chain over the pieces before a cut starts at the
-// last piece in which a sequence starts (also an instantiation of its own: the
-// kernel without ids keeps its code unchanged).
+// given (the prologue's chain over the pieces before a cut then starts at the
+// last piece in which a sequence starts); without them every branch on the ids
+// folds away at compile time, which keeps the kernel's code (and so its
+// instruction fetch) smaller.
 template <int N, bool kAcc, bool kGen, bool kSeq>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, Dims d,
                       Work wk, const float* __restrict__ log_a, const float* __restrict__ Dv,
                       const float* __restrict__ work_in, const float* __restrict__ init_states,
-                      const int32_t* __restrict__ seq_idx, __nv_bfloat16* __restrict__ Y,
+                      const int32_t* __restrict__ seq_idx_arg, __nv_bfloat16* __restrict__ Y,
                       float* __restrict__ final_states, const float* __restrict__ work_local,
                       const float* __restrict__ work_decay, unsigned int* __restrict__ err) {
     using S = FusedSmem<N>;
+    // without sequence ids every branch on them folds away at compile time
+    const int32_t* __restrict__ seq_idx = kSeq ? seq_idx_arg : nullptr;
     constexpr int NQ = N / 4;  // state columns per thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
