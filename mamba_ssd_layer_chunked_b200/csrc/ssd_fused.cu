@@ -770,11 +770,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 if (t > 0) mbar_wait(&bar_yd, (t - 1) & 1);
                 tc_fence_after();
                 const uint32_t ba = stage_b(t);
+                // descriptors of later K steps: the start-address field plus the offset in 16-byte units
+                const uint64_t dc = smem_desc_sw128(ca, 16, 1024), db = smem_desc_sw128(ba, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                    mma_bf16_ss(tm_g, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ba + off, 16, 1024),
-                                idesc_nn, k > 0 ? 1u : 0u);
+                    const uint32_t off = ((k >> 2) * kBox + (k & 3) * 32) >> 4;
+                    mma_bf16_ss(tm_g, dc + off, db + off, idesc_nn, k > 0 ? 1u : 0u);
                 }
                 mma_commit(&bar_g);
                 // Y_diag(t) = (L o G)(t) X(t), A operand from TMEM, once L o G(t) is
@@ -782,13 +783,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 // Y_diag(t-1), and before state(t-1))
                 mbar_wait(&bar_lg, t & 1);
                 tc_fence_after();
-                const uint32_t xa = stage_x(t);
+                const uint64_t dx = smem_desc_sw128(stage_x(t), kBox, 1024);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 16 * k + 8 * hh,
-                                    smem_desc_sw128(xa + hh * kBox + k * 2048, kBox, 1024), idesc_ts, k > 0 ? 1u : 0u);
+                        mma_bf16_ts(tm_yd + 64 * hh, tm_lg + 16 * k + 8 * hh, dx + ((hh * kBox + k * 2048) >> 4), idesc_ts,
+                                    k > 0 ? 1u : 0u);
                 mma_commit(&bar_yd);
                 if (fin) break;
             }
@@ -805,11 +806,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 mbar_wait(&bar_c, par);
                 mbar_wait(&bar_st, par);
                 tc_fence_after();
+                const uint64_t dc = smem_desc_sw128(ca, 16, 1024), dh = smem_desc_sw128(ha, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                    mma_bf16_ss(tm_yo, smem_desc_sw128(ca + off, 16, 1024), smem_desc_sw128(ha + off, 16, 1024),
-                                idesc_nn, k > 0 ? 1u : 0u);
+                    const uint32_t off = ((k >> 2) * kBox + (k & 3) * 32) >> 4;
+                    mma_bf16_ss(tm_yo, dc + off, dh + off, idesc_nn, k > 0 ? 1u : 0u);
                 }
                 mma_commit(&bar_yo);
                 // epilogue(t) done: store Y(t) from the staging buffer; H += X'^T B
@@ -822,11 +823,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     if (valid_of(cur, 1)) tma_store_4d(&tm_y, Hs + kBox, p0_of(cur, 1), head_of(cur, 1), cur.ts, cur.b);
                     tma_store_commit();
                 }
-                const uint32_t xa = stage_x(t), ba = stage_b(t);
+                const uint64_t dx = smem_desc_sw128(stage_x(t), kBox, 1024), db = smem_desc_sw128(stage_b(t), kBox, 1024);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16_ss(tm_h, smem_desc_sw128(xa + k * 2048, kBox, 1024), smem_desc_sw128(ba + k * 2048, kBox, 1024),
-                                idesc_st, 1u);
+                for (int k = 0; k < 8; ++k) mma_bf16_ss(tm_h, dx + k * (2048 >> 4), db + k * (2048 >> 4), idesc_st, 1u);
                 mma_commit(&bar_s);
                 mma_commit(&bar_sfree[t & 1]);  // the B/X stage of tile t is free
                 if (full) tma_store_wait_read0();

@@ -36,7 +36,10 @@ __device__ __forceinline__ void wait_guard_init(unsigned int* err) {
     }
 }
 
-__device__ __forceinline__ void wait_report(unsigned int code) {
+// Out of line: it runs at most once per CTA, and every wait would otherwise
+// carry its code inline (the scan kernel's code size limits its instruction
+// fetch).
+static __device__ __noinline__ void wait_report(unsigned int code) {
     s_wait_gave_up = 1u;
     if (s_wait_err) atomicOr(s_wait_err, code);
 }
