@@ -855,26 +855,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 #pragma unroll
                 for (int q = 0; q < N / 64; ++q) tma_load_4d(Cs + q * kBox, &tm_c, &bar_c, 64 * q, g, td.ts, td.b);
             };
-            TileDesc nx = desc(0);
-            load_c(nx);
-            load_bx(nx, 0);
-            bool more = !(nx.flags & kTileFinal);
-            if (more) {
-                nx = desc(1);
-                load_bx(nx, 1);
-            }
-            for (int t = 0; more; ++t) {
-                // C(t+1) once G(t) and Y_off(t) have read C(t) (at t = 0 the
-                // initial state can release Y_off(0) before G(0) has run)
-                mbar_wait(&bar_g, t & 1);
-                mbar_wait(&bar_yo, t & 1);
-                load_c(nx);
-                more = !(nx.flags & kTileFinal);
-                if (!more) break;
-                // B, X of tile t+2 into tile t's stage once the tile state MMA has read it
-                nx = desc(t + 2);
-                mbar_wait(&bar_sfree[t & 1], (t >> 1) & 1);
-                load_bx(nx, t & 1);
+            // in issue order: C(0), B X(0), B X(1), C(1), B X(2), C(2), ...: B, X of
+            // tile u into stage u & 1 once the tile state MMA of tile u - 2 has
+            // read it; C(u) once G(u-1) and Y_off(u-1) have read C(u-1) (at u = 1
+            // the initial state can release Y_off(0) before G(0) has run)
+            load_c(desc(0));
+            for (int u = 0;; ++u) {
+                const TileDesc td = desc(u);
+                if (u >= 2) mbar_wait(&bar_sfree[u & 1], ((u - 2) >> 1) & 1);
+                load_bx(td, u & 1);
+                if (u >= 1) {
+                    mbar_wait(&bar_g, (u - 1) & 1);
+                    mbar_wait(&bar_yo, (u - 1) & 1);
+                    load_c(td);
+                }
+                if (td.flags & kTileFinal) break;
             }
         }
         __syncwarp();
