@@ -784,7 +784,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 mbar_wait(&bar_lg, t & 1);
                 tc_fence_after();
                 const uint64_t dx = smem_desc_sw128(stage_x(t), kBox, 1024);
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
@@ -815,9 +815,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 mma_commit(&bar_yo);
                 // epilogue(t) done: store Y(t) from the staging buffer; H += X'^T B
                 mbar_wait(&bar_epi, par);
-                const TileDesc cur = desc(t);
+                // tile t's descriptor was published before epilogue(t) began; its
+                // buffer is refilled only after state(t), which needs bar_free below,
+                // so every field is read before that arrival
+                const TileDesc& cur = csb[t & (kCsBufs - 1)].td;
                 tc_fence_after();
                 const bool full = cur.v == 128;
+                const bool last = (cur.flags & kTileFinal) != 0;
                 if (full) {
                     tma_store_4d(&tm_y, Hs, p0_of(cur, 0), head_of(cur, 0), cur.ts, cur.b);
                     if (valid_of(cur, 1)) tma_store_4d(&tm_y, Hs + kBox, p0_of(cur, 1), head_of(cur, 1), cur.ts, cur.b);
@@ -830,7 +834,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 mma_commit(&bar_sfree[t & 1]);  // the B/X stage of tile t is free
                 if (full) tma_store_wait_read0();
                 mbar_arrive(&bar_free);
-                if (cur.flags & kTileFinal) break;
+                if (last) break;
             }
             tma_store_wait0();
         }
