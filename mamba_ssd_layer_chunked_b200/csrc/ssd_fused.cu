@@ -344,6 +344,7 @@ __global__ void __launch_bounds__(kSegThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    wait_guard_finish();
     if (warp == 0) tmem_dealloc(tacc, N);
 }
 
@@ -1327,6 +1328,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    wait_guard_finish();
     if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
 

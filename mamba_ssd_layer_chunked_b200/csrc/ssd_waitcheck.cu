@@ -1,8 +1,8 @@
 // ssd_waitcheck.cu -- a self-test of the bounded waits' failure report.
 //
 // The tensor-core kernels wait on shared-memory barriers; each wait gives up
-// after a time limit, sets a bit in the library's device error word and lets
-// its CTA run to its end (tc_ptx.cuh). This kernel makes that happen on
+// after a time limit and lets its CTA run to its end, which then sets a bit in
+// the library's device error word (tc_ptx.cuh). This kernel makes that happen on
 // purpose, with a short limit, on a barrier that nothing ever completes, so
 // that a test can check the report reaches the host (ssd_device_error) and is
 // cleared, and that the device stays usable. It issues no copies and no
@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(32) wait_timeout_kernel(uint64_t limit_ns, uns
         if (!mbar_wait(&bar, 0, limit_ns)) mbar_wait(&bar, 0, limit_ns);
     }
     __syncthreads();
+    wait_guard_finish();
 }
 
 }  // namespace

@@ -15,9 +15,11 @@ namespace tc {
 // Bounded waits and their error report. Every kernel that waits on an
 // mbarrier calls wait_guard_init(err) on entry, before its first
 // __syncthreads, with err the library's device error word (one 32-bit word per
-// device, read and cleared by ssd_device_error on the host). A wait that gives
-// up ORs its code into that word, marks its CTA, and returns false; the kernel
-// then runs to its end without trapping or hanging, and its output is invalid.
+// device, read and cleared by ssd_device_error on the host), and
+// wait_guard_finish() after its last __syncthreads. A wait that gives up marks
+// its CTA and returns false; the kernel then runs to its end without trapping
+// or hanging, its output is invalid, and at its end the CTA ORs the timeout
+// code into that word.
 // Later waits of the same CTA give up at once, so a CTA that lost its schedule
 // still ends within one wait limit; the mark lives in shared memory, so it ends
 // with the launch and never touches later launches.
@@ -36,12 +38,15 @@ __device__ __forceinline__ void wait_guard_init(unsigned int* err) {
     }
 }
 
-// Out of line: it runs at most once per CTA, and every wait would otherwise
-// carry its code inline (the scan kernel's code size limits its instruction
-// fetch).
-static __device__ __noinline__ void wait_report(unsigned int code) {
-    s_wait_gave_up = 1u;
-    if (s_wait_err) atomicOr(s_wait_err, code);
+// A wait that gives up only marks its CTA: the CTA's thread 0 ORs the code
+// into the device error word when the kernel ends (wait_guard_finish), so a
+// wait carries no call and no global atomic (the scan kernel's code size limits
+// its instruction fetch, and a call at its register cap spills).
+__device__ __forceinline__ void wait_report() { s_wait_gave_up = 1u; }
+
+// After the kernel's last __syncthreads (every wait of the CTA is behind it).
+__device__ __forceinline__ void wait_guard_finish() {
+    if (threadIdx.x == 0 && s_wait_gave_up != 0u && s_wait_err) atomicOr(s_wait_err, kErrBarrierTimeout);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -93,7 +98,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
         if ((it & 63u) == 0u) {  // the clock and the CTA's mark are read rarely
             if (*reinterpret_cast<volatile unsigned int*>(&s_wait_gave_up) != 0u) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
-                wait_report(kErrBarrierTimeout);
+                wait_report();
                 return false;
             }
         }
