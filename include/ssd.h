@@ -118,9 +118,9 @@ const char* ssd_last_cuda_error_string(void);
  * ssd_device_error: the failure report of the kernels' bounded waits. The
  * tensor-core kernels wait on shared-memory barriers for their copies and
  * matrix products; every such wait is bounded (about 2 s), and a wait that
- * gives up sets a bit in a device-wide 32-bit error word, after which its CTA
- * runs to its end without hanging or faulting: the outputs of that call are
- * then INVALID, although the call itself returned SSD_OK (the library does not
+ * gives up lets its CTA run to its end without hanging or faulting, where the
+ * CTA sets a bit in a device-wide 32-bit error word: the outputs of that call
+ * are then INVALID, although the call itself returned SSD_OK (the library does not
  * synchronise, so the launch cannot see it). The word is per device and shared
  * by every call and stream since it was last cleared.
  * This entry point enqueues a read of the word on `stream`, then its clearing,
