@@ -1006,20 +1006,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     const HeadF f = {rowf_s[hh][tid], rowf_s[2 + hh][tid], cs.c[hh][k],
                                      Dv ? Dv[head_of(cs.td, hh)] : 0.f};
                     uint32_t w0[8], w1[8];
+                    full_block(f, hh, 0, gw, w0);  // column block 0: full below the diagonal pair
                     if (cq == q4) {
                         // lane half hi's diagonal block is column block hi; block 0
                         // is full for half 1, block 1 zero for half 0: one pass for
                         // both halves, no divergence
-                        uint32_t dw[8], fw[8];
+                        uint32_t dw[8];
                         diag_block(cs, f, hh, rb, gw, gw + 16, hi != 0, dw);
-                        full_block(f, hh, 0, gw, fw);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            w0[e] = hi ? fw[e] : dw[e];
                             w1[e] = hi ? dw[e] : 0u;
+                            w0[e] = hi ? w0[e] : dw[e];
                         }
                     } else {
-                        full_block(f, hh, 0, gw, w0);
                         full_block(f, hh, 1, gw + 16, w1);
                     }
                     tmem_st8(tcol + 8 * hh, w0);       // column block 2 cq, head hh
@@ -1231,7 +1230,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const int64_t yoff = ((rowt + cur.ts + k) * d.nheads + head_of(cur, eh)) * (int64_t)P +
                                      p0_of(cur, eh) + p0;
                 __nv_bfloat16* yrow = Y + yoff;
-#pragma unroll
+#pragma unroll 1
                 for (int hf = 0; hf < 2; ++hf) {
                     // a later state slice: the Y this thread's outputs add to
                     uint4 ya[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
